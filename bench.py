@@ -1,0 +1,409 @@
+"""Benchmark of the VDN hybrid video-video attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload 768p-bf16]
+
+A step is one vdn_hybrid_attn_fwd call (window softmax + VDA scans + readout,
+norm, gates) over one 768p-like layer input (B=1, H=40, d=128, F=36 frames of
+48 x 84 tokens, chunks of 5, 512 text tokens) resident in HBM. Inputs are
+larger than L2 (each video tensor is 1.49 GB), so L2 is not flushed.
+
+For N > 1 (launched by torchrun) every rank runs its own independent layer
+input (weak scaling, no collective in the data path); the timed region is
+bracketed by a barrier and device synchronisation on every rank and the
+reported time is the maximum over ranks.
+
+Printed on rank 0: one JSON line with the throughput (video tokens/s over all
+ranks), the roofline of the dominant kernel (window softmax, tensor-core bound),
+the end-to-end figure through the public call with host buffers, the CPU
+oracle baseline on a bounded sample, and the SM clocks seen during timing.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "hybrid-attn fwd video tokens/s on 1 B200 (768p-like); % of TC/HBM roofline"
+UNIT = "video tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------ algorithmic work
+
+def window_pairs(lay) -> int:
+    """Allowed (query, key) pairs of one (b, h): every query token of frame f sees
+    the tokens of its window + anchor frames and all text tokens."""
+    F, N, T, c = lay.F, lay.N, lay.T, lay.c
+    total = 0
+    for f in range(F):
+        if f == 0 or f == F - 1:
+            frames = F
+        else:
+            j = f // c
+            lo, hi = max(0, c * (j - 1)), min(F - 1, c * (j + 2) - 1)
+            frames = hi - lo + 1 + (1 if lo > 0 else 0) + (1 if hi < F - 1 else 0)
+        total += N * (frames * N + T)
+    return total
+
+
+def window_flops(lay) -> float:
+    """4 d flops per allowed pair (q.k and p.v), all heads and batches."""
+    return 4.0 * lay.d * window_pairs(lay) * lay.H * lay.B
+
+
+def launches_per_step(lay) -> int:
+    """Kernels of one vdn_hybrid_attn_fwd call: window softmax, gram, inverse,
+    scan, zero-fill of unused chunk entries, readout/combine."""
+    return 6
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during timing."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self):
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self, gpu_indices):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                idx = int(p[0])
+            except ValueError:
+                continue
+            if gpu_indices is not None and idx not in gpu_indices:
+                continue
+            try:
+                sm.append(float(p[1]))
+                smax.append(float(p[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, p[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [x for x in sm if x > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- helpers
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def window_kernel_traffic(lay):
+    """Per-launch DRAM bytes of the window-softmax kernel from the committed ncu
+    summary, scaled to this workload; None when the summary is missing or was
+    taken on a different kernel source."""
+    p = os.path.join(ROOT, "profiles", "window_tc_traffic.txt")
+    src = os.path.join(ROOT, "linear_attention_video_block_b200", "csrc", "window_tc.cu")
+    if not os.path.exists(p) or not os.path.exists(src):
+        return None
+    kv = {}
+    for line in open(p):
+        if "=" in line and not line.startswith("#"):
+            a, b = line.split("=", 1)
+            kv[a.strip()] = b.strip()
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if kv.get("source_sha256_16") != digest:
+        return None
+    try:
+        bytes_per_pair = float(kv["dram_bytes_per_allowed_pair_head"])
+    except (KeyError, ValueError):
+        return None
+    return bytes_per_pair * window_pairs(lay) * lay.H * lay.B
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(lay, dtype, seed, rows_per_frame):
+    """Times the float64 oracle on a bounded sample of the workload: one head
+    drawn with the workload's recipe, the whole linear branch of that head, and
+    the softmax branch, norm and gates on `rows_per_frame` query rows of every
+    frame. Returns (extrapolated video tokens/s for the whole workload, seconds,
+    description)."""
+    import numpy as np
+    from linear_attention_video_block_b200.synth import Layout, make_inputs
+    from oracle import vdn_oracle as O
+
+    one = Layout(B=1, F=lay.F, N=lay.N, T=lay.T, c=lay.c, H=1, d=lay.d)
+    inp = make_inputs(one, dtype, seed)
+    a = {k: v.double().numpy() for k, v in inp.items()}
+    rng = np.random.default_rng(0)
+    rows = np.sort(np.concatenate([f * lay.N + rng.choice(lay.N, rows_per_frame, replace=False)
+                                   for f in range(lay.F)]))
+    t0 = time.perf_counter()
+    o_lin = O.linear_branch(a["q"], a["k"], a["v"], a["k_text"], a["v_text"], a["beta"],
+                            a["beta_text"], lay.F, lay.N, lay.c)
+    t1 = time.perf_counter()
+    o_soft = O.softmax_branch(a["q"], a["k"], a["v"], a["k_text"], a["v_text"], lay.F, lay.N,
+                              lay.c, rows=rows)
+    O.combine(o_soft[:, rows], o_lin[:, rows], a["g_s"][:, rows], a["g_l"][:, rows])
+    t2 = time.perf_counter()
+    per_head = (t1 - t0) + (t2 - t1) * (lay.L / len(rows))
+    est = per_head * lay.H * lay.B
+    desc = (f"1 of {lay.H} heads drawn with the same recipe; linear branch in full, softmax + "
+            f"gates on {rows_per_frame} query rows per frame ({len(rows)} of {lay.L}); "
+            f"extrapolated linearly to all rows and heads")
+    return lay.L * lay.B / est, t2 - t0, desc
+
+
+# ---------------------------------------------------------------- arms
+
+def run_reference(args, rank, world):
+    """The oracle as it stands, timed on the host cores (rank 0 only)."""
+    from linear_attention_video_block_b200.synth import WORKLOADS
+    if rank != 0:
+        return
+    lay, dtype, seed = WORKLOADS[args.workload]
+    rpf = args.ref_rows
+    for _ in range(args.warmup):
+        oracle_sample(lay, dtype, seed, rpf)
+    vals, secs = [], []
+    desc = ""
+    for _ in range(args.steps):
+        v, s, desc = oracle_sample(lay, dtype, seed, rpf)
+        vals.append(v)
+        secs.append(s)
+    value = statistics.median(vals)
+    cores = cpu_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * lay.L * lay.B / value, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(args.workload, lay),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(name, lay):
+    return {"workload": name, "B": lay.B, "F": lay.F, "N": lay.N, "T": lay.T, "c": lay.c,
+            "H": lay.H, "d": lay.d, "video_tokens": lay.L * lay.B,
+            "l2": "inputs larger than L2 (1.49 GB per video tensor); no flush",
+            "parallelism": "independent problem per GPU (weak scaling)"}
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from linear_attention_video_block_b200 import vdn
+    from linear_attention_video_block_b200.synth import WORKLOADS, make_inputs
+
+    lay, dtype, seed = WORKLOADS[args.workload]
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    inp = make_inputs(lay, dtype, seed + rank, device=str(dev))
+    ws = torch.empty(vdn.workspace_bytes(lay, inp["q"].dtype), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(inp["q"])
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        vdn.hybrid_attn_fwd(lay, inp["q"], inp["k"], inp["v"], inp["k_text"], inp["v_text"],
+                            inp["beta"], inp["beta_text"], inp["g_s"], inp["g_l"], out=out,
+                            workspace=ws)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert vdn.device_status() == 0, "device status set during warm-up"
+
+    clocks = ClockSampler()
+    if rank == 0:
+        clocks.start()
+        time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms = e0.elapsed_time(e1) / args.steps
+
+    # The dominant kernel alone: the window-softmax launch of the same
+    # configuration, timed over the same number of launches.
+    o_soft = torch.empty_like(inp["q"])
+    for _ in range(2):
+        vdn.window_softmax_fwd(lay, inp["q"], inp["k"], inp["v"], inp["k_text"], inp["v_text"],
+                               o_soft=o_soft)
+    torch.cuda.synchronize(dev)
+    w0 = torch.cuda.Event(enable_timing=True)
+    w1 = torch.cuda.Event(enable_timing=True)
+    w0.record(stream)
+    for _ in range(args.steps):
+        vdn.window_softmax_fwd(lay, inp["q"], inp["k"], inp["v"], inp["k_text"], inp["v_text"],
+                               o_soft=o_soft)
+    w1.record(stream)
+    torch.cuda.synchronize(dev)
+    win_ms = w0.elapsed_time(w1) / args.steps
+    clk = clocks.stop(None) if rank == 0 else None
+
+    # End to end through the public call with pinned host buffers: every step
+    # copies the inputs in and the output back.
+    host = {k: v.cpu().pin_memory() for k, v in inp.items()}
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+
+    def e2e_step():
+        vdn.hybrid_attn_fwd(lay, host["q"], host["k"], host["v"], host["k_text"], host["v_text"],
+                            host["beta"], host["beta_text"], host["g_s"], host["g_l"], out=out_h,
+                            workspace=ws, device=str(dev))
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    e2e_steps = max(1, min(args.steps, 5))
+    barrier()
+    x0 = torch.cuda.Event(enable_timing=True)
+    x1 = torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    x1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = x0.elapsed_time(x1) / e2e_steps
+    assert vdn.device_status() == 0, "device status set during timing"
+
+    if world > 1:
+        t = torch.tensor([ms, win_ms, e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, win_ms, e2e_ms = t.tolist()
+    if rank != 0:
+        return
+    tokens = lay.L * lay.B * world
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    flops = window_flops(lay)
+    achieved = flops / (win_ms * 1e-3) / 1e12
+    traffic = window_kernel_traffic(lay)
+    cpu_val, cpu_s, cpu_desc = oracle_sample(lay, dtype, seed, args.ref_rows)
+    line = {
+        "impl": "ours", "metric": METRIC, "value": tokens / (ms * 1e-3), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dtype,
+        "data": "synthetic (seeded: q, v, gates ~ N(0,1); k ~ N(0,1) L2-normalised; "
+                "beta = sigmoid(N(0,1)))",
+        "config": config_of(args.workload, lay),
+        "roofline": {"bound": "tensor", "kernel": "window softmax (tcgen05)",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{peak_kind} bf16 dense (burst)",
+                     "flops_per_launch": flops, "launch_ms": win_ms,
+                     "share_of_step": win_ms / ms},
+        "cpu_baseline": {"value": cpu_val, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                         "sample": cpu_desc, "seconds": cpu_s},
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps},
+        "clocks": clk,
+        "gpu_launches": launches_per_step(lay) * args.steps * world,
+        "when": datetime.datetime.now(datetime.timezone.utc).isoformat(timespec="seconds"),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="768p-bf16")
+    ap.add_argument("--ref-rows", type=int, default=16,
+                    help="query rows per frame in the oracle's bounded sample")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

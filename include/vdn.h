@@ -1,0 +1,142 @@
+/*
+ * vdn.h - C ABI of libvdn: the Video DeltaNet hybrid video-video attention
+ * forward on NVIDIA B200 (sm_100a).
+ *
+ * The operation (sources: the project page "Video DeltaNet: Near-Lossless
+ * Hybrid Attention for Video Models", sections "Local Softmax and Long-Range
+ * Linear Memory", "Gating the Softmax and Linear Branch Outputs" and "Video
+ * Delta Attention: A Frame-Wise Solution"; and "Faster Than It Plays", section
+ * "Two branches instead of one", for the closed form S = (S_bar + B)(I + A)^-1):
+ *
+ *   softmax branch  o_soft = softmax(q K^T / sqrt(d)) V over the key set of the
+ *                   query's frame: the frames of its chunk and of the two
+ *                   neighbouring chunks, the boundary frames 0 and F-1, and all
+ *                   T text tokens (one normaliser). Boundary-frame queries see
+ *                   every frame.
+ *   linear branch   Video Delta Attention: per frame, A = K^T Diag(beta) K,
+ *                   B = V^T Diag(beta) K, S <- (S + B)(I + A)^-1; a forward scan
+ *                   over frames 1, 2, ... and a reverse scan over F-2, F-3, ...,
+ *                   both starting from S0 = 1/2 B_T (I + A_T)^-1 (the text
+ *                   written once into a zero state, halved). A non-boundary
+ *                   frame whose window is frames [lo, hi] reads the forward
+ *                   state after frames 1..lo-1 and the reverse state after
+ *                   frames F-2..hi+1 (S0 where empty): o_lin = (S_fwd + S_rev) q.
+ *                   Boundary frames (0 and F-1) are never scanned and have
+ *                   o_lin = 0.
+ *   combine         out = sigmoid(g_s) * o_soft + sigmoid(g_l) * RMSNorm_d(o_lin)
+ *                   (element-wise gates; RMSNorm over the head dim with eps and
+ *                   an optional weight).
+ *
+ * Layout. Chunk of frame f: ch(f) = f / c (integer division; the last chunk is
+ * partial when c does not divide F). L = F * N video tokens, token index
+ * f * N + n (frame-major). All tensors are dense, row-major:
+ *   q, k, v, g_soft, g_lin, out, out_soft, out_lin, o_soft, o_lin : [B, L, H, d]
+ *   k_text, v_text                                                 : [B, T, H, d]
+ *   beta  : [B, L, H] float32      beta_text : [B, T, H] float32
+ *   lse   : [B, L, H] float32 (natural-log normaliser of the softmax branch)
+ *   chunk_states : [B, H, 2, J, d, d] float32, J = ceil(F / c); [.., 0, j] is the
+ *                  forward and [.., 1, j] the reverse state read by chunk j
+ *                  (row index = value dim, column = key dim). Entries of chunks
+ *                  that hold no non-boundary frame are zero.
+ * Tensors of element type vdn_dtype_t are float32 (VDN_F32) or bfloat16
+ * (VDN_BF16); accumulation, softmax statistics and VDA states are float32.
+ * Inputs are used as given: the library does not normalise k or rescale q.
+ *
+ * Supported: VDN_F32 with d in {16, 32, 64, 128}; VDN_BF16 with d in {64, 128}.
+ * T may be 0 (k_text, v_text, beta_text may then be NULL).
+ *
+ * Ownership and execution. Every pointer is caller-owned device memory, except
+ * the layout struct which is read on the host during the call. The library
+ * allocates no memory and keeps no state between calls besides a device-side
+ * status word (vdn_device_status). Calls are asynchronous on `stream`;
+ * the return code reports host-detectable errors (VDN_ERR_INVALID for a bad
+ * layout or a NULL required pointer, VDN_ERR_UNSUPPORTED for a dtype/d
+ * combination not built or a pointer not 16-byte aligned, VDN_ERR_WORKSPACE
+ * for a short workspace) and launch errors (VDN_ERR_CUDA). On any error
+ * nothing is launched, except for VDN_ERR_CUDA where kernels launched before
+ * the failing one may run.
+ */
+#ifndef VDN_H_
+#define VDN_H_
+
+#include <stddef.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct {
+  int B;  /* batch */
+  int F;  /* latent frames */
+  int N;  /* video tokens per frame */
+  int T;  /* text tokens */
+  int c;  /* frames per chunk */
+  int H;  /* heads */
+  int d;  /* head dim (shared by q, k, v) */
+} vdn_layout_t;
+
+typedef enum { VDN_F32 = 0, VDN_BF16 = 1 } vdn_dtype_t;
+
+typedef enum {
+  VDN_OK = 0,
+  VDN_ERR_INVALID = 1,
+  VDN_ERR_UNSUPPORTED = 2,
+  VDN_ERR_WORKSPACE = 3,
+  VDN_ERR_CUDA = 4,
+  VDN_ERR_TIMEOUT = 5
+} vdn_status_t;
+
+/* Bytes of device workspace that vdn_vda_scan_fwd and vdn_hybrid_attn_fwd need
+ * for this layout and dtype (the maximum of the two). 0 for an invalid layout. */
+size_t vdn_workspace_bytes(const vdn_layout_t* layout, int dtype);
+
+/* Softmax branch alone (project page, "Local Softmax and Long-Range Linear
+ * Memory"): o_soft = softmax over the window + anchor frames + text keys,
+ * ungated. lse (nullable) receives the natural-log normaliser per query. */
+int vdn_window_softmax_fwd(const vdn_layout_t* layout, int dtype,
+                           const void* q, const void* k, const void* v,
+                           const void* k_text, const void* v_text,
+                           void* o_soft, float* lse, cudaStream_t stream);
+
+/* Linear branch alone (project page, "Video Delta Attention: A Frame-Wise
+ * Solution"; "Faster Than It Plays", closed form): frame Gram matrices, the
+ * two scans from the half-weight text state, and the readout o_lin =
+ * (S_fwd + S_rev) q, ungated and before RMSNorm (0 for boundary frames).
+ * chunk_states (nullable) receives the per-chunk read states. */
+int vdn_vda_scan_fwd(const vdn_layout_t* layout, int dtype,
+                     const void* q, const void* k, const void* v,
+                     const void* k_text, const void* v_text,
+                     const float* beta, const float* beta_text,
+                     void* o_lin, float* chunk_states,
+                     void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* The whole hybrid forward (project page, sections "Local Softmax ..." and
+ * "Gating the Softmax and Linear Branch Outputs"): out = sigmoid(g_soft) *
+ * o_soft + sigmoid(g_lin) * RMSNorm(o_lin). rms_weight (nullable, [d] float32)
+ * defaults to ones. out_soft and out_lin (nullable) receive the two gated
+ * branches separately (out = out_soft + out_lin), for callers that apply a
+ * separate output projection per branch. */
+int vdn_hybrid_attn_fwd(const vdn_layout_t* layout, int dtype,
+                        const void* q, const void* k, const void* v,
+                        const void* k_text, const void* v_text,
+                        const float* beta, const float* beta_text,
+                        const void* g_soft, const void* g_lin,
+                        const float* rms_weight, float rms_eps,
+                        void* out, void* out_soft, void* out_lin,
+                        void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Reads and clears the device-side status word on the current device
+ * (synchronises the device). VDN_ERR_TIMEOUT means a kernel gave up a bounded
+ * wait and returned without finishing its tile; the outputs of that call are
+ * then undefined. Returns VDN_ERR_CUDA if the status cannot be read. */
+int vdn_device_status(void);
+
+/* Static string for a status code. */
+const char* vdn_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VDN_H_ */

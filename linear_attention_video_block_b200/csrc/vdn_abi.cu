@@ -1,0 +1,179 @@
+// libvdn C ABI: argument checks, workspace carving and launch sequencing on
+// the caller's stream. Every step of the operation runs in the kernels of this
+// library; the host code only validates and launches.
+#include <cstdint>
+
+#include "vdn_internal.cuh"
+
+namespace {
+
+using vdn::Layout;
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+size_t esize(int dtype) { return dtype == VDN_BF16 ? 2 : 4; }
+
+bool layout_ok(const vdn_layout_t* l) {
+  if (!l) return false;
+  if (l->B < 1 || l->F < 1 || l->N < 1 || l->T < 0 || l->c < 1 || l->H < 1 || l->d < 1) return false;
+  // token offsets and TMA coordinates are 32-bit signed per dimension
+  long long L = (long long)l->F * l->N;
+  if (L > (1LL << 30) || l->T > (1 << 30)) return false;
+  if ((long long)l->B * L * l->H * l->d > (1LL << 46)) return false;
+  return true;
+}
+
+bool dtype_d_ok(int dtype, int d) {
+  if (dtype == VDN_F32) return d == 16 || d == 32 || d == 64 || d == 128;
+  if (dtype == VDN_BF16) return d == 64 || d == 128;
+  return false;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+Layout to_layout(const vdn_layout_t* l) {
+  Layout x;
+  x.B = l->B; x.F = l->F; x.N = l->N; x.T = l->T; x.c = l->c; x.H = l->H; x.d = l->d;
+  return x;
+}
+
+struct Workspace {
+  float* am = nullptr;
+  float* bw = nullptr;
+  float* states = nullptr;
+  void* o_soft = nullptr;
+  size_t bytes = 0;
+};
+
+// Carves the workspace; with base == nullptr only computes the size.
+Workspace carve(const Layout& l, int dtype, void* base, bool need_states, bool need_osoft) {
+  Workspace w;
+  const size_t dd = (size_t)l.d * l.d;
+  const size_t bh = (size_t)l.B * l.H;
+  char* p = static_cast<char*>(base);
+  size_t off = 0;
+  auto take = [&](size_t n) -> void* {
+    void* r = p ? p + off : nullptr;
+    off = align_up(off + n);
+    return r;
+  };
+  w.am = static_cast<float*>(take(bh * l.F * dd * sizeof(float)));
+  w.bw = static_cast<float*>(take(bh * l.F * dd * sizeof(float)));
+  if (need_states) w.states = static_cast<float*>(take(bh * 2 * l.J() * dd * sizeof(float)));
+  if (need_osoft) w.o_soft = take((size_t)l.B * l.L() * l.H * l.d * esize(dtype));
+  w.bytes = off;
+  return w;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? VDN_OK : VDN_ERR_CUDA; }
+
+int run_window(const Layout& l, int dtype, const void* q, const void* k, const void* v,
+               const void* kt, const void* vt, void* o, float* lse, cudaStream_t st) {
+  if (vdn::window_tc_supported(l, dtype))
+    return cuda_status(vdn::launch_window_tc(l, q, k, v, kt, vt, o, lse, st));
+  return cuda_status(vdn::launch_window_simt(l, dtype, q, k, v, kt, vt, o, lse, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t vdn_workspace_bytes(const vdn_layout_t* layout, int dtype) {
+  if (!layout_ok(layout) || !dtype_d_ok(dtype, layout->d)) return 0;
+  return carve(to_layout(layout), dtype, nullptr, true, true).bytes;
+}
+
+int vdn_window_softmax_fwd(const vdn_layout_t* layout, int dtype, const void* q, const void* k,
+                           const void* v, const void* k_text, const void* v_text, void* o_soft,
+                           float* lse, cudaStream_t stream) {
+  if (!layout_ok(layout)) return VDN_ERR_INVALID;
+  if (!dtype_d_ok(dtype, layout->d)) return VDN_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !o_soft) return VDN_ERR_INVALID;
+  if (layout->T > 0 && (!k_text || !v_text)) return VDN_ERR_INVALID;
+  const void* ptrs[] = {q, k, v, o_soft, lse};
+  for (const void* p : ptrs) if (p && !aligned16(p)) return VDN_ERR_UNSUPPORTED;
+  if (layout->T > 0 && (!aligned16(k_text) || !aligned16(v_text))) return VDN_ERR_UNSUPPORTED;
+  const Layout l = to_layout(layout);
+  return run_window(l, dtype, q, k, v, layout->T ? k_text : nullptr,
+                    layout->T ? v_text : nullptr, o_soft, lse, stream);
+}
+
+int vdn_vda_scan_fwd(const vdn_layout_t* layout, int dtype, const void* q, const void* k,
+                     const void* v, const void* k_text, const void* v_text, const float* beta,
+                     const float* beta_text, void* o_lin, float* chunk_states, void* workspace,
+                     size_t workspace_bytes, cudaStream_t stream) {
+  if (!layout_ok(layout)) return VDN_ERR_INVALID;
+  if (!dtype_d_ok(dtype, layout->d)) return VDN_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !beta || !o_lin) return VDN_ERR_INVALID;
+  if (layout->T > 0 && (!k_text || !v_text || !beta_text)) return VDN_ERR_INVALID;
+  const void* ptrs[] = {q, k, v, beta, o_lin, chunk_states, workspace};
+  for (const void* p : ptrs) if (p && !aligned16(p)) return VDN_ERR_UNSUPPORTED;
+  if (layout->T > 0 && (!aligned16(k_text) || !aligned16(v_text) || !aligned16(beta_text)))
+    return VDN_ERR_UNSUPPORTED;
+  const Layout l = to_layout(layout);
+  const bool own_states = chunk_states == nullptr;
+  const Workspace need = carve(l, dtype, nullptr, own_states, false);
+  if (!workspace || workspace_bytes < need.bytes) return VDN_ERR_WORKSPACE;
+  const Workspace w = carve(l, dtype, workspace, own_states, false);
+  float* states = own_states ? w.states : chunk_states;
+  const void* kt = layout->T ? k_text : nullptr;
+  const void* vt = layout->T ? v_text : nullptr;
+  const float* bt = layout->T ? beta_text : nullptr;
+  int s = cuda_status(vdn::launch_vda_states(l, dtype, k, v, kt, vt, beta, bt, w.am, w.bw, states, stream));
+  if (s != VDN_OK) return s;
+  return cuda_status(vdn::launch_readout(l, dtype, 0, q, states, nullptr, nullptr, nullptr, nullptr,
+                                         0.f, o_lin, nullptr, nullptr, stream));
+}
+
+int vdn_hybrid_attn_fwd(const vdn_layout_t* layout, int dtype, const void* q, const void* k,
+                        const void* v, const void* k_text, const void* v_text, const float* beta,
+                        const float* beta_text, const void* g_soft, const void* g_lin,
+                        const float* rms_weight, float rms_eps, void* out, void* out_soft,
+                        void* out_lin, void* workspace, size_t workspace_bytes,
+                        cudaStream_t stream) {
+  if (!layout_ok(layout)) return VDN_ERR_INVALID;
+  if (!dtype_d_ok(dtype, layout->d)) return VDN_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !beta || !g_soft || !g_lin || !out) return VDN_ERR_INVALID;
+  if (layout->T > 0 && (!k_text || !v_text || !beta_text)) return VDN_ERR_INVALID;
+  if (!(rms_eps >= 0.f)) return VDN_ERR_INVALID;
+  const void* ptrs[] = {q, k, v, beta, g_soft, g_lin, rms_weight, out, out_soft, out_lin, workspace};
+  for (const void* p : ptrs) if (p && !aligned16(p)) return VDN_ERR_UNSUPPORTED;
+  if (layout->T > 0 && (!aligned16(k_text) || !aligned16(v_text) || !aligned16(beta_text)))
+    return VDN_ERR_UNSUPPORTED;
+  const Layout l = to_layout(layout);
+  const Workspace need = carve(l, dtype, nullptr, true, true);
+  if (!workspace || workspace_bytes < need.bytes) return VDN_ERR_WORKSPACE;
+  const Workspace w = carve(l, dtype, workspace, true, true);
+  const void* kt = layout->T ? k_text : nullptr;
+  const void* vt = layout->T ? v_text : nullptr;
+  const float* bt = layout->T ? beta_text : nullptr;
+  int s = run_window(l, dtype, q, k, v, kt, vt, w.o_soft, nullptr, stream);
+  if (s != VDN_OK) return s;
+  s = cuda_status(vdn::launch_vda_states(l, dtype, k, v, kt, vt, beta, bt, w.am, w.bw, w.states, stream));
+  if (s != VDN_OK) return s;
+  return cuda_status(vdn::launch_readout(l, dtype, 1, q, w.states, w.o_soft, g_soft, g_lin,
+                                         rms_weight, rms_eps, out, out_soft, out_lin, stream));
+}
+
+int vdn_device_status(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return VDN_ERR_CUDA;
+  int s = 0;
+  if (vdn::read_and_clear_tc_status(&s) != cudaSuccess) return VDN_ERR_CUDA;
+  return s;
+}
+
+const char* vdn_status_string(int status) {
+  switch (status) {
+    case VDN_OK: return "ok";
+    case VDN_ERR_INVALID: return "invalid argument (layout or required pointer)";
+    case VDN_ERR_UNSUPPORTED: return "unsupported dtype/head dim or misaligned pointer";
+    case VDN_ERR_WORKSPACE: return "workspace missing or too small";
+    case VDN_ERR_CUDA: return "CUDA error";
+    case VDN_ERR_TIMEOUT: return "a kernel gave up a bounded wait";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

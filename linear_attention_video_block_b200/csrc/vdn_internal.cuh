@@ -1,0 +1,161 @@
+// Internal declarations shared by the libvdn CUDA sources.
+//
+// The query-group schedule. Queries are partitioned into groups of rows that
+// share one key set and one pair of VDA read states:
+//   group 0          boundary frame 0          (sees every frame)
+//   group 1          boundary frame F-1        (sees every frame; absent if F < 2)
+//   group 2 + j      non-boundary frames of chunk j, j = 0 .. J-1 (may be empty)
+// The heavy boundary groups come first so that they are scheduled early.
+// Key set of a chunk group (project page "Local Softmax and Long-Range Linear
+// Memory": each chunk attends to itself and both neighbour chunks, plus the
+// 4-way boundary anchors and the text tokens): frames [lo, hi] with
+// lo = max(0, c(j-1)), hi = min(F-1, c(j+2)-1), plus frames 0 and F-1, merged
+// into at most 3 disjoint token intervals; text keys are a separate segment.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "../../include/vdn.h"
+
+namespace vdn {
+
+struct Layout {
+  int B, F, N, T, c, H, d;
+  __host__ __device__ long long L() const { return (long long)F * N; }
+  __host__ __device__ int J() const { return (F + c - 1) / c; }
+  __host__ __device__ int groups() const { return J() + 2; }
+};
+
+struct Group {
+  int q0;          // first video token of the group
+  int nq;          // number of query tokens (0 = empty group)
+  int nseg;        // video key segments
+  int seg0[3];     // segment start token
+  int segn[3];     // segment length in tokens
+  int chunk;       // chunk index (-1 for boundary groups)
+  int fwd_idx;     // forward state index: state after frames 1..fwd_idx (0 = S0)
+  int rev_idx;     // reverse state index: state after frames F-2..rev_idx (F-1 = S0)
+};
+
+__host__ __device__ inline void chunk_window(const Layout& l, int j, int& lo, int& hi) {
+  lo = l.c * (j - 1);
+  if (lo < 0) lo = 0;
+  hi = l.c * (j + 2) - 1;
+  if (hi > l.F - 1) hi = l.F - 1;
+}
+
+__host__ __device__ inline Group make_group(const Layout& l, int g) {
+  Group G;
+  G.nseg = 0;
+  G.chunk = -1;
+  G.fwd_idx = 0;
+  G.rev_idx = l.F - 1;
+  for (int s = 0; s < 3; ++s) { G.seg0[s] = 0; G.segn[s] = 0; }
+  const int N = l.N, F = l.F;
+  if (g == 0 || g == 1) {
+    int f = (g == 0) ? 0 : F - 1;
+    if (g == 1 && F < 2) { G.q0 = 0; G.nq = 0; return G; }
+    G.q0 = f * N;
+    G.nq = N;
+    G.nseg = 1;
+    G.seg0[0] = 0;
+    G.segn[0] = F * N;
+    return G;
+  }
+  int j = g - 2;
+  int f0 = j * l.c, f1 = (j + 1) * l.c - 1;
+  if (f0 < 1) f0 = 1;
+  if (f1 > F - 2) f1 = F - 2;
+  G.chunk = j;
+  if (f1 < f0) { G.q0 = 0; G.nq = 0; return G; }
+  G.q0 = f0 * N;
+  G.nq = (f1 - f0 + 1) * N;
+  int lo, hi;
+  chunk_window(l, j, lo, hi);
+  // frames {0} u [lo, hi] u {F-1}, merged
+  int a = lo, b = hi;
+  if (a <= 1) a = 0; else { G.seg0[G.nseg] = 0; G.segn[G.nseg] = N; G.nseg++; }
+  bool tail_merged = (b >= F - 2);
+  if (tail_merged) b = F - 1;
+  G.seg0[G.nseg] = a * N; G.segn[G.nseg] = (b - a + 1) * N; G.nseg++;
+  if (!tail_merged) { G.seg0[G.nseg] = (F - 1) * N; G.segn[G.nseg] = N; G.nseg++; }
+  G.fwd_idx = (lo - 1 >= 1) ? lo - 1 : 0;
+  G.rev_idx = (hi + 1 <= F - 2) ? hi + 1 : F - 1;
+  return G;
+}
+
+// Per-(b, h) tile enumeration over groups: tile t of `rows`-row tiles.
+__host__ __device__ inline int tiles_per_head(const Layout& l, int rows) {
+  int n = 0;
+  for (int g = 0; g < l.groups(); ++g) {
+    Group G = make_group(l, g);
+    n += (G.nq + rows - 1) / rows;
+  }
+  return n;
+}
+
+__host__ __device__ inline void tile_to_group(const Layout& l, int rows, int t, int& g, int& r0) {
+  for (g = 0; g < l.groups(); ++g) {
+    Group G = make_group(l, g);
+    int n = (G.nq + rows - 1) / rows;
+    if (t < n) { r0 = G.q0 + t * rows; return; }
+    t -= n;
+  }
+  g = -1;
+  r0 = 0;
+}
+
+// Scan extents: forward scan runs frames 1..fwd_max, reverse scan frames
+// F-2 down to rev_min (rev_min = F-1 means no reverse frame).
+inline void scan_extent(const Layout& l, int& fwd_max, int& rev_min) {
+  fwd_max = 0;
+  rev_min = l.F - 1;
+  for (int j = 0; j < l.J(); ++j) {
+    Group G = make_group(l, 2 + j);
+    if (G.nq == 0) continue;
+    if (G.fwd_idx > fwd_max) fwd_max = G.fwd_idx;
+    if (G.rev_idx < rev_min) rev_min = G.rev_idx;
+  }
+}
+
+template <typename T> __device__ inline float to_f32(T x);
+template <> __device__ inline float to_f32<float>(float x) { return x; }
+template <> __device__ inline float to_f32<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ inline T from_f32(float x);
+template <> __device__ inline float from_f32<float>(float x) { return x; }
+template <> __device__ inline __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+// ---------------------------------------------------------------- launchers
+// Each returns cudaGetLastError() after its launch(es).
+
+// SIMT window softmax (any supported dtype/d); o_soft in the io dtype.
+cudaError_t launch_window_simt(const Layout& l, int dtype, const void* q, const void* k,
+                               const void* v, const void* kt, const void* vt, void* o,
+                               float* lse, cudaStream_t st);
+// tcgen05 window softmax (bf16, d in {64, 128}).
+bool window_tc_supported(const Layout& l, int dtype);
+cudaError_t launch_window_tc(const Layout& l, const void* q, const void* k, const void* v,
+                             const void* kt, const void* vt, void* o, float* lse,
+                             cudaStream_t st);
+
+// Reads and clears the device status word of the tcgen05 kernels' translation
+// unit (bounded waits record VDN_ERR_TIMEOUT there).
+cudaError_t read_and_clear_tc_status(int* status);
+
+// VDA: Gram into (am, bw) slots [B, H, F, d, d] (slot 0 = text), inverse in place
+// of am, scans into states [B, H, 2, J, d, d].
+cudaError_t launch_vda_states(const Layout& l, int dtype, const void* k, const void* v,
+                              const void* kt, const void* vt, const float* beta,
+                              const float* beta_text, float* am, float* bw, float* states,
+                              cudaStream_t st);
+
+// Readout / norm / gates. mode 0: o_lin only (ungated, pre-norm) into out.
+// mode 1: out = sig(gs) o_soft + sig(gl) rms(o_lin); optional out_soft/out_lin.
+cudaError_t launch_readout(const Layout& l, int dtype, int mode, const void* q,
+                           const float* states, const void* o_soft, const void* gs,
+                           const void* gl, const float* rms_w, float eps, void* out,
+                           void* out_soft, void* out_lin, cudaStream_t st);
+
+}  // namespace vdn

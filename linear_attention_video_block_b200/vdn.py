@@ -1,0 +1,188 @@
+"""ctypes binding of libvdn (the C ABI declared in include/vdn.h).
+
+Argument marshalling only: every step of the operation runs in libvdn's CUDA
+kernels. PyTorch provides device memory and the current stream. There is no
+CPU fallback: the functions raise if the library or a CUDA device is missing.
+
+Public calls (same names as the C ABI, without the ``vdn_`` prefix):
+  window_softmax_fwd, vda_scan_fwd, hybrid_attn_fwd, workspace_bytes,
+  device_status.
+Tensors follow the C ABI's layout: q/k/v/gates/outputs [B, L, H, d],
+text k/v [B, T, H, d], beta [B, L, H] and beta_text [B, T, H] in float32.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from .synth import Layout
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvdn.so")
+_lib = None
+
+VDN_F32, VDN_BF16 = 0, 1
+STATUS = {0: "VDN_OK", 1: "VDN_ERR_INVALID", 2: "VDN_ERR_UNSUPPORTED",
+          3: "VDN_ERR_WORKSPACE", 4: "VDN_ERR_CUDA", 5: "VDN_ERR_TIMEOUT"}
+EXPORTS = ("vdn_workspace_bytes", "vdn_window_softmax_fwd", "vdn_vda_scan_fwd",
+           "vdn_hybrid_attn_fwd", "vdn_device_status", "vdn_status_string")
+
+
+class VdnError(RuntimeError):
+    def __init__(self, code, where):
+        msg = lib().vdn_status_string(code).decode() if _lib is not None else ""
+        super().__init__(f"{where}: {STATUS.get(code, code)} ({msg})")
+        self.code = code
+
+
+class _CLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("B", "F", "N", "T", "c", "H", "d")]
+
+
+def lib():
+    """Loads libvdn.so (built in-tree by ``build.py``); raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"libvdn.so not built ({_LIB_PATH}); run "
+                               "python -m linear_attention_video_block_b200.build")
+        L = ctypes.CDLL(_LIB_PATH)
+        P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        LP = ctypes.POINTER(_CLayout)
+        L.vdn_workspace_bytes.argtypes = [LP, I]
+        L.vdn_workspace_bytes.restype = S
+        L.vdn_window_softmax_fwd.argtypes = [LP, I] + [P] * 8
+        L.vdn_window_softmax_fwd.restype = I
+        L.vdn_vda_scan_fwd.argtypes = [LP, I] + [P] * 9 + [P, S, P]
+        L.vdn_vda_scan_fwd.restype = I
+        L.vdn_hybrid_attn_fwd.argtypes = [LP, I] + [P] * 9 + [P, ctypes.c_float] + [P] * 3 + [P, S, P]
+        L.vdn_hybrid_attn_fwd.restype = I
+        L.vdn_device_status.argtypes = []
+        L.vdn_device_status.restype = I
+        L.vdn_status_string.argtypes = [I]
+        L.vdn_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _clayout(layout: Layout):
+    return _CLayout(layout.B, layout.F, layout.N, layout.T, layout.c, layout.H, layout.d)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return VDN_F32
+    if t.dtype == torch.bfloat16:
+        return VDN_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check(code, where):
+    if code != 0:
+        raise VdnError(code, where)
+
+
+def _require_cuda():
+    if not torch.cuda.is_available():
+        raise RuntimeError("libvdn needs a CUDA device; there is no CPU path")
+
+
+def workspace_bytes(layout: Layout, dtype: torch.dtype) -> int:
+    code = VDN_BF16 if dtype == torch.bfloat16 else VDN_F32
+    return int(lib().vdn_workspace_bytes(ctypes.byref(_clayout(layout)), code))
+
+
+def window_softmax_fwd(layout: Layout, q, k, v, k_text, v_text, o_soft=None, lse=None,
+                       want_lse=False):
+    """Softmax branch: returns o_soft (and lse [B, L, H] if want_lse)."""
+    _require_cuda()
+    if o_soft is None:
+        o_soft = torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    code = lib().vdn_window_softmax_fwd(
+        ctypes.byref(_clayout(layout)), _dtype_code(q), _ptr(q), _ptr(k), _ptr(v),
+        _ptr(k_text), _ptr(v_text), _ptr(o_soft), _ptr(lse), _stream(q.device))
+    _check(code, "vdn_window_softmax_fwd")
+    return (o_soft, lse) if want_lse else o_soft
+
+
+def vda_scan_fwd(layout: Layout, q, k, v, k_text, v_text, beta, beta_text, o_lin=None,
+                 chunk_states=None, want_states=False, workspace=None):
+    """Linear branch: returns o_lin (ungated, pre-norm) and, if want_states, the
+    chunk table [B, H, 2, J, d, d] float32."""
+    _require_cuda()
+    if o_lin is None:
+        o_lin = torch.empty_like(q)
+    if want_states and chunk_states is None:
+        J = -(-layout.F // layout.c)
+        chunk_states = torch.empty((layout.B, layout.H, 2, J, layout.d, layout.d),
+                                   dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(workspace_bytes(layout, q.dtype), dtype=torch.uint8, device=q.device)
+    code = lib().vdn_vda_scan_fwd(
+        ctypes.byref(_clayout(layout)), _dtype_code(q), _ptr(q), _ptr(k), _ptr(v),
+        _ptr(k_text), _ptr(v_text), _ptr(beta), _ptr(beta_text), _ptr(o_lin),
+        _ptr(chunk_states), _ptr(workspace), workspace.numel(), _stream(q.device))
+    _check(code, "vdn_vda_scan_fwd")
+    return (o_lin, chunk_states) if want_states else o_lin
+
+
+def hybrid_attn_fwd(layout: Layout, q, k, v, k_text, v_text, beta, beta_text, g_soft, g_lin,
+                    rms_weight=None, rms_eps=1e-6, out=None, out_soft=None, out_lin=None,
+                    workspace=None, device=None):
+    """The hybrid forward: out = sigmoid(g_soft) o_soft + sigmoid(g_lin) RMSNorm(o_lin).
+
+    Device tensors: launched asynchronously on the current stream; returns out.
+    Host tensors: copied to ``device`` (default cuda:0), computed, and the
+    result copied back to host memory (pinned inputs make the copies async).
+    """
+    _require_cuda()
+    host = not q.is_cuda
+    out_host = None
+    if host:
+        dev = torch.device(device or "cuda:0")
+        out_host, out = out, None
+        if out_soft is not None or out_lin is not None:
+            raise ValueError("out_soft/out_lin need device tensors")
+        args = [q, k, v, k_text, v_text, beta, beta_text, g_soft, g_lin, rms_weight]
+        q, k, v, k_text, v_text, beta, beta_text, g_soft, g_lin, rms_weight = [
+            None if a is None else a.to(dev, non_blocking=True) for a in args]
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = torch.empty(workspace_bytes(layout, q.dtype), dtype=torch.uint8, device=q.device)
+    code = lib().vdn_hybrid_attn_fwd(
+        ctypes.byref(_clayout(layout)), _dtype_code(q), _ptr(q), _ptr(k), _ptr(v),
+        _ptr(k_text), _ptr(v_text), _ptr(beta), _ptr(beta_text), _ptr(g_soft), _ptr(g_lin),
+        _ptr(rms_weight), ctypes.c_float(rms_eps), _ptr(out), _ptr(out_soft), _ptr(out_lin),
+        _ptr(workspace), workspace.numel(), _stream(q.device))
+    _check(code, "vdn_hybrid_attn_fwd")
+    if host:
+        if out_host is None:
+            out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        out_host.copy_(out, non_blocking=True)
+        torch.cuda.current_stream(out.device).synchronize()
+        return out_host
+    return out
+
+
+def device_status() -> int:
+    """Reads and clears libvdn's device status word (synchronises the device)."""
+    return int(lib().vdn_device_status())

@@ -1,0 +1,191 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle on
+the same seeded inputs. Error metric: max |gpu - oracle| / RMS(oracle) over the
+checked elements; bound 1e-4 for float32 storage, 2e-2 for bf16 storage with
+fp32 accumulation (the tolerances the target statement fixes).
+
+Small workloads are checked element by element in full. At the full workload
+sizes the softmax branch is checked on sampled query rows of sampled heads
+(every frame, tile and group edges included), the linear branch and the
+chunk states in full for those heads.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from linear_attention_video_block_b200 import vdn
+from linear_attention_video_block_b200.synth import Layout, WORKLOADS, make_inputs
+from oracle import vdn_oracle as O
+
+from conftest import rel_err
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+def _dev(inp):
+    return {k: v.to("cuda") for k, v in inp.items()}
+
+
+def _np(t, heads=None):
+    t = t.detach().to("cpu")
+    if heads is not None:
+        t = t[:, :, heads]
+    return t.to(torch.float64).numpy()
+
+
+def _oracle_args(inp, heads=None):
+    keys = ["q", "k", "v", "k_text", "v_text", "beta", "beta_text", "g_s", "g_l"]
+    return {k: _np(inp[k], heads) for k in keys}
+
+
+def _sample_rows(layout, per_frame=64, seed=0):
+    """Query rows: per frame its first/last two tokens, the tokens at 128-row tile
+    edges of every query group, and random ones."""
+    rng = np.random.default_rng(seed)
+    F, N = layout.F, layout.N
+    rows = set()
+    for f in range(F):
+        base = f * N
+        rows |= {base, base + 1, base + N - 2, base + N - 1}
+        rows |= set((base + rng.integers(0, N, size=per_frame)).tolist())
+    L = F * N
+    rows |= {r for r in range(0, L, 128)} if L <= 20000 else set(range(0, L, 4096))
+    rows |= {min(L - 1, r + 127) for r in range(0, L, 8192)}
+    return np.array(sorted(r for r in rows if 0 <= r < L))
+
+
+def _check_all(layout, dtype, inp, heads=None, rows=None):
+    """Runs the three entry points and compares with the oracle on (heads, rows)."""
+    tol = TOL[dtype]
+    d = _dev(inp)
+    o_soft, lse = vdn.window_softmax_fwd(layout, d["q"], d["k"], d["v"], d["k_text"], d["v_text"],
+                                         want_lse=True)
+    o_lin, states = vdn.vda_scan_fwd(layout, d["q"], d["k"], d["v"], d["k_text"], d["v_text"],
+                                     d["beta"], d["beta_text"], want_states=True)
+    out_soft = torch.empty_like(d["q"])
+    out_lin = torch.empty_like(d["q"])
+    out = vdn.hybrid_attn_fwd(layout, d["q"], d["k"], d["v"], d["k_text"], d["v_text"], d["beta"],
+                              d["beta_text"], d["g_s"], d["g_l"], out_soft=out_soft, out_lin=out_lin)
+    torch.cuda.synchronize()
+    assert vdn.device_status() == 0
+    hsel = list(range(layout.H)) if heads is None else heads
+    a = _oracle_args(inp, hsel)
+    F, N, c = layout.F, layout.N, layout.c
+    ref_soft, ref_lse = O.softmax_branch(a["q"], a["k"], a["v"], a["k_text"], a["v_text"], F, N, c,
+                                         rows=rows, return_lse=True)
+    ref_lin, st = O.linear_branch(a["q"], a["k"], a["v"], a["k_text"], a["v_text"], a["beta"],
+                                  a["beta_text"], F, N, c, return_states=True)
+    ref_out, ref_gs, ref_gl = O.combine(ref_soft, ref_lin, a["g_s"], a["g_l"])
+    res = {}
+    res["o_soft"] = rel_err(_np(o_soft, hsel), ref_soft)
+    res["lse"] = float(np.nanmax(np.abs(lse.cpu().double().numpy()[:, :, hsel] - ref_lse)))
+    res["o_lin"] = rel_err(_np(o_lin, hsel), ref_lin)
+    res["out"] = rel_err(_np(out, hsel), ref_out)
+    res["out_soft"] = rel_err(_np(out_soft, hsel), ref_gs)
+    res["out_lin"] = rel_err(_np(out_lin, hsel), ref_gl)
+    np.testing.assert_allclose(_np(out_soft, hsel) + _np(out_lin, hsel), _np(out, hsel),
+                               atol=tol * 4 * np.sqrt(np.mean(_np(out, hsel) ** 2)))
+    # chunk states against the oracle's per-frame read states
+    J = layout.J if hasattr(layout, "J") else -(-F // c)
+    st_gpu = states.cpu().double().numpy()
+    worst = 0.0
+    for hi, h in enumerate(hsel):
+        S0, fwd, rev = st[(0, hi)]
+        for j in range(J):
+            frames = [f for f in range(j * c, min(F, (j + 1) * c)) if not O.is_boundary(f, F)]
+            if not frames:
+                assert np.all(st_gpu[0, h, :, j] == 0)
+                continue
+            sf, sr = O.read_states(frames[0], F, c, fwd, rev, S0)
+            for dirn, ref in ((0, sf), (1, sr)):
+                scale = max(np.sqrt(np.mean(ref ** 2)), 1e-30)
+                worst = max(worst, np.abs(st_gpu[0, h, dirn, j] - ref).max() / scale)
+    res["states"] = worst
+    for key in ("o_soft", "o_lin", "out", "out_soft", "out_lin", "states"):
+        assert res[key] <= tol, (key, res)
+    assert res["lse"] <= (1e-4 if dtype == "f32" else 1e-2), res
+    return res
+
+
+@pytest.mark.parametrize("name", ["tiny-f32", "small-bf16"])
+def test_small_workloads_full(name):
+    layout, dtype, seed = WORKLOADS[name]
+    inp = make_inputs(layout, dtype, seed)
+    _check_all(layout, dtype, inp)
+
+
+@pytest.mark.parametrize("repeated", [False, True])
+def test_480p_like(repeated):
+    layout, dtype, seed = WORKLOADS["480p-bf16"]
+    inp = make_inputs(layout, dtype, seed, repeated_keys=repeated)
+    _check_all(layout, dtype, inp, heads=[0, layout.H - 1], rows=_sample_rows(layout, 32))
+
+
+@pytest.mark.parametrize("name", ["768p-bf16", "long-bf16"])
+def test_full_size_sampled(name):
+    layout, dtype, seed = WORKLOADS[name]
+    inp = make_inputs(layout, dtype, seed)
+    _check_all(layout, dtype, inp, heads=[0, layout.H - 1], rows=_sample_rows(layout, 24))
+
+
+EDGE = [
+    # (name, layout, dtype)
+    ("one-frame", Layout(B=1, F=1, N=37, T=5, c=2, H=2, d=64), "bf16"),
+    ("two-frames", Layout(B=2, F=2, N=130, T=3, c=3, H=1, d=128), "bf16"),
+    ("three-frames", Layout(B=1, F=3, N=50, T=7, c=1, H=2, d=64), "bf16"),
+    ("no-text", Layout(B=1, F=9, N=70, T=0, c=2, H=2, d=128), "bf16"),
+    ("one-token-frames", Layout(B=1, F=12, N=1, T=2, c=2, H=3, d=64), "bf16"),
+    ("c-over-F", Layout(B=1, F=6, N=40, T=9, c=8, H=1, d=128), "bf16"),
+    ("c1-ragged", Layout(B=2, F=7, N=200, T=130, c=1, H=2, d=128), "bf16"),
+    ("f32-d32", Layout(B=1, F=10, N=33, T=6, c=3, H=2, d=32), "f32"),
+    ("f32-d64", Layout(B=1, F=11, N=20, T=4, c=2, H=1, d=64), "f32"),
+    ("f32-d128", Layout(B=2, F=7, N=19, T=1, c=2, H=1, d=128), "f32"),
+    ("f32-d16-no-text", Layout(B=1, F=13, N=8, T=0, c=4, H=2, d=16), "f32"),
+]
+
+
+@pytest.mark.parametrize("name,layout,dtype", EDGE, ids=[e[0] for e in EDGE])
+def test_edge_layouts(name, layout, dtype):
+    inp = make_inputs(layout, dtype, seed=100 + len(name))
+    _check_all(layout, dtype, inp)
+
+
+def test_rms_weight_and_eps():
+    layout = Layout(B=1, F=9, N=40, T=5, c=2, H=2, d=64)
+    inp = make_inputs(layout, "bf16", 7)
+    d = _dev(inp)
+    w = torch.linspace(0.5, 1.5, layout.d, dtype=torch.float32, device="cuda")
+    out = vdn.hybrid_attn_fwd(layout, d["q"], d["k"], d["v"], d["k_text"], d["v_text"], d["beta"],
+                              d["beta_text"], d["g_s"], d["g_l"], rms_weight=w, rms_eps=1e-3)
+    a = _oracle_args(inp)
+    ref = O.hybrid(a["q"], a["k"], a["v"], a["k_text"], a["v_text"], a["beta"], a["beta_text"],
+                   a["g_s"], a["g_l"], layout.F, layout.N, layout.c, eps=1e-3,
+                   weight=w.cpu().double().numpy())["out"]
+    assert rel_err(_np(out), ref) <= TOL["bf16"]
+
+
+def test_host_buffers_public_api():
+    """The public call with host tensors copies in, computes on the GPU and copies
+    the result back; same values as the device call."""
+    layout, dtype, seed = WORKLOADS["small-bf16"]
+    inp = make_inputs(layout, dtype, seed)
+    host = {k: v.pin_memory() for k, v in inp.items()}
+    out_h = vdn.hybrid_attn_fwd(layout, host["q"], host["k"], host["v"], host["k_text"],
+                                host["v_text"], host["beta"], host["beta_text"], host["g_s"], host["g_l"])
+    assert not out_h.is_cuda
+    d = _dev(inp)
+    out_d = vdn.hybrid_attn_fwd(layout, d["q"], d["k"], d["v"], d["k_text"], d["v_text"], d["beta"],
+                                d["beta_text"], d["g_s"], d["g_l"])
+    assert torch.equal(out_h, out_d.cpu())
+
+
+def test_repeated_calls_are_deterministic():
+    layout, dtype, seed = WORKLOADS["small-bf16"]
+    d = _dev(make_inputs(layout, dtype, seed))
+    args = (layout, d["q"], d["k"], d["v"], d["k_text"], d["v_text"], d["beta"], d["beta_text"],
+            d["g_s"], d["g_l"])
+    a = vdn.hybrid_attn_fwd(*args).clone()
+    b = vdn.hybrid_attn_fwd(*args)
+    assert torch.equal(a, b)

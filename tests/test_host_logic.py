@@ -1,0 +1,145 @@
+"""Host-side logic of the CUDA path, checked on the CPU (no GPU calls):
+the exported C ABI, its argument validation, and the query-group schedule the
+kernels use, against the oracle's key sets and read states."""
+
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+from oracle import vdn_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "vdn.h")
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(vdn_[a-z_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from linear_attention_video_block_b200 import vdn
+    return vdn.lib()
+
+
+def test_library_exports_every_declared_function(lib):
+    names = _declared_functions()
+    assert {"vdn_window_softmax_fwd", "vdn_vda_scan_fwd", "vdn_hybrid_attn_fwd"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert lib.vdn_status_string(code)
+    assert lib.vdn_status_string(99) == b"unknown status"
+
+
+def _layout(**kw):
+    from linear_attention_video_block_b200 import vdn
+    base = dict(B=1, F=8, N=16, T=4, c=2, H=1, d=16)
+    base.update(kw)
+    return vdn._CLayout(*[base[k] for k in ("B", "F", "N", "T", "c", "H", "d")])
+
+
+FAKE = ctypes.c_void_p(1 << 20)        # never dereferenced: validation fails first
+MISALIGNED = ctypes.c_void_p((1 << 20) + 8)
+
+
+def test_validation_rejects_before_any_launch(lib):
+    """Every rejected call returns before touching CUDA (these run without a GPU)."""
+    w = lib.vdn_window_softmax_fwd
+    ok = _layout()
+    args = [FAKE] * 6 + [None, None]
+    assert w(ctypes.byref(_layout(B=0)), 0, *args) == 1          # invalid layout
+    assert w(ctypes.byref(_layout(c=0)), 0, *args) == 1
+    assert w(None, 0, *args) == 1
+    assert w(ctypes.byref(ok), 7, *args) == 2                    # unknown dtype
+    assert w(ctypes.byref(_layout(d=16)), 1, *args) == 2         # bf16 needs d in {64,128}
+    assert w(ctypes.byref(_layout(d=48)), 0, *args) == 2
+    assert w(ctypes.byref(ok), 0, None, FAKE, FAKE, FAKE, FAKE, FAKE, None, None) == 1
+    assert w(ctypes.byref(ok), 0, FAKE, FAKE, FAKE, None, FAKE, FAKE, None, None) == 1  # T>0 needs text
+    assert w(ctypes.byref(ok), 0, MISALIGNED, FAKE, FAKE, FAKE, FAKE, FAKE, None, None) == 2
+    need = lib.vdn_workspace_bytes(ctypes.byref(ok), 0)
+    assert need > 0 and lib.vdn_workspace_bytes(ctypes.byref(_layout(N=0)), 0) == 0
+    v = lib.vdn_vda_scan_fwd
+    vargs = [FAKE] * 8 + [None, FAKE]
+    assert v(ctypes.byref(ok), 0, *vargs, 256, None) == 3        # short workspace
+    assert v(ctypes.byref(ok), 0, *vargs[:-1], None, need, None) == 3
+    h = lib.vdn_hybrid_attn_fwd
+    hargs = [FAKE] * 9 + [None, ctypes.c_float(1e-6), FAKE, None, None, FAKE]
+    assert h(ctypes.byref(ok), 0, *hargs, need - 1, None) == 3
+    assert h(ctypes.byref(ok), 0, *hargs[:9], None, ctypes.c_float(-1.0), FAKE, None, None, FAKE, need, None) == 1
+
+
+@pytest.fixture(scope="module")
+def schedule_dump():
+    out = os.path.join(tempfile.mkdtemp(), "schedule_dump")
+    src = os.path.join(ROOT, "tests", "host", "schedule_dump.cu")
+    nvcc = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+    subprocess.run([nvcc, "-std=c++17", "-o", out, src], check=True, capture_output=True)
+    return out
+
+
+def _parse(text):
+    groups, tiles = [], []
+    extent = None
+    for line in text.splitlines():
+        t = line.split()
+        if t[0] == "extent":
+            extent = (int(t[1]), int(t[2]), int(t[4]))
+        elif t[0] == "group":
+            segs = [tuple(map(int, s.split(":"))) for s in t[13:]]
+            groups.append(dict(g=int(t[1]), q0=int(t[3]), nq=int(t[5]), chunk=int(t[7]),
+                               fwd=int(t[9]), rev=int(t[11]), segs=segs))
+        elif t[0] == "tile":
+            tiles.append((int(t[3]), int(t[5])))
+    return extent, groups, tiles
+
+
+@pytest.mark.parametrize("F", [1, 2, 3, 4, 5, 7, 8, 11, 16, 21, 36])
+@pytest.mark.parametrize("c", [1, 2, 3, 5, 6])
+def test_cuda_schedule_matches_oracle_key_sets(schedule_dump, F, c):
+    N, rows = 3, 4
+    r = subprocess.run([schedule_dump, str(F), str(N), str(c), str(rows)], check=True,
+                       capture_output=True, text=True)
+    (fwd_max, rev_min, ntiles), groups, tiles = _parse(r.stdout)
+    covered = []
+    need_fwd, need_rev = 0, F - 1
+    for G in groups:
+        if G["nq"] == 0:
+            continue
+        frames = sorted({t // N for t in range(G["q0"], G["q0"] + G["nq"])})
+        covered += list(range(G["q0"], G["q0"] + G["nq"]))
+        key_tokens = set()
+        for s0, sn in G["segs"]:
+            seg = set(range(s0, s0 + sn))
+            assert not (seg & key_tokens), "segments overlap"
+            key_tokens |= seg
+        for f in frames:
+            want = {g * N + n for g in O.softmax_key_frames(f, F, c) for n in range(N)}
+            assert key_tokens == want, (F, c, f)
+            fr, rr = O.forward_region(f, F, c), O.reverse_region(f, F, c)
+            if O.is_boundary(f, F):
+                assert G["chunk"] == -1 and len(frames) == 1
+                continue
+            assert G["chunk"] == O.chunk_of(f, c)
+            assert G["fwd"] == (max(fr) if fr else 0)
+            assert G["rev"] == (min(rr) if rr else F - 1)
+            need_fwd = max(need_fwd, G["fwd"])
+            need_rev = min(need_rev, G["rev"])
+    assert sorted(covered) == list(range(F * N))
+    assert (fwd_max, rev_min) == (need_fwd, need_rev)
+    # tiles: every query row in exactly one tile of its group
+    seen = []
+    for g, r0 in tiles:
+        G = groups[g]
+        assert G["q0"] <= r0 < G["q0"] + G["nq"]
+        seen += [t for t in range(r0, min(r0 + rows, G["q0"] + G["nq"]))]
+    assert sorted(seen) == list(range(F * N)) and len(tiles) == ntiles
