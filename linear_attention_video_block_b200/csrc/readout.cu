@@ -21,7 +21,7 @@ __device__ inline float sigmoidf_(float x) { return 1.f / (1.f + expf(-x)); }
 template <typename T, int D>
 __global__ void __launch_bounds__(NT)
 readout_kernel(Layout l, int mode, const T* __restrict__ q, const float* __restrict__ states,
-               const T* __restrict__ o_soft, const T* __restrict__ gs, const T* __restrict__ gl,
+               const float* __restrict__ o_soft, const T* __restrict__ gs, const T* __restrict__ gl,
                const float* __restrict__ rms_w, float eps, T* __restrict__ out,
                T* __restrict__ out_soft, T* __restrict__ out_lin) {
   extern __shared__ __align__(16) float ro_smem[];
@@ -81,7 +81,7 @@ readout_kernel(Layout l, int mode, const T* __restrict__ q, const float* __restr
 #pragma unroll
   for (int i = 0; i < OC; ++i) {
     const float w = rms_w ? rms_w[c0 + i] : 1.f;
-    const float a = sigmoidf_(to_f32(gs[base + i])) * to_f32(o_soft[base + i]);
+    const float a = sigmoidf_(to_f32(gs[base + i])) * o_soft[base + i];
     const float bb = sigmoidf_(to_f32(gl[base + i])) * (acc[i] * rstd * w);
     out[base + i] = from_f32<T>(a + bb);
     if (out_soft) out_soft[base + i] = from_f32<T>(a);
@@ -91,7 +91,7 @@ readout_kernel(Layout l, int mode, const T* __restrict__ q, const float* __restr
 
 template <typename T, int D>
 cudaError_t launch_readout_t(const Layout& l, int mode, const void* q, const float* states,
-                             const void* o_soft, const void* gs, const void* gl,
+                             const float* o_soft, const void* gs, const void* gl,
                              const float* rms_w, float eps, void* out, void* out_soft,
                              void* out_lin, cudaStream_t st) {
   auto kern = readout_kernel<T, D>;
@@ -100,7 +100,7 @@ cudaError_t launch_readout_t(const Layout& l, int mode, const void* q, const flo
   if (e != cudaSuccess) return e;
   dim3 grid(tiles_per_head(l, BQ), l.H, l.B);
   if (grid.x == 0) return cudaSuccess;
-  kern<<<grid, NT, smem, st>>>(l, mode, (const T*)q, states, (const T*)o_soft, (const T*)gs,
+  kern<<<grid, NT, smem, st>>>(l, mode, (const T*)q, states, o_soft, (const T*)gs,
                                (const T*)gl, rms_w, eps, (T*)out, (T*)out_soft, (T*)out_lin);
   return cudaGetLastError();
 }
@@ -108,7 +108,7 @@ cudaError_t launch_readout_t(const Layout& l, int mode, const void* q, const flo
 }  // namespace
 
 cudaError_t launch_readout(const Layout& l, int dtype, int mode, const void* q,
-                           const float* states, const void* o_soft, const void* gs,
+                           const float* states, const float* o_soft, const void* gs,
                            const void* gl, const float* rms_w, float eps, void* out,
                            void* out_soft, void* out_lin, cudaStream_t st) {
 #define VDN_RO(T, D) \

@@ -13,8 +13,6 @@ constexpr size_t kAlign = 256;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
-size_t esize(int dtype) { return dtype == VDN_BF16 ? 2 : 4; }
-
 bool layout_ok(const vdn_layout_t* l) {
   if (!l) return false;
   if (l->B < 1 || l->F < 1 || l->N < 1 || l->T < 0 || l->c < 1 || l->H < 1 || l->d < 1) return false;
@@ -43,7 +41,7 @@ struct Workspace {
   float* am = nullptr;
   float* bw = nullptr;
   float* states = nullptr;
-  void* o_soft = nullptr;
+  float* o_soft = nullptr;  // float32 intermediate of the hybrid path
   size_t bytes = 0;
 };
 
@@ -62,7 +60,7 @@ Workspace carve(const Layout& l, int dtype, void* base, bool need_states, bool n
   w.am = static_cast<float*>(take(bh * l.F * dd * sizeof(float)));
   w.bw = static_cast<float*>(take(bh * l.F * dd * sizeof(float)));
   if (need_states) w.states = static_cast<float*>(take(bh * 2 * l.J() * dd * sizeof(float)));
-  if (need_osoft) w.o_soft = take((size_t)l.B * l.L() * l.H * l.d * esize(dtype));
+  if (need_osoft) w.o_soft = static_cast<float*>(take((size_t)l.B * l.L() * l.H * l.d * sizeof(float)));
   w.bytes = off;
   return w;
 }
@@ -70,10 +68,11 @@ Workspace carve(const Layout& l, int dtype, void* base, bool need_states, bool n
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? VDN_OK : VDN_ERR_CUDA; }
 
 int run_window(const Layout& l, int dtype, const void* q, const void* k, const void* v,
-               const void* kt, const void* vt, void* o, float* lse, cudaStream_t st) {
+               const void* kt, const void* vt, void* o, bool out_f32, float* lse,
+               cudaStream_t st) {
   if (vdn::window_tc_supported(l, dtype))
-    return cuda_status(vdn::launch_window_tc(l, q, k, v, kt, vt, o, lse, st));
-  return cuda_status(vdn::launch_window_simt(l, dtype, q, k, v, kt, vt, o, lse, st));
+    return cuda_status(vdn::launch_window_tc(l, q, k, v, kt, vt, o, out_f32, lse, st));
+  return cuda_status(vdn::launch_window_simt(l, dtype, q, k, v, kt, vt, o, out_f32, lse, st));
 }
 
 }  // namespace
@@ -97,7 +96,7 @@ int vdn_window_softmax_fwd(const vdn_layout_t* layout, int dtype, const void* q,
   if (layout->T > 0 && (!aligned16(k_text) || !aligned16(v_text))) return VDN_ERR_UNSUPPORTED;
   const Layout l = to_layout(layout);
   return run_window(l, dtype, q, k, v, layout->T ? k_text : nullptr,
-                    layout->T ? v_text : nullptr, o_soft, lse, stream);
+                    layout->T ? v_text : nullptr, o_soft, false, lse, stream);
 }
 
 int vdn_vda_scan_fwd(const vdn_layout_t* layout, int dtype, const void* q, const void* k,
@@ -149,7 +148,7 @@ int vdn_hybrid_attn_fwd(const vdn_layout_t* layout, int dtype, const void* q, co
   const void* kt = layout->T ? k_text : nullptr;
   const void* vt = layout->T ? v_text : nullptr;
   const float* bt = layout->T ? beta_text : nullptr;
-  int s = run_window(l, dtype, q, k, v, kt, vt, w.o_soft, nullptr, stream);
+  int s = run_window(l, dtype, q, k, v, kt, vt, w.o_soft, true, nullptr, stream);
   if (s != VDN_OK) return s;
   s = cuda_status(vdn::launch_vda_states(l, dtype, k, v, kt, vt, beta, bt, w.am, w.bw, w.states, stream));
   if (s != VDN_OK) return s;

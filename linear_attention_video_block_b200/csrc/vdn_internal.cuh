@@ -130,14 +130,15 @@ template <> __device__ inline __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { r
 // ---------------------------------------------------------------- launchers
 // Each returns cudaGetLastError() after its launch(es).
 
-// SIMT window softmax (any supported dtype/d); o_soft in the io dtype.
+// SIMT window softmax (any supported dtype/d); o_soft in the io dtype, or in
+// float32 when out_f32 (the hybrid path's intermediate).
 cudaError_t launch_window_simt(const Layout& l, int dtype, const void* q, const void* k,
                                const void* v, const void* kt, const void* vt, void* o,
-                               float* lse, cudaStream_t st);
+                               bool out_f32, float* lse, cudaStream_t st);
 // tcgen05 window softmax (bf16, d in {64, 128}).
 bool window_tc_supported(const Layout& l, int dtype);
 cudaError_t launch_window_tc(const Layout& l, const void* q, const void* k, const void* v,
-                             const void* kt, const void* vt, void* o, float* lse,
+                             const void* kt, const void* vt, void* o, bool out_f32, float* lse,
                              cudaStream_t st);
 
 // Reads and clears the device status word of the tcgen05 kernels' translation
@@ -153,8 +154,9 @@ cudaError_t launch_vda_states(const Layout& l, int dtype, const void* k, const v
 
 // Readout / norm / gates. mode 0: o_lin only (ungated, pre-norm) into out.
 // mode 1: out = sig(gs) o_soft + sig(gl) rms(o_lin); optional out_soft/out_lin.
+// o_soft is float32 [B, L, H, d].
 cudaError_t launch_readout(const Layout& l, int dtype, int mode, const void* q,
-                           const float* states, const void* o_soft, const void* gs,
+                           const float* states, const float* o_soft, const void* gs,
                            const void* gl, const float* rms_w, float eps, void* out,
                            void* out_soft, void* out_lin, cudaStream_t st);
 

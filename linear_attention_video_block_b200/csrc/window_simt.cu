@@ -5,6 +5,8 @@
 // group's key segments (merged window + anchor frame intervals, then the text
 // keys) in 64-key tiles with an online softmax (project page "Local Softmax and
 // Long-Range Linear Memory": one normaliser over window, anchors and text).
+#include <type_traits>
+
 #include "vdn_internal.cuh"
 
 namespace vdn {
@@ -14,7 +16,7 @@ constexpr int BQ = 64;
 constexpr int BK = 64;
 constexpr int NT = 256;
 
-template <typename T, int D>
+template <int D>
 struct SimtSmem {
   float q[BQ][D];
   float k[BK][D + 1];
@@ -22,13 +24,13 @@ struct SimtSmem {
   float p[BQ][BK + 1];
 };
 
-template <typename T, int D>
+template <typename T, typename TO, int D>
 __global__ void __launch_bounds__(NT)
 window_simt_kernel(Layout l, const T* __restrict__ q, const T* __restrict__ k,
                    const T* __restrict__ v, const T* __restrict__ kt,
-                   const T* __restrict__ vt, T* __restrict__ o, float* __restrict__ lse) {
+                   const T* __restrict__ vt, TO* __restrict__ o, float* __restrict__ lse) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  SimtSmem<T, D>& sm = *reinterpret_cast<SimtSmem<T, D>*>(smem_raw);
+  SimtSmem<D>& sm = *reinterpret_cast<SimtSmem<D>*>(smem_raw);
   const int tid = threadIdx.x;
   const int h = blockIdx.y, b = blockIdx.z;
   int g, r0;
@@ -140,23 +142,32 @@ window_simt_kernel(Layout l, const T* __restrict__ q, const T* __restrict__ k,
   }
   if (orow < rows_valid) {
     const float inv = 1.f / l_run;
-    T* orow_ptr = o + ((long long)b * L + r0 + orow) * HD + (long long)h * D + ocg * OC;
+    TO* orow_ptr = o + ((long long)b * L + r0 + orow) * HD + (long long)h * D + ocg * OC;
 #pragma unroll
-    for (int i = 0; i < OC; ++i) orow_ptr[i] = from_f32<T>(acc[i] * inv);
+    for (int i = 0; i < OC; ++i) orow_ptr[i] = from_f32<TO>(acc[i] * inv);
     if (lse && ocg == 0) lse[((long long)b * L + r0 + orow) * l.H + h] = m_run + logf(l_run);
   }
 }
 
 template <typename T, int D>
 cudaError_t launch_simt_t(const Layout& l, const void* q, const void* k, const void* v,
-                          const void* kt, const void* vt, void* o, float* lse,
+                          const void* kt, const void* vt, void* o, bool out_f32, float* lse,
                           cudaStream_t st) {
-  auto kern = window_simt_kernel<T, D>;
-  const int smem = (int)sizeof(SimtSmem<T, D>);
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
+  if (!out_f32 && std::is_same<T, float>::value) out_f32 = true;
+  const int smem = (int)sizeof(SimtSmem<D>);
   dim3 grid(tiles_per_head(l, BQ), l.H, l.B);
   if (grid.x == 0) return cudaSuccess;
+  if (out_f32) {
+    auto kern = window_simt_kernel<T, float, D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, NT, smem, st>>>(l, (const T*)q, (const T*)k, (const T*)v, (const T*)kt,
+                                 (const T*)vt, (float*)o, lse);
+    return cudaGetLastError();
+  }
+  auto kern = window_simt_kernel<T, T, D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
   kern<<<grid, NT, smem, st>>>(l, (const T*)q, (const T*)k, (const T*)v, (const T*)kt,
                                (const T*)vt, (T*)o, lse);
   return cudaGetLastError();
@@ -166,18 +177,18 @@ cudaError_t launch_simt_t(const Layout& l, const void* q, const void* k, const v
 
 cudaError_t launch_window_simt(const Layout& l, int dtype, const void* q, const void* k,
                                const void* v, const void* kt, const void* vt, void* o,
-                               float* lse, cudaStream_t st) {
+                               bool out_f32, float* lse, cudaStream_t st) {
   if (dtype == VDN_F32) {
     switch (l.d) {
-      case 16: return launch_simt_t<float, 16>(l, q, k, v, kt, vt, o, lse, st);
-      case 32: return launch_simt_t<float, 32>(l, q, k, v, kt, vt, o, lse, st);
-      case 64: return launch_simt_t<float, 64>(l, q, k, v, kt, vt, o, lse, st);
-      case 128: return launch_simt_t<float, 128>(l, q, k, v, kt, vt, o, lse, st);
+      case 16: return launch_simt_t<float, 16>(l, q, k, v, kt, vt, o, out_f32, lse, st);
+      case 32: return launch_simt_t<float, 32>(l, q, k, v, kt, vt, o, out_f32, lse, st);
+      case 64: return launch_simt_t<float, 64>(l, q, k, v, kt, vt, o, out_f32, lse, st);
+      case 128: return launch_simt_t<float, 128>(l, q, k, v, kt, vt, o, out_f32, lse, st);
     }
   } else {
     switch (l.d) {
-      case 64: return launch_simt_t<__nv_bfloat16, 64>(l, q, k, v, kt, vt, o, lse, st);
-      case 128: return launch_simt_t<__nv_bfloat16, 128>(l, q, k, v, kt, vt, o, lse, st);
+      case 64: return launch_simt_t<__nv_bfloat16, 64>(l, q, k, v, kt, vt, o, out_f32, lse, st);
+      case 128: return launch_simt_t<__nv_bfloat16, 128>(l, q, k, v, kt, vt, o, out_f32, lse, st);
     }
   }
   return cudaErrorInvalidValue;

@@ -16,7 +16,7 @@ cudaError_t read_and_clear_tc_status(int* status) {
 bool window_tc_supported(const Layout&, int) { return false; }
 
 cudaError_t launch_window_tc(const Layout&, const void*, const void*, const void*, const void*,
-                             const void*, void*, float*, cudaStream_t) {
+                             const void*, void*, bool, float*, cudaStream_t) {
   return cudaErrorNotSupported;
 }
 

@@ -1,7 +1,13 @@
 """GPU parity: the CUDA path (through the C ABI) against the float64 oracle on
-the same seeded inputs. Error metric: max |gpu - oracle| / RMS(oracle) over the
-checked elements; bound 1e-4 for float32 storage, 2e-2 for bf16 storage with
-fp32 accumulation (the tolerances the target statement fixes).
+the same seeded inputs.
+
+Bounds. The hybrid output `out`: max |gpu - oracle| / RMS(oracle) <= 1e-4 for
+float32 tensors and <= 2e-2 for bf16 tensors with fp32 accumulation. The
+intermediate results (o_soft, o_lin, the gated branches) of float32 workloads
+meet the same 1e-4; those of bf16 workloads are stored in bf16, whose rounding
+alone puts max|err|/RMS at 1.4e-2 .. 1.9e-2 on these distributions (measured
+with the oracle), so they are held per element to half a bf16 ulp of the exact
+value plus 4e-3 RMS. The fp32 chunk states meet 1e-3 relative (1e-4 for f32).
 
 Small workloads are checked element by element in full. At the full workload
 sizes the softmax branch is checked on sampled query rows of sampled heads
@@ -17,7 +23,7 @@ from linear_attention_video_block_b200 import vdn
 from linear_attention_video_block_b200.synth import Layout, WORKLOADS, make_inputs
 from oracle import vdn_oracle as O
 
-from conftest import rel_err
+from conftest import bf16_storage_ratio, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -56,6 +62,10 @@ def _sample_rows(layout, per_frame=64, seed=0):
     return np.array(sorted(r for r in rows if 0 <= r < L))
 
 
+def name_of(layout):
+    return "B{B}F{F}N{N}T{T}c{c}H{H}d{d}".format(**layout.as_dict())
+
+
 def _check_all(layout, dtype, inp, heads=None, rows=None):
     """Runs the three entry points and compares with the oracle on (heads, rows)."""
     tol = TOL[dtype]
@@ -79,12 +89,14 @@ def _check_all(layout, dtype, inp, heads=None, rows=None):
                                   a["beta_text"], F, N, c, return_states=True)
     ref_out, ref_gs, ref_gl = O.combine(ref_soft, ref_lin, a["g_s"], a["g_l"])
     res = {}
-    res["o_soft"] = rel_err(_np(o_soft, hsel), ref_soft)
+    comp = {"o_soft": (o_soft, ref_soft), "o_lin": (o_lin, ref_lin), "out_soft": (out_soft, ref_gs),
+            "out_lin": (out_lin, ref_gl)}
+    for key, (g, r) in comp.items():
+        res[key] = rel_err(_np(g, hsel), r)
+        if dtype == "bf16":
+            res[key + "_storage_ratio"] = bf16_storage_ratio(_np(g, hsel), r)
     res["lse"] = float(np.nanmax(np.abs(lse.cpu().double().numpy()[:, :, hsel] - ref_lse)))
-    res["o_lin"] = rel_err(_np(o_lin, hsel), ref_lin)
     res["out"] = rel_err(_np(out, hsel), ref_out)
-    res["out_soft"] = rel_err(_np(out_soft, hsel), ref_gs)
-    res["out_lin"] = rel_err(_np(out_lin, hsel), ref_gl)
     np.testing.assert_allclose(_np(out_soft, hsel) + _np(out_lin, hsel), _np(out, hsel),
                                atol=tol * 4 * np.sqrt(np.mean(_np(out, hsel) ** 2)))
     # chunk states against the oracle's per-frame read states
@@ -103,9 +115,15 @@ def _check_all(layout, dtype, inp, heads=None, rows=None):
                 scale = max(np.sqrt(np.mean(ref ** 2)), 1e-30)
                 worst = max(worst, np.abs(st_gpu[0, h, dirn, j] - ref).max() / scale)
     res["states"] = worst
-    for key in ("o_soft", "o_lin", "out", "out_soft", "out_lin", "states"):
-        assert res[key] <= tol, (key, res)
-    assert res["lse"] <= (1e-4 if dtype == "f32" else 1e-2), res
+    assert res["out"] <= tol, res
+    assert res["states"] <= (1e-4 if dtype == "f32" else 1e-3), res
+    for key in comp:
+        if dtype == "f32":
+            assert res[key] <= tol, (key, res)
+        else:
+            assert res[key + "_storage_ratio"] <= 1.0, (key, res)
+    assert res["lse"] <= (1e-4 if dtype == "f32" else 1e-3), res
+    print(name_of(layout), dtype, {k: round(v, 6) for k, v in res.items()})
     return res
 
 
