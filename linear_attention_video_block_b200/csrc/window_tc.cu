@@ -1,4 +1,37 @@
-// tcgen05 / TMEM / TMA window softmax for bf16 (sm_100a).
+// Block-sparse window softmax on the 5th-generation tensor cores (sm_100a):
+// tcgen05.mma with TMEM accumulators, operands staged by TMA, bf16 inputs,
+// fp32 scores / softmax statistics / output accumulation.
+//
+// What it computes (project page "Local Softmax and Long-Range Linear Memory"):
+// for every video query, softmax(q K^T / sqrt(d)) V over the keys of its
+// chunk window, the boundary anchor frames and all text tokens, one
+// normaliser. Keys are visited per query group as merged token segments
+// (window/anchor intervals, then text) in 128-key tiles; only the last tile of
+// each segment is partially masked.
+//
+// CTA = 256 query rows (two 128-row Q tiles) of one query group of one
+// (b, h); 320 threads:
+//   warps 0-3   softmax warpgroup of Q tile 0 (thread i owns row i = TMEM lane i)
+//   warps 4-7   softmax warpgroup of Q tile 1
+//   warp  8     TMA producer (one elected lane): Q once, then K_t, V_t tiles
+//               into a ring of shared-memory slots
+//   warp  9     MMA issuer (one elected lane) and TMEM owner
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+d) O1 [256+d,256+2d).
+// P (bf16) overwrites the first 64 columns of S and is the A operand of P.V
+// straight from TMEM. MMA issue order per key tile t:
+//   PV0(t), S0(t+1), PV1(t), S1(t+1)
+// so softmax of one Q tile overlaps the tensor-core work of the other.
+// The tcgen05.commit after S_w(t) also covers PV_w(t-1), so when softmax w sees
+// S_w(t) its O accumulator is stable and can be rescaled in place (lazy
+// rescaling: only when the running max grows by more than 2^8).
+//
+// Every mbarrier wait is bounded (%globaltimer, 4 s); a timeout records
+// VDN_ERR_TIMEOUT in the status word, the roles leave their loops, the
+// producer waits (bounded) for its copies in flight, the MMA issuer waits for
+// its MMAs, and TMEM is freed before exit.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "vdn_internal.cuh"
 
 namespace vdn {
@@ -13,11 +46,564 @@ cudaError_t read_and_clear_tc_status(int* status) {
   return cudaMemcpyToSymbol(g_vdn_status, &zero, sizeof(int));
 }
 
-bool window_tc_supported(const Layout&, int) { return false; }
+namespace {
 
-cudaError_t launch_window_tc(const Layout&, const void*, const void*, const void*, const void*,
-                             const void*, void*, bool, float*, cudaStream_t) {
-  return cudaErrorNotSupported;
+constexpr int kRows = 128;           // rows of a Q tile = keys of a K/V tile
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kTmemCols = 512;
+constexpr unsigned long long kWaitLimitNs = 4000000000ull;
+
+template <int D>
+struct Cfg {
+  static constexpr int kHalves = D / 64;               // 128-byte swizzle atoms per row
+  static constexpr int kTileBytes = kRows * D * 2;     // one 128 x D bf16 tile
+  static constexpr int kHalfBytes = kRows * 128;       // one 128-row x 64-column atom column
+  static constexpr int kSlots = (D == 128) ? 4 : 8;
+  static constexpr int kQBytes = 2 * kTileBytes;
+  static constexpr int kSmemBytes = 1024 + kQBytes + kSlots * kTileBytes + 256;
+};
+
+struct Bars {
+  unsigned long long q_full;
+  unsigned long long kv_full[8];
+  unsigned long long kv_empty[8];
+  unsigned long long s_full[2];
+  unsigned long long p_full[2];
+  unsigned long long o_full;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// ------------------------------------------------------------- PTX wrappers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(unsigned long long* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(unsigned long long* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(unsigned long long* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Waits for the phase of `bar` with the given parity to complete. Gives up when
+// another role has aborted (if watch_abort) or after kWaitLimitNs, in which case
+// it records VDN_ERR_TIMEOUT and raises the CTA's abort flag.
+__device__ bool mbar_wait(unsigned long long* bar, uint32_t parity, volatile int* abort,
+                          bool watch_abort = true) {
+  const uint32_t addr = smem_u32(bar);
+  if (mbar_try_wait(addr, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(addr, parity)) return true;
+    if ((i & 63u) == 0u) {
+      if (watch_abort && *abort) return false;
+      if (global_ns() - t0 > kWaitLimitNs) {
+        atomicCAS(&g_vdn_status, 0, (int)VDN_ERR_TIMEOUT);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map,
+                                            unsigned long long* bar, int c0, int c1, int c2,
+                                            int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<unsigned long long>(map)), "r"(smem_u32(bar)),
+        "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_commit(unsigned long long* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+               ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Loads 32 consecutive 32-bit TMEM columns of this thread's lane and waits.
+__device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+// Loads 128 consecutive 32-bit TMEM columns of this thread's lane and waits.
+__device__ __forceinline__ void tmem_ld_x128(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x128.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64, %65, %66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, %77, %78, %79, %80, %81, %82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95, %96, %97, %98, %99, %100, %101, %102, %103, %104, %105, %106, %107, %108, %109, %110, %111, %112, %113, %114, %115, %116, %117, %118, %119, %120, %121, %122, %123, %124, %125, %126, %127}, [%128];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]), "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]), "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]), "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]), "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]), "=r"(r[96]), "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]), "=r"(r[103]), "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]), "=r"(r[110]), "=r"(r[111]), "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]), "=r"(r[119]), "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])
+      : "r"(taddr)
+      : "memory");
+}
+
+// Stores 32 consecutive 32-bit TMEM columns of this thread's lane and waits.
+__device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};\n\t"
+      "tcgen05.wait::st.sync.aligned;\n"
+      :
+      : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+// Stores 64 consecutive 32-bit TMEM columns of this thread's lane and waits.
+__device__ __forceinline__ void tmem_st_x64(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64};\n\t"
+      "tcgen05.wait::st.sync.aligned;\n"
+      :
+      : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]), "r"(r[32]), "r"(r[33]), "r"(r[34]), "r"(r[35]), "r"(r[36]), "r"(r[37]), "r"(r[38]), "r"(r[39]), "r"(r[40]), "r"(r[41]), "r"(r[42]), "r"(r[43]), "r"(r[44]), "r"(r[45]), "r"(r[46]), "r"(r[47]), "r"(r[48]), "r"(r[49]), "r"(r[50]), "r"(r[51]), "r"(r[52]), "r"(r[53]), "r"(r[54]), "r"(r[55]), "r"(r[56]), "r"(r[57]), "r"(r[58]), "r"(r[59]), "r"(r[60]), "r"(r[61]), "r"(r[62]), "r"(r[63])
+      : "memory");
+}
+
+
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x (low half) = lo
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle, version 1 (sm_100).
+// K-major operand (rows of 128 bytes = 64 bf16 along K, 8-row groups 1024 B
+// apart): LBO unused (1), SBO = 1024 B.
+__device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) |
+         ((uint64_t)(1024u >> 4) << 32) | ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+// MN-major operand (64 contiguous elements along N per 128-byte row, one row per
+// K index): LBO = distance between 64-element N blocks, SBO = 1024 B between
+// groups of 8 K rows.
+__device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t saddr, uint32_t lbo_bytes) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)(1024u >> 4) << 32) | ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+
+// Instruction descriptor, kind::f16: D f32, A and B bf16, M = 128, N given,
+// A K-major, B K-major or MN-major.
+__host__ __device__ constexpr uint32_t make_idesc(int n, bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+// Key tile t of a query group: video segments first, then the text keys.
+struct KeyTile {
+  int text;   // 1: rows index the text tensor
+  int row;    // first key row of the tile
+  int valid;  // keys of the tile that belong to the segment (<= 128)
+};
+
+__device__ __forceinline__ int key_tile_count(const Group& G, int T) {
+  int n = 0;
+  for (int s = 0; s < G.nseg; ++s) n += (G.segn[s] + kRows - 1) / kRows;
+  return n + (T + kRows - 1) / kRows;
+}
+
+__device__ __forceinline__ KeyTile key_tile(const Group& G, int T, int t) {
+  for (int s = 0; s < G.nseg; ++s) {
+    const int n = (G.segn[s] + kRows - 1) / kRows;
+    if (t < n) return KeyTile{0, G.seg0[s] + t * kRows, min(kRows, G.segn[s] - t * kRows)};
+    t -= n;
+  }
+  return KeyTile{1, t * kRows, min(kRows, T - t * kRows)};
+}
+
+// ------------------------------------------------------------------ kernel
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kt,
+                 const __grid_constant__ CUtensorMap tm_vt, const Layout l, void* out, int out_f32,
+                 float* lse) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sKV = smem + C::kQBytes;
+  Bars* bars = reinterpret_cast<Bars*>(sKV + C::kSlots * C::kTileBytes);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int h = blockIdx.y, b = blockIdx.z;
+  int g, r0;
+  tile_to_group(l, 2 * kRows, blockIdx.x, g, r0);
+  const Group G = make_group(l, g < 0 ? 0 : g);
+  const int n_tiles = key_tile_count(G, l.T);
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int i = 0; i < C::kSlots; ++i) {
+      mbar_init(&bars->kv_full[i], 1);
+      mbar_init(&bars->kv_empty[i], 1);
+    }
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&bars->s_full[w], 1);
+      mbar_init(&bars->p_full[w], 128);
+    }
+    mbar_init(&bars->o_full, 1);
+    bars->abort = (g < 0) ? 1 : 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(smem_u32(&bars->tmem_base)), "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  volatile int* abort = &bars->abort;
+
+  if (warp == kProducerWarp) {
+    if (lane == 0 && !*abort) {
+      // ------------------------------------------------------- TMA producer
+      mbar_expect_tx(&bars->q_full, 2 * C::kTileBytes);
+      for (int qt = 0; qt < 2; ++qt)
+        for (int hf = 0; hf < C::kHalves; ++hf)
+          tma_load_4d(sQ + qt * C::kTileBytes + hf * C::kHalfBytes, &tm_q, &bars->q_full, hf * 64,
+                      h, r0 + qt * kRows, b);
+      int fills[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      int fill = 0;
+      bool ok = true;
+      for (int t = 0; t < n_tiles && ok; ++t) {
+        const KeyTile kt = key_tile(G, l.T, t);
+        for (int kv = 0; kv < 2; ++kv, ++fill) {
+          const int slot = fill % C::kSlots;
+          const int use = fill / C::kSlots;
+          if (use > 0 && !mbar_wait(&bars->kv_empty[slot], (use - 1) & 1, abort)) {
+            ok = false;
+            break;
+          }
+          const CUtensorMap* map = kt.text ? (kv ? &tm_vt : &tm_kt) : (kv ? &tm_v : &tm_k);
+          mbar_expect_tx(&bars->kv_full[slot], C::kTileBytes);
+          for (int hf = 0; hf < C::kHalves; ++hf)
+            tma_load_4d(sKV + slot * C::kTileBytes + hf * C::kHalfBytes, map, &bars->kv_full[slot],
+                        hf * 64, h, kt.row, b);
+          fills[slot] = use + 1;
+        }
+      }
+      if (!ok) {
+        // leave no copy in flight into this CTA's shared memory
+        mbar_wait(&bars->q_full, 0, abort, false);
+        for (int s = 0; s < C::kSlots; ++s)
+          if (fills[s] > 0) mbar_wait(&bars->kv_full[s], (fills[s] - 1) & 1, abort, false);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0 && !*abort) {
+      // ------------------------------------------------------- MMA issuer
+      constexpr uint32_t idesc_s = make_idesc(kRows, false);
+      constexpr uint32_t idesc_o = make_idesc(D, true);
+      const uint32_t tS[2] = {tmem, tmem + 128};
+      const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
+      const uint32_t q_addr = smem_u32(sQ);
+      const uint32_t kv_addr = smem_u32(sKV);
+      int use = 0;
+      bool ok = mbar_wait(&bars->q_full, 0, abort);
+      auto take_slot = [&](int& slot) -> bool {
+        slot = use % C::kSlots;
+        const bool r = mbar_wait(&bars->kv_full[slot], (use / C::kSlots) & 1, abort);
+        ++use;
+        tc_fence_after();
+        return r;
+      };
+      auto issue_s = [&](int w, int slot) {
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (uint32_t)((ks / 4) * C::kHalfBytes + (ks % 4) * 32);
+          mma_ss(tS[w], desc_k_sw128(q_addr + w * C::kTileBytes + off),
+                 desc_k_sw128(kv_addr + slot * C::kTileBytes + off), idesc_s, ks > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int w, int slot, bool acc) {
+#pragma unroll
+        for (int ks = 0; ks < kRows / 16; ++ks) {
+          mma_ts(tO[w], tS[w] + ks * 8,
+                 desc_mn_sw128(kv_addr + slot * C::kTileBytes + ks * 16 * 128, C::kHalfBytes),
+                 idesc_o, (acc || ks > 0) ? 1u : 0u);
+        }
+      };
+      int ks_cur = 0;
+      if (ok) ok = take_slot(ks_cur);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, ks_cur);
+        tc_commit(&bars->s_full[0]);
+        issue_s(1, ks_cur);
+        tc_commit(&bars->s_full[1]);
+        tc_commit(&bars->kv_empty[ks_cur]);
+      }
+      for (int t = 0; t < n_tiles && ok; ++t) {
+        int vs = 0, ks_next = 0;
+        if (!take_slot(vs)) { ok = false; break; }
+        if (!mbar_wait(&bars->p_full[0], t & 1, abort)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(0, vs, t > 0);
+        const bool more = t + 1 < n_tiles;
+        if (more) {
+          if (!take_slot(ks_next)) { ok = false; break; }
+          issue_s(0, ks_next);
+          tc_commit(&bars->s_full[0]);
+        }
+        if (!mbar_wait(&bars->p_full[1], t & 1, abort)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(1, vs, t > 0);
+        tc_commit(&bars->kv_empty[vs]);
+        if (more) {
+          issue_s(1, ks_next);
+          tc_commit(&bars->s_full[1]);
+          tc_commit(&bars->kv_empty[ks_next]);
+        }
+      }
+      tc_commit(&bars->o_full);
+      // every MMA issued must finish before TMEM is freed
+      if (!ok) mbar_wait(&bars->o_full, 0, abort, false);
+    }
+  } else {
+    // ----------------------------------------------------------- softmax
+    const int w = warp / 4;
+    const int row = threadIdx.x & 127;
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    const uint32_t tS = tmem + lane_base + 128 * w;
+    const uint32_t tO = tmem + lane_base + 256 + D * w;
+    const float sl2 = 1.4426950408889634f / sqrtf((float)D);  // log2(e) / sqrt(d)
+    float m = -INFINITY, lsum = 0.f;
+    bool ok = !*abort;
+    for (int t = 0; t < n_tiles && ok; ++t) {
+      // the TMEM loads below are warp-collective: leave only as a whole warp
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[w], t & 1, abort))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[128];
+      tmem_ld_x128(tS, sr);
+      float* s = reinterpret_cast<float*>(sr);
+      const int valid = key_tile(G, l.T, t).valid;
+      if (valid < kRows) {
+#pragma unroll
+        for (int j = 0; j < kRows; ++j)
+          if (j >= valid) s[j] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int j = 1; j < kRows; ++j) mx = fmaxf(mx, s[j]);
+      const float mc = mx * sl2;
+      if (t == 0) {
+        m = mc;
+      } else {
+        const bool need = mc > m + 8.f;
+        if (__any_sync(0xffffffffu, need)) {
+          const float f = need ? ex2(m - mc) : 1.f;
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld_x32(tO + c0, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+            tmem_st_x32(tO + c0, o);
+          }
+          if (need) {
+            lsum *= f;
+            m = mc;
+          }
+        }
+      }
+      const float nm = -m;
+      uint32_t p[64];
+      float rs = 0.f;
+#pragma unroll
+      for (int j = 0; j < 64; ++j) {
+        const float a = ex2(fmaf(s[2 * j], sl2, nm));
+        const float c = ex2(fmaf(s[2 * j + 1], sl2, nm));
+        rs += a + c;
+        p[j] = pack_bf16(a, c);
+      }
+      lsum += rs;
+      tmem_st_x64(tS, p);
+      tc_fence_before();
+      mbar_arrive(&bars->p_full[w]);
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_full, 0, abort));
+    if (ok) {
+      tc_fence_after();
+      const int grow = r0 + kRows * w + row;
+      const bool store = grow < G.q0 + G.nq;
+      const float inv = 1.f / lsum;
+      const long long base = (((long long)b * l.L() + grow) * l.H + h) * D;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        tmem_ld_x32(tO + c0, o);
+        if (store) {
+          if (out_f32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + base + c0);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
+                                   __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + base + c0);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(pack_bf16(__uint_as_float(o[8 * i]) * inv, __uint_as_float(o[8 * i + 1]) * inv),
+                                  pack_bf16(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv),
+                                  pack_bf16(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv),
+                                  pack_bf16(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv));
+          }
+        }
+      }
+      if (store && lse) lse[((long long)b * l.L() + grow) * l.H + h] = (m + log2f(lsum)) * 0.6931471805599453f;
+    }
+  }
+  __syncwarp();  // elected lanes rejoin their warps
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// ------------------------------------------------------------------- host
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 4-D map over a [B, rows, H, D] bf16 tensor: dims (D, H, rows, B), box
+// (64, 1, 128, 1), 128-byte swizzle; rows past the end read as zero.
+bool make_map(CUtensorMap* m, const void* base, int D, int H, long long rows, int B) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)rows * H * D * 2};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)kRows, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t launch_tc_t(const Layout& l, const void* q, const void* k, const void* v,
+                        const void* kt, const void* vt, void* o, bool out_f32, float* lse,
+                        cudaStream_t st) {
+  CUtensorMap mq, mk, mv, mkt, mvt;
+  const long long L = l.L();
+  if (!make_map(&mq, q, D, l.H, L, l.B) || !make_map(&mk, k, D, l.H, L, l.B) ||
+      !make_map(&mv, v, D, l.H, L, l.B))
+    return cudaErrorInvalidValue;
+  if (l.T > 0) {
+    if (!make_map(&mkt, kt, D, l.H, l.T, l.B) || !make_map(&mvt, vt, D, l.H, l.T, l.B))
+      return cudaErrorInvalidValue;
+  } else {
+    mkt = mk;  // never read: no text tiles
+    mvt = mv;
+  }
+  auto kern = window_tc_kernel<D>;
+  const int smem = Cfg<D>::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(tiles_per_head(l, 2 * kRows), l.H, l.B);
+  if (grid.x == 0) return cudaSuccess;
+  kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, mkt, mvt, l, o, out_f32 ? 1 : 0, lse);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool window_tc_supported(const Layout& l, int dtype) {
+  return dtype == VDN_BF16 && (l.d == 64 || l.d == 128);
+}
+
+cudaError_t launch_window_tc(const Layout& l, const void* q, const void* k, const void* v,
+                             const void* kt, const void* vt, void* o, bool out_f32, float* lse,
+                             cudaStream_t st) {
+  if (l.d == 128) return launch_tc_t<128>(l, q, k, v, kt, vt, o, out_f32, lse, st);
+  if (l.d == 64) return launch_tc_t<64>(l, q, k, v, kt, vt, o, out_f32, lse, st);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace vdn
