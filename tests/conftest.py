@@ -28,14 +28,16 @@ def relerr():
     return rel_err
 
 
-def bf16_storage_ratio(got, ref, allowance=4e-3):
+def bf16_storage_ratio(got, ref, allowance=4e-3, rms=None):
     """Worst ratio of |got - ref| to the error a bf16-stored result can carry:
     half a bf16 ulp of the exact value (2^-8 |ref|, rounding to 8 significant
-    bits) plus an accumulation allowance times RMS(ref). <= 1 passes."""
+    bits) plus an accumulation allowance times an RMS (of ref unless given).
+    <= 1 passes."""
     import numpy as np
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     m = ~np.isnan(ref)
-    rms = np.sqrt(np.mean(ref[m] ** 2))
+    if rms is None:
+        rms = np.sqrt(np.mean(ref[m] ** 2))
     bound = 2.0 ** -8 * np.abs(ref[m]) + allowance * max(rms, 1e-300)
     return float(np.max(np.abs(got[m] - ref[m]) / bound))

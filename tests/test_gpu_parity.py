@@ -7,7 +7,8 @@ bf16, whose rounding alone (half an ulp, up to 2^-8 |x|) puts max|err|/RMS at
 1.4e-2 .. 2.4e-2 on these distributions (measured by rounding the oracle's own
 output), above the 2e-2 target on some layouts. So every bf16 result (out,
 o_soft, o_lin, the gated branches) is held per element to half a bf16 ulp of
-the exact value plus 1e-2 RMS: half the 2e-2 target for everything beyond the
+the exact value plus 1e-2 RMS (of `out` for its two gated summands, of the
+result itself otherwise): half the 2e-2 target for everything beyond the
 storage rounding, which leaves room for the softmax weights P entering the
 tensor cores in bf16 (about 2^-9 relative each; the observed excess is
 0.5e-2 .. 0.8e-2 RMS at the maximum). The raw max|err|/RMS is printed. The
@@ -95,10 +96,12 @@ def _check_all(layout, dtype, inp, heads=None, rows=None):
     res = {}
     comp = {"out": (out, ref_out), "o_soft": (o_soft, ref_soft), "o_lin": (o_lin, ref_lin),
             "out_soft": (out_soft, ref_gs), "out_lin": (out_lin, ref_gl)}
+    rms_out = float(np.sqrt(np.nanmean(ref_out ** 2)))
     for key, (g, r) in comp.items():
         res[key] = rel_err(_np(g, hsel), r)
         if dtype == "bf16":
-            res[key + "_storage_ratio"] = bf16_storage_ratio(_np(g, hsel), r, allowance=1e-2)
+            scale = rms_out if key in ("out_soft", "out_lin") else None
+            res[key + "_storage_ratio"] = bf16_storage_ratio(_np(g, hsel), r, allowance=1e-2, rms=scale)
     res["lse"] = float(np.nanmax(np.abs(lse.cpu().double().numpy()[:, :, hsel] - ref_lse)))
     np.testing.assert_allclose(_np(out_soft, hsel) + _np(out_lin, hsel), _np(out, hsel),
                                atol=tol * 4 * np.sqrt(np.mean(_np(out, hsel) ** 2)))
