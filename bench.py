@@ -1,7 +1,7 @@
 """Benchmark of the VDN hybrid video-video attention forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload 768p-bf16]
+                    [--workload 768p-bf16] [--entry hybrid|window|vda]
 
 A step is one vdn_hybrid_attn_fwd call (window softmax + VDA scans + readout,
 norm, gates) over one 768p-like layer input (B=1, H=40, d=128, F=36 frames of
@@ -12,6 +12,11 @@ For N > 1 (launched by torchrun) every rank runs its own independent layer
 input (weak scaling, no collective in the data path); the timed region is
 bracketed by a barrier and device synchronisation on every rank and the
 reported time is the maximum over ranks.
+
+--entry selects the public entry point that forms the step: the hybrid
+forward (default, the headline), or the softmax branch or the linear branch
+alone (vdn_window_softmax_fwd / vdn_vda_scan_fwd), for per-branch numbers and
+for profiling one kernel family at a time.
 
 Printed on rank 0: one JSON line with the throughput (video tokens/s over all
 ranks), the roofline of the dominant kernel (window softmax, tensor-core bound),
@@ -373,6 +378,79 @@ def run_ours(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def vda_bytes(lay) -> float:
+    """Algorithmic HBM bytes of vdn_vda_scan_fwd: k, v and beta of the scanned
+    frames and the text, q read and o_lin written once, the chunk table."""
+    from linear_attention_video_block_b200.synth import Layout  # noqa: F401
+    F, N, T, c, H, d, B = lay.F, lay.N, lay.T, lay.c, lay.H, lay.d, lay.B
+    J = -(-F // c)
+    fwd_max, rev_min = 0, F - 1
+    for j in range(J):
+        f0, f1 = max(j * c, 1), min((j + 1) * c - 1, F - 2)
+        if f1 < f0:
+            continue
+        lo, hi = max(0, c * (j - 1)), min(F - 1, c * (j + 2) - 1)
+        fwd_max = max(fwd_max, lo - 1 if lo - 1 >= 1 else 0)
+        rev_min = min(rev_min, hi + 1 if hi + 1 <= F - 2 else F - 1)
+    frames = set(range(1, fwd_max + 1)) | set(range(rev_min, F - 1))
+    tok = len(frames) * N + T
+    per_bh = tok * (2 * d * 2 + 4) + 2 * F * N * d * 2 + 2 * J * d * d * 4
+    return float(per_bh * H * B)
+
+
+def run_entry(args, rank, world, local_rank):
+    """One branch entry point as the step (no e2e / CPU baseline legs)."""
+    import torch
+    from linear_attention_video_block_b200 import vdn
+    from linear_attention_video_block_b200.synth import WORKLOADS, make_inputs
+
+    lay, dtype, seed = WORKLOADS[args.workload]
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    inp = make_inputs(lay, dtype, seed + rank, device=str(dev))
+    out = torch.empty_like(inp["q"])
+    ws = torch.empty(vdn.workspace_bytes(lay, inp["q"].dtype), dtype=torch.uint8, device=dev)
+    if args.entry == "window":
+        def step():
+            vdn.window_softmax_fwd(lay, inp["q"], inp["k"], inp["v"], inp["k_text"], inp["v_text"],
+                                   o_soft=out)
+    else:
+        def step():
+            vdn.vda_scan_fwd(lay, inp["q"], inp["k"], inp["v"], inp["k_text"], inp["v_text"],
+                             inp["beta"], inp["beta_text"], o_lin=out, workspace=ws)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    assert vdn.device_status() == 0
+    ms = e0.elapsed_time(e1) / args.steps
+    if rank != 0:
+        return
+    peaks, kind = load_peaks()
+    if args.entry == "window":
+        work, unit, peak = window_flops(lay) / 1e12, "TFLOP/s", float(peaks["bf16_tflops"])
+        bound = "tensor"
+    else:
+        work, unit, peak = vda_bytes(lay) / 1e9, "GB/s", float(peaks["hbm_gbs"])
+        bound = "hbm"
+    ach = work / (ms * 1e-3)
+    print(json.dumps({
+        "impl": "ours", "entry": args.entry, "metric": f"{args.entry} fwd video tokens/s",
+        "value": lay.L * lay.B / (ms * 1e-3), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "dtype": dtype,
+        "config": config_of(args.workload, lay),
+        "roofline": {"bound": bound, "achieved": ach, "peak": peak, "unit": unit,
+                     "frac": ach / peak, "peak_source": kind},
+    }), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -380,7 +458,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="768p-bf16")
-    ap.add_argument("--ref-rows", type=int, default=16,
+    ap.add_argument("--entry", choices=["hybrid", "window", "vda"], default="hybrid")
+    ap.add_argument("--ref-rows", type=int, default=96,
                     help="query rows per frame in the oracle's bounded sample")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -398,7 +477,10 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        run_ours(args, rank, world, local_rank)
+        if args.entry == "hybrid":
+            run_ours(args, rank, world, local_rank)
+        else:
+            run_entry(args, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -50,6 +50,9 @@ WORKLOADS = {
     "480p-bf16": (Layout(B=1, F=21, N=1560, T=256, c=5, H=24, d=128), "bf16", 2),
     "768p-bf16": (Layout(B=1, F=36, N=4032, T=512, c=5, H=40, d=128), "bf16", 3),
     "long-bf16": (Layout(B=1, F=90, N=4032, T=512, c=5, H=40, d=128), "bf16", 4),
+    # profiling case: the 768p-like token grid with 4 heads (inputs 149 MB per
+    # video tensor, above the 126 MB L2, a few GB on the device in total)
+    "768p-h4-bf16": (Layout(B=1, F=36, N=4032, T=512, c=5, H=4, d=128), "bf16", 3),
 }
 
 TORCH_DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16}
