@@ -81,7 +81,8 @@ extern "C" {
 
 size_t vdn_workspace_bytes(const vdn_layout_t* layout, int dtype) {
   if (!layout_ok(layout) || !dtype_d_ok(dtype, layout->d)) return 0;
-  return carve(to_layout(layout), dtype, nullptr, true, true).bytes;
+  const Layout l = to_layout(layout);
+  return carve(l, dtype, nullptr, true, !vdn::window_tc_supported(l, dtype)).bytes;
 }
 
 int vdn_window_softmax_fwd(const vdn_layout_t* layout, int dtype, const void* q, const void* k,
@@ -142,15 +143,21 @@ int vdn_hybrid_attn_fwd(const vdn_layout_t* layout, int dtype, const void* q, co
   if (layout->T > 0 && (!aligned16(k_text) || !aligned16(v_text) || !aligned16(beta_text)))
     return VDN_ERR_UNSUPPORTED;
   const Layout l = to_layout(layout);
-  const Workspace need = carve(l, dtype, nullptr, true, true);
+  // The tcgen05 path fuses readout, norm and gates into the window kernel and
+  // needs no o_soft intermediate; the CUDA-core path keeps it in fp32.
+  const bool fused = vdn::window_tc_supported(l, dtype);
+  const Workspace need = carve(l, dtype, nullptr, true, !fused);
   if (!workspace || workspace_bytes < need.bytes) return VDN_ERR_WORKSPACE;
-  const Workspace w = carve(l, dtype, workspace, true, true);
+  const Workspace w = carve(l, dtype, workspace, true, !fused);
   const void* kt = layout->T ? k_text : nullptr;
   const void* vt = layout->T ? v_text : nullptr;
   const float* bt = layout->T ? beta_text : nullptr;
-  int s = run_window(l, dtype, q, k, v, kt, vt, w.o_soft, true, nullptr, stream);
+  int s = cuda_status(vdn::launch_vda_states(l, dtype, k, v, kt, vt, beta, bt, w.am, w.bw, w.states, stream));
   if (s != VDN_OK) return s;
-  s = cuda_status(vdn::launch_vda_states(l, dtype, k, v, kt, vt, beta, bt, w.am, w.bw, w.states, stream));
+  if (fused)
+    return cuda_status(vdn::launch_hybrid_tc(l, q, k, v, kt, vt, w.states, g_soft, g_lin, rms_weight,
+                                             rms_eps, out, out_soft, out_lin, stream));
+  s = run_window(l, dtype, q, k, v, kt, vt, w.o_soft, true, nullptr, stream);
   if (s != VDN_OK) return s;
   return cuda_status(vdn::launch_readout(l, dtype, 1, q, w.states, w.o_soft, g_soft, g_lin,
                                          rms_weight, rms_eps, out, out_soft, out_lin, stream));

@@ -141,6 +141,14 @@ cudaError_t launch_window_tc(const Layout& l, const void* q, const void* k, cons
                              const void* kt, const void* vt, void* o, bool out_f32, float* lse,
                              cudaStream_t st);
 
+// tcgen05 window softmax with the hybrid epilogue fused (bf16, d in {64, 128}):
+// needs the chunk read states first; writes out (and optionally the two gated
+// branches) directly.
+cudaError_t launch_hybrid_tc(const Layout& l, const void* q, const void* k, const void* v,
+                             const void* kt, const void* vt, const float* states, const void* gs,
+                             const void* gl, const float* rms_w, float eps, void* out,
+                             void* out_soft, void* out_lin, cudaStream_t st);
+
 // Reads and clears the device status word of the tcgen05 kernels' translation
 // unit (bounded waits record VDN_ERR_TIMEOUT there).
 cudaError_t read_and_clear_tc_status(int* status);

@@ -10,12 +10,19 @@
 // each segment is partially masked.
 //
 // CTA = 256 query rows (two 128-row Q tiles) of one query group of one
-// (b, h); 320 threads:
+// (b, h); 384 threads:
 //   warps 0-3   softmax warpgroup of Q tile 0 (thread i owns row i = TMEM lane i)
 //   warps 4-7   softmax warpgroup of Q tile 1
 //   warp  8     TMA producer (one elected lane): Q once, then K_t, V_t tiles
 //               into a ring of shared-memory slots
 //   warp  9     MMA issuer (one elected lane) and TMEM owner
+//   warps 10-11 hybrid epilogue helpers (fused variant only): stage the chunk's
+//               VDA read state S_sum = S_fwd + S_rev in shared memory as a bf16
+//               K-major operand while the mainloop runs
+// Fused hybrid variant (project page, "Gating the Softmax and Linear Branch
+// Outputs"): after the last P.V the MMA issuer computes O_lin = Q S_sum^T into
+// the freed S columns of TMEM, and each softmax thread, owning a whole row,
+// finishes out = sigmoid(g_s) o_soft + sigmoid(g_l) RMSNorm(o_lin) in registers.
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+d) O1 [256+d,256+2d).
 // P (bf16) overwrites the first 64 columns of S and is the A operand of P.V
 // straight from TMEM. MMA issue order per key tile t:
@@ -49,7 +56,7 @@ cudaError_t read_and_clear_tc_status(int* status) {
 namespace {
 
 constexpr int kRows = 128;           // rows of a Q tile = keys of a K/V tile
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kTmemCols = 512;
@@ -62,7 +69,8 @@ struct Cfg {
   static constexpr int kHalfBytes = kRows * 128;       // one 128-row x 64-column atom column
   static constexpr int kSlots = (D == 128) ? 4 : 8;
   static constexpr int kQBytes = 2 * kTileBytes;
-  static constexpr int kSmemBytes = 1024 + kQBytes + kSlots * kTileBytes + 256;
+  static constexpr int kSsumBytes = kRows * D * 2;     // bf16 S_sum, 128 x D (fused only)
+  static constexpr int kSmemBytes = 1024 + kQBytes + kSlots * kTileBytes + kSsumBytes + 256;
 };
 
 struct Bars {
@@ -72,6 +80,7 @@ struct Bars {
   unsigned long long s_full[2];
   unsigned long long p_full[2];
   unsigned long long o_full;
+  unsigned long long ssum_ready;
   uint32_t tmem_base;
   int abort;
 };
@@ -277,19 +286,36 @@ __device__ __forceinline__ KeyTile key_tile(const Group& G, int T, int t) {
 
 // ------------------------------------------------------------------ kernel
 
-template <int D>
+// Extra arguments of the fused hybrid epilogue.
+struct HybridArgs {
+  const float* states;             // [B, H, 2, J, D, D] fp32 chunk read states
+  const __nv_bfloat16* g_soft;     // [B, L, H, D]
+  const __nv_bfloat16* g_lin;      // [B, L, H, D]
+  const float* rms_w;              // [D] or null
+  float eps;
+  __nv_bfloat16* out;              // [B, L, H, D]
+  __nv_bfloat16* out_soft;         // nullable
+  __nv_bfloat16* out_lin;          // nullable
+};
+
+__device__ __forceinline__ float sigmoid_fast(float x) {
+  return 1.f / (1.f + ex2(-1.4426950408889634f * x));
+}
+
+template <int D, bool kFuse>
 __global__ void __launch_bounds__(kThreads, 1)
 window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kt,
                  const __grid_constant__ CUtensorMap tm_vt, const Layout l, void* out, int out_f32,
-                 float* lse) {
+                 float* lse, const HybridArgs hy) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = smem;
   uint8_t* sKV = smem + C::kQBytes;
-  Bars* bars = reinterpret_cast<Bars*>(sKV + C::kSlots * C::kTileBytes);
+  uint8_t* sSsum = sKV + C::kSlots * C::kTileBytes;
+  Bars* bars = reinterpret_cast<Bars*>(sSsum + (kFuse ? C::kSsumBytes : 0));
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -298,6 +324,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   tile_to_group(l, 2 * kRows, blockIdx.x, g, r0);
   const Group G = make_group(l, g < 0 ? 0 : g);
   const int n_tiles = key_tile_count(G, l.T);
+  const bool has_lin = kFuse && G.chunk >= 0;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -310,6 +337,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       mbar_init(&bars->p_full[w], 128);
     }
     mbar_init(&bars->o_full, 1);
+    mbar_init(&bars->ssum_ready, 64);
     bars->abort = (g < 0) ? 1 : 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -333,7 +361,6 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int hf = 0; hf < C::kHalves; ++hf)
           tma_load_4d(sQ + qt * C::kTileBytes + hf * C::kHalfBytes, &tm_q, &bars->q_full, hf * 64,
                       h, r0 + qt * kRows, b);
-      int fills[8] = {0, 0, 0, 0, 0, 0, 0, 0};
       int fill = 0;
       bool ok = true;
       for (int t = 0; t < n_tiles && ok; ++t) {
@@ -350,14 +377,16 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           for (int hf = 0; hf < C::kHalves; ++hf)
             tma_load_4d(sKV + slot * C::kTileBytes + hf * C::kHalfBytes, map, &bars->kv_full[slot],
                         hf * 64, h, kt.row, b);
-          fills[slot] = use + 1;
         }
       }
       if (!ok) {
-        // leave no copy in flight into this CTA's shared memory
+        // leave no copy in flight into this CTA's shared memory: the last fill
+        // of slot s was number (fill - 1 - ((fill - 1 - s) mod kSlots))
         mbar_wait(&bars->q_full, 0, abort, false);
-        for (int s = 0; s < C::kSlots; ++s)
-          if (fills[s] > 0) mbar_wait(&bars->kv_full[s], (fills[s] - 1) & 1, abort, false);
+        for (int s = 0; s < C::kSlots && s < fill; ++s) {
+          const int last = fill - 1 - ((fill - 1 - s) % C::kSlots);
+          mbar_wait(&bars->kv_full[s], (last / C::kSlots) & 1, abort, false);
+        }
       }
     }
   } else if (warp == kMmaWarp) {
@@ -365,8 +394,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       // ------------------------------------------------------- MMA issuer
       constexpr uint32_t idesc_s = make_idesc(kRows, false);
       constexpr uint32_t idesc_o = make_idesc(D, true);
-      const uint32_t tS[2] = {tmem, tmem + 128};
-      const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
+      constexpr uint32_t idesc_lin = make_idesc(D, false);
       const uint32_t q_addr = smem_u32(sQ);
       const uint32_t kv_addr = smem_u32(sKV);
       int use = 0;
@@ -379,17 +407,20 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         return r;
       };
       auto issue_s = [&](int w, int slot) {
+        const uint32_t d_tmem = tmem + 128 * w;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (uint32_t)((ks / 4) * C::kHalfBytes + (ks % 4) * 32);
-          mma_ss(tS[w], desc_k_sw128(q_addr + w * C::kTileBytes + off),
+          mma_ss(d_tmem, desc_k_sw128(q_addr + w * C::kTileBytes + off),
                  desc_k_sw128(kv_addr + slot * C::kTileBytes + off), idesc_s, ks > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int w, int slot, bool acc) {
+        const uint32_t d_tmem = tmem + 256 + D * w;
+        const uint32_t a_tmem = tmem + 128 * w;
 #pragma unroll
         for (int ks = 0; ks < kRows / 16; ++ks) {
-          mma_ts(tO[w], tS[w] + ks * 8,
+          mma_ts(d_tmem, a_tmem + ks * 8,
                  desc_mn_sw128(kv_addr + slot * C::kTileBytes + ks * 16 * 128, C::kHalfBytes),
                  idesc_o, (acc || ks > 0) ? 1u : 0u);
         }
@@ -397,7 +428,6 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       int ks_cur = 0;
       if (ok) ok = take_slot(ks_cur);
       if (ok) {
-        tc_fence_after();
         issue_s(0, ks_cur);
         tc_commit(&bars->s_full[0]);
         issue_s(1, ks_cur);
@@ -426,9 +456,48 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           tc_commit(&bars->kv_empty[ks_next]);
         }
       }
+      if (ok && has_lin) {
+        // O_lin_w = Q_w S_sum^T into the S columns of TMEM (issued after the last
+        // P.V, which reads P from those columns; tcgen05.mma runs in issue order)
+        ok = mbar_wait(&bars->ssum_ready, 0, abort);
+        if (ok) {
+          tc_fence_after();
+          const uint32_t s_addr = smem_u32(sSsum);
+          for (int w = 0; w < 2; ++w) {
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+              const uint32_t off = (uint32_t)((ks / 4) * C::kHalfBytes + (ks % 4) * 32);
+              mma_ss(tmem + 128 * w, desc_k_sw128(q_addr + w * C::kTileBytes + off),
+                     desc_k_sw128(s_addr + off), idesc_lin, ks > 0 ? 1u : 0u);
+            }
+          }
+        }
+      }
       tc_commit(&bars->o_full);
       // every MMA issued must finish before TMEM is freed
       if (!ok) mbar_wait(&bars->o_full, 0, abort, false);
+    }
+  } else if (warp >= 10) {
+    // ---------------------------------------------- S_sum staging (fused)
+    if (has_lin && !*abort) {
+      const int t = threadIdx.x - 320;
+      const int J = l.J();
+      const float* sf = hy.states + ((((long long)b * l.H + h) * 2 + 0) * J + G.chunk) * D * D;
+      const float* sr = hy.states + ((((long long)b * l.H + h) * 2 + 1) * J + G.chunk) * D * D;
+      constexpr int kChunks = D / 8;  // 16-byte chunks per row
+      for (int ch = t; ch < kRows * kChunks; ch += 64) {
+        const int n = ch / kChunks, kc = ch % kChunks;
+        const float4 a0 = *reinterpret_cast<const float4*>(sf + n * D + kc * 8);
+        const float4 a1 = *reinterpret_cast<const float4*>(sf + n * D + kc * 8 + 4);
+        const float4 b0 = *reinterpret_cast<const float4*>(sr + n * D + kc * 8);
+        const float4 b1 = *reinterpret_cast<const float4*>(sr + n * D + kc * 8 + 4);
+        const uint4 v = make_uint4(pack_bf16(a0.x + b0.x, a0.y + b0.y), pack_bf16(a0.z + b0.z, a0.w + b0.w),
+                                   pack_bf16(a1.x + b1.x, a1.y + b1.y), pack_bf16(a1.z + b1.z, a1.w + b1.w));
+        const int half = kc / 8, c16 = kc % 8;
+        *reinterpret_cast<uint4*>(sSsum + half * C::kHalfBytes + n * 128 + ((c16 ^ (n & 7)) * 16)) = v;
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(&bars->ssum_ready);
     }
   } else {
     // ----------------------------------------------------------- softmax
@@ -456,10 +525,15 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int j = 0; j < kRows; ++j)
           if (j >= valid) s[j] = -INFINITY;
       }
-      float mx = s[0];
+      float mx4[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-      for (int j = 1; j < kRows; ++j) mx = fmaxf(mx, s[j]);
-      const float mc = mx * sl2;
+      for (int j = 4; j < kRows; j += 4) {
+        mx4[0] = fmaxf(mx4[0], s[j]);
+        mx4[1] = fmaxf(mx4[1], s[j + 1]);
+        mx4[2] = fmaxf(mx4[2], s[j + 2]);
+        mx4[3] = fmaxf(mx4[3], s[j + 3]);
+      }
+      const float mc = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
       if (t == 0) {
         m = mc;
       } else {
@@ -482,15 +556,15 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
       const float nm = -m;
       uint32_t p[64];
-      float rs = 0.f;
+      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int j = 0; j < 64; ++j) {
         const float a = ex2(fmaf(s[2 * j], sl2, nm));
         const float c = ex2(fmaf(s[2 * j + 1], sl2, nm));
-        rs += a + c;
+        rs4[j & 3] += a + c;
         p[j] = pack_bf16(a, c);
       }
-      lsum += rs;
+      lsum += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
       tmem_st_x64(tS, p);
       tc_fence_before();
       mbar_arrive(&bars->p_full[w]);
@@ -502,29 +576,92 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const bool store = grow < G.q0 + G.nq;
       const float inv = 1.f / lsum;
       const long long base = (((long long)b * l.L() + grow) * l.H + h) * D;
+      if constexpr (!kFuse) {
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t o[32];
-        tmem_ld_x32(tO + c0, o);
-        if (store) {
-          if (out_f32) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + base + c0);
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld_x32(tO + c0, o);
+          if (store) {
+            if (out_f32) {
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + base + c0);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
-                                   __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
-          } else {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + base + c0);
+              for (int i = 0; i < 8; ++i)
+                dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
+                                     __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + base + c0);
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              dst[i] = make_uint4(pack_bf16(__uint_as_float(o[8 * i]) * inv, __uint_as_float(o[8 * i + 1]) * inv),
-                                  pack_bf16(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv),
-                                  pack_bf16(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv),
-                                  pack_bf16(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv));
+              for (int i = 0; i < 4; ++i)
+                dst[i] = make_uint4(pack_bf16(__uint_as_float(o[8 * i]) * inv, __uint_as_float(o[8 * i + 1]) * inv),
+                                    pack_bf16(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv),
+                                    pack_bf16(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv),
+                                    pack_bf16(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv));
+            }
+          }
+        }
+        if (store && lse) lse[((long long)b * l.L() + grow) * l.H + h] = (m + log2f(lsum)) * 0.6931471805599453f;
+      } else {
+        // RMSNorm statistic of o_lin (whole row in this thread)
+        float rstd = 0.f;
+        if (has_lin) {
+          float ss4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld_x32(tS + c0, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float x = __uint_as_float(o[i]);
+              ss4[i & 3] = fmaf(x, x, ss4[i & 3]);
+            }
+          }
+          rstd = rsqrtf(((ss4[0] + ss4[1]) + (ss4[2] + ss4[3])) / (float)D + hy.eps);
+        }
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t os[32], ol[32];
+          tmem_ld_x32(tO + c0, os);
+          if (has_lin) tmem_ld_x32(tS + c0, ol);
+          if (store) {
+            const uint4* gsp = reinterpret_cast<const uint4*>(hy.g_soft + base + c0);
+            const uint4* glp = reinterpret_cast<const uint4*>(hy.g_lin + base + c0);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) {
+              const uint4 gs4 = gsp[v4];
+              const uint4 gl4 = glp[v4];
+              const uint32_t gsw[4] = {gs4.x, gs4.y, gs4.z, gs4.w};
+              const uint32_t glw[4] = {gl4.x, gl4.y, gl4.z, gl4.w};
+              uint32_t ow[4], osw[4], olw[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                float r2[2], a2[2], b2[2];
+#pragma unroll
+                for (int k2 = 0; k2 < 2; ++k2) {
+                  const int i = v4 * 8 + e * 2 + k2;
+                  const float gsv = __uint_as_float(k2 ? (gsw[e] & 0xFFFF0000u) : (gsw[e] << 16));
+                  const float glv = __uint_as_float(k2 ? (glw[e] & 0xFFFF0000u) : (glw[e] << 16));
+                  a2[k2] = sigmoid_fast(gsv) * (__uint_as_float(os[i]) * inv);
+                  float lin = 0.f;
+                  if (has_lin) {
+                    const float wv = hy.rms_w ? hy.rms_w[c0 + i] : 1.f;
+                    lin = sigmoid_fast(glv) * (__uint_as_float(ol[i]) * rstd * wv);
+                  }
+                  b2[k2] = lin;
+                  r2[k2] = a2[k2] + lin;
+                }
+                ow[e] = pack_bf16(r2[0], r2[1]);
+                osw[e] = pack_bf16(a2[0], a2[1]);
+                olw[e] = pack_bf16(b2[0], b2[1]);
+              }
+              reinterpret_cast<uint4*>(hy.out + base + c0)[v4] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+              if (hy.out_soft)
+                reinterpret_cast<uint4*>(hy.out_soft + base + c0)[v4] = make_uint4(osw[0], osw[1], osw[2], osw[3]);
+              if (hy.out_lin)
+                reinterpret_cast<uint4*>(hy.out_lin + base + c0)[v4] = make_uint4(olw[0], olw[1], olw[2], olw[3]);
+            }
           }
         }
       }
-      if (store && lse) lse[((long long)b * l.L() + grow) * l.H + h] = (m + log2f(lsum)) * 0.6931471805599453f;
     }
   }
   __syncwarp();  // elected lanes rejoin their warps
@@ -566,10 +703,10 @@ bool make_map(CUtensorMap* m, const void* base, int D, int H, long long rows, in
   return r == CUDA_SUCCESS;
 }
 
-template <int D>
+template <int D, bool kFuse>
 cudaError_t launch_tc_t(const Layout& l, const void* q, const void* k, const void* v,
                         const void* kt, const void* vt, void* o, bool out_f32, float* lse,
-                        cudaStream_t st) {
+                        const HybridArgs& hy, cudaStream_t st) {
   CUtensorMap mq, mk, mv, mkt, mvt;
   const long long L = l.L();
   if (!make_map(&mq, q, D, l.H, L, l.B) || !make_map(&mk, k, D, l.H, L, l.B) ||
@@ -582,13 +719,13 @@ cudaError_t launch_tc_t(const Layout& l, const void* q, const void* k, const voi
     mkt = mk;  // never read: no text tiles
     mvt = mv;
   }
-  auto kern = window_tc_kernel<D>;
-  const int smem = Cfg<D>::kSmemBytes;
+  auto kern = window_tc_kernel<D, kFuse>;
+  const int smem = Cfg<D>::kSmemBytes - (kFuse ? 0 : Cfg<D>::kSsumBytes);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(tiles_per_head(l, 2 * kRows), l.H, l.B);
   if (grid.x == 0) return cudaSuccess;
-  kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, mkt, mvt, l, o, out_f32 ? 1 : 0, lse);
+  kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, mkt, mvt, l, o, out_f32 ? 1 : 0, lse, hy);
   return cudaGetLastError();
 }
 
@@ -601,8 +738,27 @@ bool window_tc_supported(const Layout& l, int dtype) {
 cudaError_t launch_window_tc(const Layout& l, const void* q, const void* k, const void* v,
                              const void* kt, const void* vt, void* o, bool out_f32, float* lse,
                              cudaStream_t st) {
-  if (l.d == 128) return launch_tc_t<128>(l, q, k, v, kt, vt, o, out_f32, lse, st);
-  if (l.d == 64) return launch_tc_t<64>(l, q, k, v, kt, vt, o, out_f32, lse, st);
+  HybridArgs hy{};
+  if (l.d == 128) return launch_tc_t<128, false>(l, q, k, v, kt, vt, o, out_f32, lse, hy, st);
+  if (l.d == 64) return launch_tc_t<64, false>(l, q, k, v, kt, vt, o, out_f32, lse, hy, st);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_hybrid_tc(const Layout& l, const void* q, const void* k, const void* v,
+                             const void* kt, const void* vt, const float* states, const void* gs,
+                             const void* gl, const float* rms_w, float eps, void* out,
+                             void* out_soft, void* out_lin, cudaStream_t st) {
+  HybridArgs hy;
+  hy.states = states;
+  hy.g_soft = static_cast<const __nv_bfloat16*>(gs);
+  hy.g_lin = static_cast<const __nv_bfloat16*>(gl);
+  hy.rms_w = rms_w;
+  hy.eps = eps;
+  hy.out = static_cast<__nv_bfloat16*>(out);
+  hy.out_soft = static_cast<__nv_bfloat16*>(out_soft);
+  hy.out_lin = static_cast<__nv_bfloat16*>(out_lin);
+  if (l.d == 128) return launch_tc_t<128, true>(l, q, k, v, kt, vt, nullptr, false, nullptr, hy, st);
+  if (l.d == 64) return launch_tc_t<64, true>(l, q, k, v, kt, vt, nullptr, false, nullptr, hy, st);
   return cudaErrorInvalidValue;
 }
 
