@@ -18,10 +18,12 @@
 //   warp  9     MMA issuer (one elected lane) and TMEM owner
 //   warps 10-11 hybrid epilogue helpers (fused variant only): stage the chunk's
 //               VDA read state S_sum = S_fwd + S_rev in shared memory as a bf16
-//               K-major operand while the mainloop runs
+//               K-major operand while the mainloop runs, in two parts
+//               S_hi = bf16(S_sum) and S_lo = bf16(S_sum - S_hi), so that the
+//               readout keeps about 16 significant bits of the fp32 state
 // Fused hybrid variant (project page, "Gating the Softmax and Linear Branch
-// Outputs"): after the last P.V the MMA issuer computes O_lin = Q S_sum^T into
-// the freed S columns of TMEM, and each softmax thread, owning a whole row,
+// Outputs"): after the last P.V the MMA issuer computes O_lin = Q S_hi^T +
+// Q S_lo^T into the freed S columns of TMEM, and each softmax thread, owning a whole row,
 // finishes out = sigmoid(g_s) o_soft + sigmoid(g_l) RMSNorm(o_lin) in registers.
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+d) O1 [256+d,256+2d).
 // P (bf16) overwrites the first 64 columns of S and is the A operand of P.V
@@ -81,6 +83,7 @@ struct Bars {
   unsigned long long p_full[2];
   unsigned long long o_full;
   unsigned long long ssum_ready;
+  unsigned long long ssum_free;
   uint32_t tmem_base;
   int abort;
 };
@@ -338,6 +341,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->ssum_ready, 64);
+    mbar_init(&bars->ssum_free, 1);
     bars->abort = (g < 0) ? 1 : 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -457,20 +461,24 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
       }
       if (ok && has_lin) {
-        // O_lin_w = Q_w S_sum^T into the S columns of TMEM (issued after the last
-        // P.V, which reads P from those columns; tcgen05.mma runs in issue order)
-        ok = mbar_wait(&bars->ssum_ready, 0, abort);
-        if (ok) {
+        // O_lin_w = Q_w S_hi^T + Q_w S_lo^T into the S columns of TMEM (issued after
+        // the last P.V, which reads P from those columns; tcgen05.mma runs in
+        // issue order). The helpers restage S_lo into the same buffer once the
+        // S_hi products have completed.
+        const uint32_t s_addr = smem_u32(sSsum);
+        for (int part = 0; part < 2 && ok; ++part) {
+          ok = mbar_wait(&bars->ssum_ready, part, abort);
+          if (!ok) break;
           tc_fence_after();
-          const uint32_t s_addr = smem_u32(sSsum);
           for (int w = 0; w < 2; ++w) {
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
               const uint32_t off = (uint32_t)((ks / 4) * C::kHalfBytes + (ks % 4) * 32);
               mma_ss(tmem + 128 * w, desc_k_sw128(q_addr + w * C::kTileBytes + off),
-                     desc_k_sw128(s_addr + off), idesc_lin, ks > 0 ? 1u : 0u);
+                     desc_k_sw128(s_addr + off), idesc_lin, (part > 0 || ks > 0) ? 1u : 0u);
             }
           }
+          if (part == 0) tc_commit(&bars->ssum_free);
         }
       }
       tc_commit(&bars->o_full);
@@ -485,19 +493,28 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const float* sf = hy.states + ((((long long)b * l.H + h) * 2 + 0) * J + G.chunk) * D * D;
       const float* sr = hy.states + ((((long long)b * l.H + h) * 2 + 1) * J + G.chunk) * D * D;
       constexpr int kChunks = D / 8;  // 16-byte chunks per row
-      for (int ch = t; ch < kRows * kChunks; ch += 64) {
-        const int n = ch / kChunks, kc = ch % kChunks;
-        const float4 a0 = *reinterpret_cast<const float4*>(sf + n * D + kc * 8);
-        const float4 a1 = *reinterpret_cast<const float4*>(sf + n * D + kc * 8 + 4);
-        const float4 b0 = *reinterpret_cast<const float4*>(sr + n * D + kc * 8);
-        const float4 b1 = *reinterpret_cast<const float4*>(sr + n * D + kc * 8 + 4);
-        const uint4 v = make_uint4(pack_bf16(a0.x + b0.x, a0.y + b0.y), pack_bf16(a0.z + b0.z, a0.w + b0.w),
-                                   pack_bf16(a1.x + b1.x, a1.y + b1.y), pack_bf16(a1.z + b1.z, a1.w + b1.w));
-        const int half = kc / 8, c16 = kc % 8;
-        *reinterpret_cast<uint4*>(sSsum + half * C::kHalfBytes + n * 128 + ((c16 ^ (n & 7)) * 16)) = v;
+      for (int part = 0; part < 2; ++part) {
+        if (part == 1 && !mbar_wait(&bars->ssum_free, 0, abort)) break;
+        for (int ch = t; ch < kRows * kChunks; ch += 64) {
+          const int n = ch / kChunks, kc = ch % kChunks;
+          const float4 a0 = *reinterpret_cast<const float4*>(sf + n * D + kc * 8);
+          const float4 a1 = *reinterpret_cast<const float4*>(sf + n * D + kc * 8 + 4);
+          const float4 b0 = *reinterpret_cast<const float4*>(sr + n * D + kc * 8);
+          const float4 b1 = *reinterpret_cast<const float4*>(sr + n * D + kc * 8 + 4);
+          float x[8] = {a0.x + b0.x, a0.y + b0.y, a0.z + b0.z, a0.w + b0.w,
+                        a1.x + b1.x, a1.y + b1.y, a1.z + b1.z, a1.w + b1.w};
+          if (part == 1) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] -= __bfloat162float(__float2bfloat16_rn(x[e]));
+          }
+          const uint4 v = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]),
+                                     pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
+          const int half = kc / 8, c16 = kc % 8;
+          *reinterpret_cast<uint4*>(sSsum + half * C::kHalfBytes + n * 128 + ((c16 ^ (n & 7)) * 16)) = v;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive(&bars->ssum_ready);
       }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive(&bars->ssum_ready);
     }
   } else {
     // ----------------------------------------------------------- softmax
