@@ -1,0 +1,309 @@
+// Frame Gram matrices of Video Delta Attention on the 5th-generation tensor
+// cores (project page "Video Delta Attention: A Frame-Wise Solution"):
+//   A_f = K_f^T Diag(beta_f) K_f,   B_f = V_f^T Diag(beta_f) K_f
+// over the U tokens of one frame (or of the text, slot 0), fp32 results.
+//
+// CTA = one (b, h, slot); 192 threads:
+//   warp 0     TMA producer: 64-token K and V tiles into a ring of stages
+//   warp 1     MMA issuer (one lane) and TMEM owner
+//   warps 2-5  scalers: write Kw = beta (.) K (bf16) next to K, one token row per
+//              thread (beta = 0 past the frame, which also masks the ragged
+//              last tile); then the epilogue reads A and B out of TMEM.
+// Both MMA operands are MN-major (token = K dimension, contiguous along d):
+//   d = 128: D_A[i][j] += sum_u K[u][i] Kw[u][j] (TMEM columns 0..127) and
+//            D_B[i][j] += sum_u V[u][i] Kw[u][j] (columns 128..255);
+//   d = 64:  one M = 128 MMA with [K^T; V^T] stacked along M (the V tile sits
+//            one leading-byte-offset after the K tile): lanes 0-63 = A, 64-127 = B.
+// The work is HBM-bound: each token's k and v are read once.
+#include "tc_common.cuh"
+
+namespace vdn {
+
+__device__ int g_gram_status = 0;
+
+cudaError_t read_and_clear_gram_status(int* status) {
+  cudaError_t e = cudaMemcpyFromSymbol(status, g_gram_status, sizeof(int));
+  if (e != cudaSuccess) return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_gram_status, &zero, sizeof(int));
+}
+
+namespace {
+
+constexpr int kTok = 64;        // tokens per tile
+constexpr int kThreads = 192;
+constexpr int kHalfBytes = kTok * 128;  // 64 tokens x 64 bf16 (one swizzle atom column)
+
+template <int D>
+struct GCfg {
+  static constexpr int kHalves = D / 64;
+  static constexpr int kTileBytes = kTok * D * 2;
+  static constexpr int kStageBytes = 3 * kTileBytes;          // K, V, Kw
+  static constexpr int kStages = (D == 128) ? 4 : 8;
+  static constexpr int kTmemCols = (D == 128) ? 256 : 64;
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 256;
+};
+
+struct GBars {
+  unsigned long long full[8];
+  unsigned long long scaled[8];
+  unsigned long long empty[8];
+  unsigned long long done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ bool gwait(unsigned long long* bar, uint32_t parity, volatile int* abort,
+                                      bool watch_abort = true) {
+  if (mbar_try_wait(smem_u32(bar), parity)) return true;
+  return mbar_wait_impl(bar, parity, abort, &g_gram_status, watch_abort);
+}
+
+// kind::f16 instruction descriptor with both operands MN-major.
+__host__ __device__ constexpr uint32_t idesc_mn_mn(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) | ((uint32_t)(n >> 3) << 17) |
+         ((uint32_t)(128 >> 4) << 24);
+}
+
+// Slot s -> frame: slot 0 = text (when present), then frames 1..fwd_max, then rev_lo..F-2.
+struct GramSlots {
+  int has_text, fwd_max, rev_lo;
+  __device__ int frame(int i) const {
+    if (has_text) {
+      if (i == 0) return 0;
+      --i;
+    }
+    if (i < fwd_max) return 1 + i;
+    return rev_lo + (i - fwd_max);
+  }
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+               const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUtensorMap tm_vt,
+               const Layout l, const GramSlots slots, const float* __restrict__ beta,
+               const float* __restrict__ beta_t, float* __restrict__ am, float* __restrict__ bw) {
+  using C = GCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  GBars* bars = reinterpret_cast<GBars*>(smem + C::kStages * C::kStageBytes);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const bool text = slots.has_text && blockIdx.x == 0;
+  const int f = slots.frame(blockIdx.x);
+  const int U = text ? l.T : l.N;
+  const int row0 = text ? 0 : f * l.N;         // first token row in the tensor
+  const int n_tiles = (U + kTok - 1) / kTok;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->scaled[s], 128);
+      mbar_init(&bars->empty[s], 1);
+    }
+    mbar_init(&bars->done, 1);
+    bars->abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(smem_u32(&bars->tmem_base)), "r"(C::kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  volatile int* abort = &bars->abort;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ----------------------------------------------------------- producer
+      const CUtensorMap* mk = text ? &tm_kt : &tm_k;
+      const CUtensorMap* mv = text ? &tm_vt : &tm_v;
+      int issued = 0;
+      bool ok = true;
+      for (int t = 0; t < n_tiles; ++t) {
+        const int s = t % C::kStages, use = t / C::kStages;
+        if (use > 0 && !gwait(&bars->empty[s], (use - 1) & 1, abort)) {
+          ok = false;
+          break;
+        }
+        uint8_t* st = smem + s * C::kStageBytes;
+        mbar_expect_tx(&bars->full[s], 2 * C::kTileBytes);
+        for (int hf = 0; hf < C::kHalves; ++hf) {
+          tma_load_4d(st + hf * kHalfBytes, mk, &bars->full[s], hf * 64, h, row0 + t * kTok, b);
+          tma_load_4d(st + C::kTileBytes + hf * kHalfBytes, mv, &bars->full[s], hf * 64, h,
+                      row0 + t * kTok, b);
+        }
+        ++issued;
+      }
+      if (!ok) {
+        // no copy may still be landing when the CTA exits
+        for (int s = 0; s < C::kStages && s < issued; ++s) {
+          const int last = issued - 1 - ((issued - 1 - s) % C::kStages);
+          gwait(&bars->full[s], (last / C::kStages) & 1, abort, false);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      constexpr uint32_t idesc = idesc_mn_mn(D);
+      bool ok = true;
+      for (int t = 0; t < n_tiles && ok; ++t) {
+        const int s = t % C::kStages, use = t / C::kStages;
+        if (!gwait(&bars->scaled[s], use & 1, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t st = smem_u32(smem + s * C::kStageBytes);
+        const uint32_t k_addr = st, v_addr = st + C::kTileBytes, w_addr = st + 2 * C::kTileBytes;
+#pragma unroll
+        for (int ks = 0; ks < kTok / 16; ++ks) {
+          const uint32_t acc = (t > 0 || ks > 0) ? 1u : 0u;
+          const uint32_t koff = ks * 16 * 128;
+          const uint64_t bdesc = desc_mn_sw128(w_addr + koff, kHalfBytes);
+          if (D == 128) {
+            mma_ss(tmem, desc_mn_sw128(k_addr + koff, kHalfBytes), bdesc, idesc, acc);
+            mma_ss(tmem + 128, desc_mn_sw128(v_addr + koff, kHalfBytes), bdesc, idesc, acc);
+          } else {
+            // [K^T; V^T]: the two 64-wide M blocks are the K and V tiles
+            mma_ss(tmem, desc_mn_sw128(k_addr + koff, C::kTileBytes), bdesc, idesc, acc);
+          }
+        }
+        tc_commit(&bars->empty[s]);
+      }
+      tc_commit(&bars->done);
+      if (!ok) gwait(&bars->done, 0, abort, false);
+    }
+  } else {
+    // ---------------------------------------------------- scalers / epilogue
+    const int u = threadIdx.x - 64;  // token row within a tile, 0..127? only 0..63 used
+    bool ok = true;
+    for (int t = 0; t < n_tiles && ok; ++t) {
+      const int s = t % C::kStages, use = t / C::kStages;
+      if (!__all_sync(0xffffffffu, gwait(&bars->full[s], use & 1, abort))) {
+        ok = false;
+        break;
+      }
+      // 128 threads, 64 token rows x kHalves halves: thread -> (row, half pair)
+      uint8_t* st = smem + s * C::kStageBytes;
+      for (int item = u; item < kTok * C::kHalves; item += 128) {
+        const int r = item % kTok, hf = item / kTok;
+        const int tok = t * kTok + r;
+        float bu = 0.f;
+        if (tok < U)
+          bu = text ? beta_t[((long long)b * l.T + tok) * l.H + h]
+                    : beta[((long long)b * l.L() + row0 + tok) * l.H + h];
+        const uint4* src = reinterpret_cast<const uint4*>(st + hf * kHalfBytes + r * 128);
+        uint4* dst = reinterpret_cast<uint4*>(st + 2 * C::kTileBytes + hf * kHalfBytes + r * 128);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint4 x = src[c];
+          uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float lo = __uint_as_float(w[e] << 16) * bu;
+            const float hi = __uint_as_float(w[e] & 0xFFFF0000u) * bu;
+            w[e] = pack_bf16(lo, hi);
+          }
+          dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(&bars->scaled[s]);
+    }
+    if (ok) ok = __all_sync(0xffffffffu, gwait(&bars->done, 0, abort));
+    if (ok) {
+      tc_fence_after();
+      const int m = 32 * (warp & 3) + lane;  // TMEM lane = output row
+      const uint32_t taddr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+      const long long slot = ((long long)b * l.H + h) * l.F + f;
+      float* arow;
+      float* brow;
+      if (D == 128) {
+        arow = am + slot * D * D + (long long)m * D;
+        brow = bw + slot * D * D + (long long)m * D;
+      } else {
+        arow = (m < 64) ? am + slot * D * D + (long long)m * D : bw + slot * D * D + (long long)(m - 64) * D;
+        brow = nullptr;
+      }
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld_x32(taddr + c0, r);
+        float4* dst = reinterpret_cast<float4*>(arow + c0);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          dst[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                               __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+      }
+      if (D == 128) {
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld_x32(taddr + 128 + c0, r);
+          float4* dst = reinterpret_cast<float4*>(brow + c0);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                 __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::kTmemCols)
+                 : "memory");
+  }
+}
+
+template <int D>
+cudaError_t launch_gram_t(const Layout& l, const GramSlots& slots, int nslots, const void* k,
+                          const void* v, const void* kt, const void* vt, const float* beta,
+                          const float* beta_t, float* am, float* bw, cudaStream_t st) {
+  CUtensorMap mk, mv, mkt, mvt;
+  if (!make_map(&mk, k, D, l.H, l.L(), l.B, kTok) || !make_map(&mv, v, D, l.H, l.L(), l.B, kTok))
+    return cudaErrorInvalidValue;
+  if (l.T > 0) {
+    if (!make_map(&mkt, kt, D, l.H, l.T, l.B, kTok) || !make_map(&mvt, vt, D, l.H, l.T, l.B, kTok))
+      return cudaErrorInvalidValue;
+  } else {
+    mkt = mk;
+    mvt = mv;
+  }
+  auto kern = gram_tc_kernel<D>;
+  const int smem = GCfg<D>::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(nslots, l.H, l.B), kThreads, smem, st>>>(mk, mv, mkt, mvt, l, slots, beta, beta_t, am, bw);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool gram_tc_supported(const Layout& l, int dtype) {
+  return dtype == VDN_BF16 && (l.d == 64 || l.d == 128);
+}
+
+cudaError_t launch_gram_tc(const Layout& l, int has_text, int fwd_max, int rev_lo, int nslots,
+                           const void* k, const void* v, const void* kt, const void* vt,
+                           const float* beta, const float* beta_t, float* am, float* bw,
+                           cudaStream_t st) {
+  GramSlots slots{has_text, fwd_max, rev_lo};
+  if (nslots <= 0) return cudaSuccess;
+  if (l.d == 128) return launch_gram_t<128>(l, slots, nslots, k, v, kt, vt, beta, beta_t, am, bw, st);
+  if (l.d == 64) return launch_gram_t<64>(l, slots, nslots, k, v, kt, vt, beta, beta_t, am, bw, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace vdn

@@ -4,8 +4,9 @@
 //
 // Three frame-parallel / lane-parallel phases:
 //   gram     A_f = K_f^T Diag(beta_f) K_f and B_f = V_f^T Diag(beta_f) K_f for
-//            every scanned frame and for the text (slot 0), fp32.
-//   inverse  M_f = (I + A_f)^-1 in place of A_f (Gauss-Jordan in shared memory;
+//            every scanned frame and for the text (slot 0), fp32 (bf16 inputs:
+//            tensor-core kernel in gram_tc.cu; fp32 inputs: CUDA-core kernel here).
+//   inverse  M_f = (I + A_f)^-1 in place of A_f (register-blocked Gauss-Jordan;
 //            I + A_f is SPD with every pivot >= 1, so no pivoting is needed).
 //   scan     S <- (S + B_f) M_f, forward over 1..fwd_max and reverse over
 //            F-2..rev_min, from S0 = 1/2 B_T M_T. Rows of S evolve independently
@@ -111,41 +112,76 @@ gram_kernel(Layout l, SlotMap sm_map, const T* __restrict__ k, const T* __restri
     }
 }
 
-// In-place inverse of (I + A) for one slot: Gauss-Jordan elimination.
+// In-place inverse of (I + A) for one slot: Gauss-Jordan elimination without
+// pivoting (every pivot of an SPD matrix with eigenvalues >= 1 is >= 1).
+// Thread (tr, tc) of a 16 x 16 grid keeps the interleaved block of rows
+// tr + 16a and columns tc + 16c in registers; the pivot row and column of
+// each step go through double-buffered shared memory, one barrier per step.
 template <int D>
 __global__ void __launch_bounds__(NT)
 inverse_kernel(Layout l, SlotMap sm_map, float* __restrict__ am) {
-  extern __shared__ __align__(16) float inv_smem[];
-  float* a = inv_smem;             // [D][D]
-  float* rowk = a + D * D;         // [D]
-  float* colk = rowk + D;          // [D]
+  constexpr int RA = D / 16;
+  __shared__ float rowk[2][D];
+  __shared__ float colk[2][D];
   const int tid = threadIdx.x;
+  const int tr = tid / 16, tc = tid % 16;
   const int h = blockIdx.y, b = blockIdx.z;
   const int f = sm_map.frame(blockIdx.x);
   const long long slot = ((long long)b * l.H + h) * l.F + f;
   float* g = am + slot * D * D;
-  for (int i = tid; i < D * D; i += NT) a[i] = g[i] + ((i / D) == (i % D) ? 1.f : 0.f);
-  for (int kx = 0; kx < D; ++kx) {
-    __syncthreads();
-    const float piv = a[kx * D + kx];
-    const float rp = 1.f / piv;
-    for (int j = tid; j < D; j += NT) {
-      rowk[j] = (j == kx) ? rp : a[kx * D + j] * rp;
-      colk[j] = a[j * D + kx];
+  float a[RA][RA];
+#pragma unroll
+  for (int x = 0; x < RA; ++x)
+#pragma unroll
+    for (int y = 0; y < RA; ++y) {
+      const int i = tr + 16 * x, j = tc + 16 * y;
+      a[x][y] = g[i * D + j] + (i == j ? 1.f : 0.f);
     }
-    __syncthreads();
-    for (int i = tid; i < D * D; i += NT) {
-      int r = i / D, cidx = i % D;
-      if (r == kx) {
-        a[i] = rowk[cidx];
-      } else {
-        float base = (cidx == kx) ? 0.f : a[i];
-        a[i] = base - colk[r] * rowk[cidx];
+  // pivot k = 16 kb + kr; kb is a compile-time index into the register block
+#pragma unroll
+  for (int kb = 0; kb < RA; ++kb) {
+#pragma unroll 1
+    for (int kr = 0; kr < 16; ++kr) {
+      const int k = 16 * kb + kr;
+      const int buf = k & 1;
+      // owners publish row k and column k of the current matrix
+      if (tr == kr) {
+#pragma unroll
+        for (int y = 0; y < RA; ++y) rowk[buf][tc + 16 * y] = a[kb][y];
+      }
+      if (tc == kr) {
+#pragma unroll
+        for (int x = 0; x < RA; ++x) colk[buf][tr + 16 * x] = a[x][kb];
+      }
+      __syncthreads();
+      const float rp = 1.f / rowk[buf][k];
+      float rjs[RA];
+#pragma unroll
+      for (int y = 0; y < RA; ++y) {
+        const int j = tc + 16 * y;
+        rjs[y] = (j == k) ? rp : rowk[buf][j] * rp;
+      }
+#pragma unroll
+      for (int x = 0; x < RA; ++x) {
+        const int i = tr + 16 * x;
+        if (i == k) {
+#pragma unroll
+          for (int y = 0; y < RA; ++y) a[x][y] = rjs[y];
+        } else {
+          const float ci = colk[buf][i];
+#pragma unroll
+          for (int y = 0; y < RA; ++y) {
+            const int j = tc + 16 * y;
+            a[x][y] = fmaf(-ci, rjs[y], (j == k) ? 0.f : a[x][y]);
+          }
+        }
       }
     }
   }
-  __syncthreads();
-  for (int i = tid; i < D * D; i += NT) g[i] = a[i];
+#pragma unroll
+  for (int x = 0; x < RA; ++x)
+#pragma unroll
+    for (int y = 0; y < RA; ++y) g[(tr + 16 * x) * D + tc + 16 * y] = a[x][y];
 }
 
 // Row-split scan. grid (D/16, 2, B*H); 16 rows of S per CTA.
@@ -234,7 +270,7 @@ __global__ void zero_unused_chunks(Layout l, float* __restrict__ states) {
 }
 
 template <typename T, int D>
-cudaError_t launch_states_t(const Layout& l, const void* k, const void* v, const void* kt,
+cudaError_t launch_states_t(const Layout& l, int dtype, const void* k, const void* v, const void* kt,
                             const void* vt, const float* beta, const float* beta_t, float* am,
                             float* bw, float* states, cudaStream_t st) {
   int fwd_max, rev_min;
@@ -248,14 +284,17 @@ cudaError_t launch_states_t(const Layout& l, const void* k, const void* v, const
   const int nslots = map.has_text + fwd_max + (nrev > 0 ? nrev : 0);
   if (nslots > 0) {
     dim3 grid(nslots, l.H, l.B);
-    gram_kernel<T, D><<<grid, NT, 0, st>>>(l, map, (const T*)k, (const T*)v, (const T*)kt,
-                                           (const T*)vt, beta, beta_t, am, bw);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e;
+    if (gram_tc_supported(l, dtype)) {
+      e = launch_gram_tc(l, map.has_text, map.fwd_max, map.rev_lo, nslots, k, v, kt, vt, beta,
+                         beta_t, am, bw, st);
+    } else {
+      gram_kernel<T, D><<<grid, NT, 0, st>>>(l, map, (const T*)k, (const T*)v, (const T*)kt,
+                                             (const T*)vt, beta, beta_t, am, bw);
+      e = cudaGetLastError();
+    }
     if (e != cudaSuccess) return e;
-    const int smem = (D * D + 2 * D) * (int)sizeof(float);
-    e = cudaFuncSetAttribute(inverse_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    inverse_kernel<D><<<grid, NT, smem, st>>>(l, map, am);
+    inverse_kernel<D><<<grid, NT, 0, st>>>(l, map, am);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -277,15 +316,15 @@ cudaError_t launch_vda_states(const Layout& l, int dtype, const void* k, const v
                               cudaStream_t st) {
   if (dtype == VDN_F32) {
     switch (l.d) {
-      case 16: return launch_states_t<float, 16>(l, k, v, kt, vt, beta, beta_text, am, bw, states, st);
-      case 32: return launch_states_t<float, 32>(l, k, v, kt, vt, beta, beta_text, am, bw, states, st);
-      case 64: return launch_states_t<float, 64>(l, k, v, kt, vt, beta, beta_text, am, bw, states, st);
-      case 128: return launch_states_t<float, 128>(l, k, v, kt, vt, beta, beta_text, am, bw, states, st);
+      case 16: return launch_states_t<float, 16>(l, dtype, k, v, kt, vt, beta, beta_text, am, bw, states, st);
+      case 32: return launch_states_t<float, 32>(l, dtype, k, v, kt, vt, beta, beta_text, am, bw, states, st);
+      case 64: return launch_states_t<float, 64>(l, dtype, k, v, kt, vt, beta, beta_text, am, bw, states, st);
+      case 128: return launch_states_t<float, 128>(l, dtype, k, v, kt, vt, beta, beta_text, am, bw, states, st);
     }
   } else {
     switch (l.d) {
-      case 64: return launch_states_t<__nv_bfloat16, 64>(l, k, v, kt, vt, beta, beta_text, am, bw, states, st);
-      case 128: return launch_states_t<__nv_bfloat16, 128>(l, k, v, kt, vt, beta, beta_text, am, bw, states, st);
+      case 64: return launch_states_t<__nv_bfloat16, 64>(l, dtype, k, v, kt, vt, beta, beta_text, am, bw, states, st);
+      case 128: return launch_states_t<__nv_bfloat16, 128>(l, dtype, k, v, kt, vt, beta, beta_text, am, bw, states, st);
     }
   }
   return cudaErrorInvalidValue;

@@ -165,9 +165,10 @@ int vdn_hybrid_attn_fwd(const vdn_layout_t* layout, int dtype, const void* q, co
 
 int vdn_device_status(void) {
   if (cudaDeviceSynchronize() != cudaSuccess) return VDN_ERR_CUDA;
-  int s = 0;
+  int s = 0, s2 = 0;
   if (vdn::read_and_clear_tc_status(&s) != cudaSuccess) return VDN_ERR_CUDA;
-  return s;
+  if (vdn::read_and_clear_gram_status(&s2) != cudaSuccess) return VDN_ERR_CUDA;
+  return s != 0 ? s : s2;
 }
 
 const char* vdn_status_string(int status) {

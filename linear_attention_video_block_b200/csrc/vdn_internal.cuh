@@ -153,6 +153,14 @@ cudaError_t launch_hybrid_tc(const Layout& l, const void* q, const void* k, cons
 // unit (bounded waits record VDN_ERR_TIMEOUT there).
 cudaError_t read_and_clear_tc_status(int* status);
 
+// tcgen05 frame Gram (bf16, d in {64, 128}) into the (am, bw) slots.
+bool gram_tc_supported(const Layout& l, int dtype);
+cudaError_t launch_gram_tc(const Layout& l, int has_text, int fwd_max, int rev_lo, int nslots,
+                           const void* k, const void* v, const void* kt, const void* vt,
+                           const float* beta, const float* beta_t, float* am, float* bw,
+                           cudaStream_t st);
+cudaError_t read_and_clear_gram_status(int* status);
+
 // VDA: Gram into (am, bw) slots [B, H, F, d, d] (slot 0 = text), inverse in place
 // of am, scans into states [B, H, 2, J, d, d].
 cudaError_t launch_vda_states(const Layout& l, int dtype, const void* k, const void* v,
