@@ -6,12 +6,16 @@
 // CTA = one (b, h, slot); 192 threads:
 //   warp 0     TMA producer: 64-token K and V tiles into a ring of stages
 //   warp 1     MMA issuer (one lane) and TMEM owner
-//   warps 2-5  scalers: write Kw = beta (.) K (bf16) next to K, one token row per
-//              thread (beta = 0 past the frame, which also masks the ragged
-//              last tile); then the epilogue reads A and B out of TMEM.
+//   warps 2-5  scalers: write Kw = beta (.) K next to K as two bf16 parts,
+//              Kw_hi = bf16(beta k) and Kw_lo = bf16(beta k - Kw_hi), so that the
+//              products keep ~16 significant bits of beta k (a single bf16 copy
+//              put the chunk states 1e-2 off); one token row per thread, beta = 0
+//              past the frame (which also masks the ragged last tile); then the
+//              epilogue reads A and B out of TMEM.
 // Both MMA operands are MN-major (token = K dimension, contiguous along d):
 //   d = 128: D_A[i][j] += sum_u K[u][i] Kw[u][j] (TMEM columns 0..127) and
-//            D_B[i][j] += sum_u V[u][i] Kw[u][j] (columns 128..255);
+//            D_B[i][j] += sum_u V[u][i] Kw[u][j] (columns 128..255), each as the
+//            two MMAs with Kw_hi and Kw_lo;
 //   d = 64:  one M = 128 MMA with [K^T; V^T] stacked along M (the V tile sits
 //            one leading-byte-offset after the K tile): lanes 0-63 = A, 64-127 = B.
 // The work is HBM-bound: each token's k and v are read once.
@@ -38,8 +42,8 @@ template <int D>
 struct GCfg {
   static constexpr int kHalves = D / 64;
   static constexpr int kTileBytes = kTok * D * 2;
-  static constexpr int kStageBytes = 3 * kTileBytes;          // K, V, Kw
-  static constexpr int kStages = (D == 128) ? 4 : 8;
+  static constexpr int kStageBytes = 4 * kTileBytes;          // K, V, Kw_hi, Kw_lo
+  static constexpr int kStages = (D == 128) ? 3 : 6;
   static constexpr int kTmemCols = (D == 128) ? 256 : 64;
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 256;
 };
@@ -162,18 +166,21 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         }
         tc_fence_after();
         const uint32_t st = smem_u32(smem + s * C::kStageBytes);
-        const uint32_t k_addr = st, v_addr = st + C::kTileBytes, w_addr = st + 2 * C::kTileBytes;
+        const uint32_t k_addr = st, v_addr = st + C::kTileBytes;
 #pragma unroll
         for (int ks = 0; ks < kTok / 16; ++ks) {
-          const uint32_t acc = (t > 0 || ks > 0) ? 1u : 0u;
           const uint32_t koff = ks * 16 * 128;
-          const uint64_t bdesc = desc_mn_sw128(w_addr + koff, kHalfBytes);
-          if (D == 128) {
-            mma_ss(tmem, desc_mn_sw128(k_addr + koff, kHalfBytes), bdesc, idesc, acc);
-            mma_ss(tmem + 128, desc_mn_sw128(v_addr + koff, kHalfBytes), bdesc, idesc, acc);
-          } else {
-            // [K^T; V^T]: the two 64-wide M blocks are the K and V tiles
-            mma_ss(tmem, desc_mn_sw128(k_addr + koff, C::kTileBytes), bdesc, idesc, acc);
+#pragma unroll
+          for (int part = 0; part < 2; ++part) {
+            const uint32_t acc = (t > 0 || ks > 0 || part > 0) ? 1u : 0u;
+            const uint64_t bdesc = desc_mn_sw128(st + (2 + part) * C::kTileBytes + koff, kHalfBytes);
+            if (D == 128) {
+              mma_ss(tmem, desc_mn_sw128(k_addr + koff, kHalfBytes), bdesc, idesc, acc);
+              mma_ss(tmem + 128, desc_mn_sw128(v_addr + koff, kHalfBytes), bdesc, idesc, acc);
+            } else {
+              // [K^T; V^T]: the two 64-wide M blocks are the K and V tiles
+              mma_ss(tmem, desc_mn_sw128(k_addr + koff, C::kTileBytes), bdesc, idesc, acc);
+            }
           }
         }
         tc_commit(&bars->empty[s]);
@@ -201,18 +208,24 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
           bu = text ? beta_t[((long long)b * l.T + tok) * l.H + h]
                     : beta[((long long)b * l.L() + row0 + tok) * l.H + h];
         const uint4* src = reinterpret_cast<const uint4*>(st + hf * kHalfBytes + r * 128);
-        uint4* dst = reinterpret_cast<uint4*>(st + 2 * C::kTileBytes + hf * kHalfBytes + r * 128);
+        uint4* dhi = reinterpret_cast<uint4*>(st + 2 * C::kTileBytes + hf * kHalfBytes + r * 128);
+        uint4* dlo = reinterpret_cast<uint4*>(st + 3 * C::kTileBytes + hf * kHalfBytes + r * 128);
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           uint4 x = src[c];
           uint32_t w[4] = {x.x, x.y, x.z, x.w};
+          uint32_t hi4[4], lo4[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float lo = __uint_as_float(w[e] << 16) * bu;
-            const float hi = __uint_as_float(w[e] & 0xFFFF0000u) * bu;
-            w[e] = pack_bf16(lo, hi);
+            const float p0 = __uint_as_float(w[e] << 16) * bu;       // even element
+            const float p1 = __uint_as_float(w[e] & 0xFFFF0000u) * bu;  // odd element
+            const float h0 = __bfloat162float(__float2bfloat16_rn(p0));
+            const float h1 = __bfloat162float(__float2bfloat16_rn(p1));
+            hi4[e] = pack_bf16(h0, h1);
+            lo4[e] = pack_bf16(p0 - h0, p1 - h1);
           }
-          dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+          dhi[c] = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
+          dlo[c] = make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
         }
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
