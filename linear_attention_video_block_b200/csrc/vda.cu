@@ -11,7 +11,8 @@
 //   scan     S <- (S + B_f) M_f, forward over 1..fwd_max and reverse over
 //            F-2..rev_min, from S0 = 1/2 B_T M_T. Rows of S evolve independently
 //            (the update multiplies on the right), so each CTA owns 16 rows of
-//            one (b, h, direction) state and the chain needs no cross-CTA sync.
+//            one (b, h, direction) state and the chain needs no cross-CTA sync;
+//            M_f and B_f stream into shared memory two steps ahead.
 //            States read by each chunk are stored into [B, H, 2, J, d, d].
 #include "vdn_internal.cuh"
 
@@ -184,17 +185,33 @@ inverse_kernel(Layout l, SlotMap sm_map, float* __restrict__ am) {
     for (int y = 0; y < RA; ++y) g[(tr + 16 * x) * D + tc + 16 * y] = a[x][y];
 }
 
-// Row-split scan. grid (D/16, 2, B*H); 16 rows of S per CTA.
+// Row-split scan. grid (D/16, 2, B*H); 16 rows of S per CTA, 2*D threads, each
+// owning a 2 x 4 block of those rows. One thread bulk-copies M_f (D x D) and
+// the CTA's 16 rows of B_f into double-buffered shared memory two steps ahead
+// (cp.async.bulk completing on an mbarrier); the first step is the text slot
+// (S0 = 1/2 B_T M_T) when there is text.
 template <int D>
-__global__ void __launch_bounds__(NT)
+struct ScanSmem {
+  float m[2][D * D];
+  float bw[2][16 * D];
+  float x[16 * D];
+  unsigned long long full[2];
+};
+
+__device__ __forceinline__ uint32_t scan_smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+template <int D>
+__global__ void __launch_bounds__(2 * D)
 scan_kernel(Layout l, int fwd_max, int rev_min, int has_text, const float* __restrict__ am,
             const float* __restrict__ bw, float* __restrict__ states) {
   constexpr int R = 16;
-  constexpr int RG = NT / D;       // row groups
-  constexpr int RR = R / RG;       // rows per thread
-  __shared__ float x[R][D];
+  constexpr int CG = D / 4;             // column groups of 4
+  extern __shared__ __align__(128) unsigned char scan_raw[];
+  ScanSmem<D>& sm = *reinterpret_cast<ScanSmem<D>*>(scan_raw);
   const int tid = threadIdx.x;
-  const int col = tid % D, rg = tid / D;
+  const int cg = tid % CG, rg = tid / CG;   // rows 2rg, 2rg+1; cols 4cg..4cg+3
   const int row0 = blockIdx.x * R;
   const int dir = blockIdx.y;
   const int bh = blockIdx.z;
@@ -202,53 +219,114 @@ scan_kernel(Layout l, int fwd_max, int rev_min, int has_text, const float* __res
   const float* am_bh = am + (long long)bh * l.F * D * D;
   const float* bw_bh = bw + (long long)bh * l.F * D * D;
   float* st_bh = states + (long long)bh * 2 * J * D * D + (long long)dir * J * D * D;
-
-  float s[RR];
-  // S0 = 1/2 B_T M_T (slot 0), or 0 without text.
-  if (has_text) {
-    for (int i = tid; i < R * D; i += NT) x[i / D][i % D] = 0.5f * bw_bh[(row0 + i / D) * D + i % D];
-    __syncthreads();
-#pragma unroll
-    for (int r = 0; r < RR; ++r) s[r] = 0.f;
-    for (int i = 0; i < D; ++i) {
-      const float m = am_bh[i * D + col];
-#pragma unroll
-      for (int r = 0; r < RR; ++r) s[r] = fmaf(x[rg * RR + r][i], m, s[r]);
-    }
-  } else {
-#pragma unroll
-    for (int r = 0; r < RR; ++r) s[r] = 0.f;
+  const int nframes = dir == 0 ? fwd_max : (l.F - 1 - rev_min);
+  const int nsteps = has_text + nframes;
+  auto frame_of = [&](int t) { return (has_text && t == 0) ? 0 : (dir == 0 ? 1 + (t - has_text) : l.F - 2 - (t - has_text)); };
+  constexpr uint32_t kBytes = (D * D + R * D) * 4;
+  auto issue = [&](int t) {
+    const int f = frame_of(t);
+    const int buf = t & 1;
+    const uint32_t bar = scan_smem_u32(&sm.full[buf]);
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(kBytes) : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(scan_smem_u32(sm.m[buf])), "l"(am_bh + (long long)f * D * D), "r"(D * D * 4), "r"(bar)
+                 : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(scan_smem_u32(sm.bw[buf])), "l"(bw_bh + (long long)f * D * D + (long long)row0 * D),
+                   "r"(R * D * 4), "r"(bar)
+                 : "memory");
+  };
+  if (tid == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(scan_smem_u32(&sm.full[0])) : "memory");
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(scan_smem_u32(&sm.full[1])) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  __syncthreads();
+  if (tid == 0) {
+    if (nsteps > 0) issue(0);
+    if (nsteps > 1) issue(1);
+  }
+  float s[2][4];
+#pragma unroll
+  for (int r = 0; r < 2; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) s[r][c] = 0.f;
   auto store_for = [&](int idx) {
     for (int j = 0; j < J; ++j) {
       Group G = make_group(l, 2 + j);
       if (G.nq == 0) continue;
-      int want = dir == 0 ? G.fwd_idx : G.rev_idx;
+      const int want = dir == 0 ? G.fwd_idx : G.rev_idx;
       if (want != idx) continue;
       float* dst = st_bh + (long long)j * D * D;
 #pragma unroll
-      for (int r = 0; r < RR; ++r) dst[(row0 + rg * RR + r) * D + col] = s[r];
+      for (int r = 0; r < 2; ++r)
+        *reinterpret_cast<float4*>(dst + (row0 + 2 * rg + r) * D + 4 * cg) =
+            make_float4(s[r][0], s[r][1], s[r][2], s[r][3]);
     }
   };
-  store_for(dir == 0 ? 0 : l.F - 1);
-  const int nsteps = dir == 0 ? fwd_max : (l.F - 1 - rev_min);
+  if (!has_text) store_for(dir == 0 ? 0 : l.F - 1);
   for (int t = 0; t < nsteps; ++t) {
-    const int f = dir == 0 ? 1 + t : l.F - 2 - t;
-    const float* mf = am_bh + (long long)f * D * D;
-    const float* bf = bw_bh + (long long)f * D * D;
-    __syncthreads();
-#pragma unroll
-    for (int r = 0; r < RR; ++r) x[rg * RR + r][col] = s[r] + bf[(row0 + rg * RR + r) * D + col];
-    __syncthreads();
-#pragma unroll
-    for (int r = 0; r < RR; ++r) s[r] = 0.f;
-#pragma unroll 8
-    for (int i = 0; i < D; ++i) {
-      const float m = mf[i * D + col];
-#pragma unroll
-      for (int r = 0; r < RR; ++r) s[r] = fmaf(x[rg * RR + r][i], m, s[r]);
+    const int buf = t & 1;
+    const bool text = has_text && t == 0;
+    // the copy lands within microseconds; the spin is bounded anyway
+    {
+      const uint32_t bar = scan_smem_u32(&sm.full[buf]);
+      const uint32_t parity = (t >> 1) & 1;
+      uint32_t ok = 0;
+      for (uint32_t it = 0; it < (1u << 26) && !ok; ++it) {
+        asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                     "selp.u32 %0, 1, 0, p;\n\t}\n"
+                     : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+      }
+      // (not reached in practice; if it were, the CTA carries on with stale
+      // shared memory rather than leave the others waiting at the barrier)
     }
-    store_for(f);
+    // X = S + B_f rows (text step: X = 1/2 B_T rows)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const float4 bv = *reinterpret_cast<const float4*>(&sm.bw[buf][(2 * rg + r) * D + 4 * cg]);
+      float4 xv;
+      if (text) {
+        xv = make_float4(0.5f * bv.x, 0.5f * bv.y, 0.5f * bv.z, 0.5f * bv.w);
+      } else {
+        xv = make_float4(s[r][0] + bv.x, s[r][1] + bv.y, s[r][2] + bv.z, s[r][3] + bv.w);
+      }
+      *reinterpret_cast<float4*>(&sm.x[(2 * rg + r) * D + 4 * cg]) = xv;
+    }
+    __syncthreads();
+    float acc[2][4];
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
+    const float* mb = sm.m[buf];
+#pragma unroll 4
+    for (int i = 0; i < D; i += 4) {
+      const float4 x0 = *reinterpret_cast<const float4*>(&sm.x[(2 * rg) * D + i]);
+      const float4 x1 = *reinterpret_cast<const float4*>(&sm.x[(2 * rg + 1) * D + i]);
+      const float xa[4] = {x0.x, x0.y, x0.z, x0.w};
+      const float xb[4] = {x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+      for (int ii = 0; ii < 4; ++ii) {
+        const float4 m = *reinterpret_cast<const float4*>(&mb[(i + ii) * D + 4 * cg]);
+        acc[0][0] = fmaf(xa[ii], m.x, acc[0][0]);
+        acc[0][1] = fmaf(xa[ii], m.y, acc[0][1]);
+        acc[0][2] = fmaf(xa[ii], m.z, acc[0][2]);
+        acc[0][3] = fmaf(xa[ii], m.w, acc[0][3]);
+        acc[1][0] = fmaf(xb[ii], m.x, acc[1][0]);
+        acc[1][1] = fmaf(xb[ii], m.y, acc[1][1]);
+        acc[1][2] = fmaf(xb[ii], m.z, acc[1][2]);
+        acc[1][3] = fmaf(xb[ii], m.w, acc[1][3]);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) s[r][c] = acc[r][c];
+    __syncthreads();  // everyone is done with buffer `buf` and with x
+    if (tid == 0 && t + 2 < nsteps) issue(t + 2);
+    if (text) store_for(dir == 0 ? 0 : l.F - 1);
+    else store_for(frame_of(t));
   }
 }
 
@@ -300,8 +378,11 @@ cudaError_t launch_states_t(const Layout& l, int dtype, const void* k, const voi
   }
   {
     dim3 grid(D / 16, 2, l.B * l.H);
-    scan_kernel<D><<<grid, NT, 0, st>>>(l, fwd_max, rev_min, map.has_text, am, bw, states);
-    cudaError_t e = cudaGetLastError();
+    const int smem = (int)sizeof(ScanSmem<D>);
+    cudaError_t e = cudaFuncSetAttribute(scan_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    scan_kernel<D><<<grid, 2 * D, smem, st>>>(l, fwd_max, rev_min, map.has_text, am, bw, states);
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     zero_unused_chunks<<<dim3(32, l.B * l.H), 256, 0, st>>>(l, states);
   }
