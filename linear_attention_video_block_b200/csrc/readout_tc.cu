@@ -1,0 +1,267 @@
+// Linear-branch readout o_lin = (S_fwd + S_rev) q on the 5th-generation tensor
+// cores, for the standalone linear-branch entry point with bf16 tensors
+// (project page "Local Softmax and Long-Range Linear Memory": both states are
+// read and their outputs added; boundary frames read nothing).
+//
+// CTA = up to 8 consecutive 128-row query tiles of one query group of one
+// (b, h); 192 threads:
+//   warp 0     TMA producer: Q tiles into two shared-memory stages
+//   warp 1     MMA issuer and TMEM owner: O = Q S_hi^T + Q S_lo^T into one of two
+//              TMEM accumulators
+//   warps 2-5  stage S_sum = S_fwd + S_rev once as two bf16 K-major operands
+//              (S_hi = bf16(S_sum), S_lo = bf16(S_sum - S_hi)), then drain each
+//              accumulator to global memory as bf16 (one row per thread)
+// Boundary-frame groups write zeros. HBM-bound: q is read once, o_lin written once.
+#include "tc_common.cuh"
+
+namespace vdn {
+
+__device__ int g_readout_status = 0;
+
+cudaError_t read_and_clear_readout_status(int* status) {
+  cudaError_t e = cudaMemcpyFromSymbol(status, g_readout_status, sizeof(int));
+  if (e != cudaSuccess) return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_readout_status, &zero, sizeof(int));
+}
+
+namespace {
+
+constexpr int kRows = 128;
+constexpr int kTilesPerCta = 8;
+constexpr int kThreads = 192;
+
+template <int D>
+struct RCfg {
+  static constexpr int kHalves = D / 64;
+  static constexpr int kHalfBytes = kRows * 128;
+  static constexpr int kTileBytes = kRows * D * 2;
+  static constexpr int kTmemCols = 2 * D;
+  static constexpr int kSmemBytes = 1024 + 4 * kTileBytes + 256;  // S_hi, S_lo, 2 Q stages
+};
+
+struct RBars {
+  unsigned long long q_full[2];
+  unsigned long long q_empty[2];
+  unsigned long long d_full[2];
+  unsigned long long d_empty[2];
+  unsigned long long ssum_ready;
+  unsigned long long done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ bool rwait(unsigned long long* bar, uint32_t parity, volatile int* abort,
+                                      bool watch_abort = true) {
+  if (mbar_try_wait(smem_u32(bar), parity)) return true;
+  return mbar_wait_impl(bar, parity, abort, &g_readout_status, watch_abort);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Layout l,
+                  const float* __restrict__ states, __nv_bfloat16* __restrict__ o_lin) {
+  using C = RCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sHi = smem;
+  uint8_t* sLo = smem + C::kTileBytes;
+  uint8_t* sQ = smem + 2 * C::kTileBytes;
+  RBars* bars = reinterpret_cast<RBars*>(smem + 4 * C::kTileBytes);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int h = blockIdx.y, b = blockIdx.z;
+  int g, r0;
+  tile_to_group(l, kRows * kTilesPerCta, blockIdx.x, g, r0);
+  if (g < 0) return;  // grid is sized by the same enumeration; uniform per CTA
+  const Group G = make_group(l, g);
+  const int rows = min(kRows * kTilesPerCta, G.q0 + G.nq - r0);
+  const long long HD = (long long)l.H * D;
+
+  if (G.chunk < 0) {
+    // boundary frame: no linear readout
+    for (int i = threadIdx.x; i < rows * (D / 8); i += kThreads) {
+      const int r = i / (D / 8), c = i % (D / 8);
+      reinterpret_cast<uint4*>(o_lin + ((long long)b * l.L() + r0 + r) * HD + (long long)h * D)[c] =
+          make_uint4(0u, 0u, 0u, 0u);
+    }
+    return;
+  }
+  const int n_tiles = (rows + kRows - 1) / kRows;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->q_full[i], 1);
+      mbar_init(&bars->q_empty[i], 1);
+      mbar_init(&bars->d_full[i], 1);
+      mbar_init(&bars->d_empty[i], 128);
+    }
+    mbar_init(&bars->ssum_ready, 128);
+    mbar_init(&bars->done, 1);
+    bars->abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(smem_u32(&bars->tmem_base)), "r"(C::kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  volatile int* abort = &bars->abort;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      bool ok = true;
+      for (int t = 0; t < n_tiles; ++t) {
+        const int s = t & 1, use = t >> 1;
+        if (use > 0 && !rwait(&bars->q_empty[s], (use - 1) & 1, abort)) {
+          ok = false;
+          break;
+        }
+        mbar_expect_tx(&bars->q_full[s], C::kTileBytes);
+        for (int hf = 0; hf < C::kHalves; ++hf)
+          tma_load_4d(sQ + s * C::kTileBytes + hf * C::kHalfBytes, &tm_q, &bars->q_full[s], hf * 64, h,
+                      r0 + t * kRows, b);
+        ++issued;
+      }
+      if (!ok) {
+        for (int s = 0; s < 2 && s < issued; ++s) {
+          const int last = issued - 1 - ((issued - 1 - s) % 2);
+          rwait(&bars->q_full[s], (last >> 1) & 1, abort, false);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = make_idesc(D, false);
+      bool ok = rwait(&bars->ssum_ready, 0, abort);
+      const uint32_t hi_addr = smem_u32(sHi), lo_addr = smem_u32(sLo), q_addr = smem_u32(sQ);
+      for (int t = 0; t < n_tiles && ok; ++t) {
+        const int s = t & 1, use = t >> 1;
+        if (!rwait(&bars->q_full[s], use & 1, abort)) { ok = false; break; }
+        if (use > 0 && !rwait(&bars->d_empty[s], (use - 1) & 1, abort)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + s * D;
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t off = (uint32_t)((ks / 4) * C::kHalfBytes + (ks % 4) * 32);
+            mma_ss(d_tmem, desc_k_sw128(q_addr + s * C::kTileBytes + off),
+                   desc_k_sw128((part ? lo_addr : hi_addr) + off), idesc, (part > 0 || ks > 0) ? 1u : 0u);
+          }
+        }
+        tc_commit(&bars->q_empty[s]);
+        tc_commit(&bars->d_full[s]);
+      }
+      if (!ok) {
+        // every MMA issued must finish before TMEM is freed
+        tc_commit(&bars->done);
+        rwait(&bars->done, 0, abort, false);
+      }
+    }
+  } else {
+    const int t128 = threadIdx.x - 64;
+    // stage S_sum (hi, lo) once
+    {
+      const int J = l.J();
+      const float* sf = states + ((((long long)b * l.H + h) * 2 + 0) * J + G.chunk) * D * D;
+      const float* sr = states + ((((long long)b * l.H + h) * 2 + 1) * J + G.chunk) * D * D;
+      constexpr int kChunks = D / 8;
+      for (int ch = t128; ch < kRows * kChunks; ch += 128) {
+        const int n = ch / kChunks, kc = ch % kChunks;
+        if (n >= D) continue;  // rows beyond d (d = 64) stay unused: the MMA reads N = d rows
+        const float4 a0 = *reinterpret_cast<const float4*>(sf + n * D + kc * 8);
+        const float4 a1 = *reinterpret_cast<const float4*>(sf + n * D + kc * 8 + 4);
+        const float4 b0 = *reinterpret_cast<const float4*>(sr + n * D + kc * 8);
+        const float4 b1 = *reinterpret_cast<const float4*>(sr + n * D + kc * 8 + 4);
+        const float x[8] = {a0.x + b0.x, a0.y + b0.y, a0.z + b0.z, a0.w + b0.w,
+                            a1.x + b1.x, a1.y + b1.y, a1.z + b1.z, a1.w + b1.w};
+        float hi[8], lo[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          hi[e] = __bfloat162float(__float2bfloat16_rn(x[e]));
+          lo[e] = x[e] - hi[e];
+        }
+        const int half = kc / 8, c16 = kc % 8;
+        const int off = half * C::kHalfBytes + n * 128 + ((c16 ^ (n & 7)) * 16);
+        *reinterpret_cast<uint4*>(sHi + off) = make_uint4(pack_bf16(hi[0], hi[1]), pack_bf16(hi[2], hi[3]),
+                                                          pack_bf16(hi[4], hi[5]), pack_bf16(hi[6], hi[7]));
+        *reinterpret_cast<uint4*>(sLo + off) = make_uint4(pack_bf16(lo[0], lo[1]), pack_bf16(lo[2], lo[3]),
+                                                          pack_bf16(lo[4], lo[5]), pack_bf16(lo[6], lo[7]));
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(&bars->ssum_ready);
+    }
+    // drain accumulators
+    const int m = 32 * (warp & 3) + lane;
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    for (int t = 0; t < n_tiles; ++t) {
+      const int s = t & 1, use = t >> 1;
+      if (!__all_sync(0xffffffffu, rwait(&bars->d_full[s], use & 1, abort))) break;
+      tc_fence_after();
+      const int grow = r0 + t * kRows + m;
+      const bool store = grow < G.q0 + G.nq;
+      __nv_bfloat16* dst = o_lin + ((long long)b * l.L() + grow) * HD + (long long)h * D;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld_x32(tmem + lane_base + s * D + c0, r);
+        if (store) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            d4[i] = make_uint4(pack_bf16(__uint_as_float(r[8 * i]), __uint_as_float(r[8 * i + 1])),
+                               pack_bf16(__uint_as_float(r[8 * i + 2]), __uint_as_float(r[8 * i + 3])),
+                               pack_bf16(__uint_as_float(r[8 * i + 4]), __uint_as_float(r[8 * i + 5])),
+                               pack_bf16(__uint_as_float(r[8 * i + 6]), __uint_as_float(r[8 * i + 7])));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars->d_empty[s]);
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::kTmemCols)
+                 : "memory");
+  }
+}
+
+template <int D>
+cudaError_t launch_readout_t(const Layout& l, const void* q, const float* states, void* o_lin,
+                             cudaStream_t st) {
+  CUtensorMap mq;
+  if (!make_map(&mq, q, D, l.H, l.L(), l.B)) return cudaErrorInvalidValue;
+  auto kern = readout_tc_kernel<D>;
+  const int smem = RCfg<D>::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(tiles_per_head(l, kRows * kTilesPerCta), l.H, l.B);
+  if (grid.x == 0) return cudaSuccess;
+  kern<<<grid, kThreads, smem, st>>>(mq, l, states, static_cast<__nv_bfloat16*>(o_lin));
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool readout_tc_supported(const Layout& l, int dtype) {
+  return dtype == VDN_BF16 && (l.d == 64 || l.d == 128);
+}
+
+cudaError_t launch_readout_tc(const Layout& l, const void* q, const float* states, void* o_lin,
+                              cudaStream_t st) {
+  if (l.d == 128) return launch_readout_t<128>(l, q, states, o_lin, st);
+  if (l.d == 64) return launch_readout_t<64>(l, q, states, o_lin, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace vdn

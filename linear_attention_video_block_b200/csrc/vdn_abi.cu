@@ -123,6 +123,8 @@ int vdn_vda_scan_fwd(const vdn_layout_t* layout, int dtype, const void* q, const
   const float* bt = layout->T ? beta_text : nullptr;
   int s = cuda_status(vdn::launch_vda_states(l, dtype, k, v, kt, vt, beta, bt, w.am, w.bw, states, stream));
   if (s != VDN_OK) return s;
+  if (vdn::readout_tc_supported(l, dtype))
+    return cuda_status(vdn::launch_readout_tc(l, q, states, o_lin, stream));
   return cuda_status(vdn::launch_readout(l, dtype, 0, q, states, nullptr, nullptr, nullptr, nullptr,
                                          0.f, o_lin, nullptr, nullptr, stream));
 }
@@ -165,10 +167,13 @@ int vdn_hybrid_attn_fwd(const vdn_layout_t* layout, int dtype, const void* q, co
 
 int vdn_device_status(void) {
   if (cudaDeviceSynchronize() != cudaSuccess) return VDN_ERR_CUDA;
-  int s = 0, s2 = 0;
-  if (vdn::read_and_clear_tc_status(&s) != cudaSuccess) return VDN_ERR_CUDA;
-  if (vdn::read_and_clear_gram_status(&s2) != cudaSuccess) return VDN_ERR_CUDA;
-  return s != 0 ? s : s2;
+  int s[3] = {0, 0, 0};
+  if (vdn::read_and_clear_tc_status(&s[0]) != cudaSuccess) return VDN_ERR_CUDA;
+  if (vdn::read_and_clear_gram_status(&s[1]) != cudaSuccess) return VDN_ERR_CUDA;
+  if (vdn::read_and_clear_readout_status(&s[2]) != cudaSuccess) return VDN_ERR_CUDA;
+  for (int i = 0; i < 3; ++i)
+    if (s[i] != 0) return s[i];
+  return VDN_OK;
 }
 
 const char* vdn_status_string(int status) {

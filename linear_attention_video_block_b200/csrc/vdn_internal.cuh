@@ -161,6 +161,12 @@ cudaError_t launch_gram_tc(const Layout& l, int has_text, int fwd_max, int rev_l
                            cudaStream_t st);
 cudaError_t read_and_clear_gram_status(int* status);
 
+// tcgen05 linear readout o_lin = S_sum q (bf16, d in {64, 128}).
+bool readout_tc_supported(const Layout& l, int dtype);
+cudaError_t launch_readout_tc(const Layout& l, const void* q, const float* states, void* o_lin,
+                              cudaStream_t st);
+cudaError_t read_and_clear_readout_status(int* status);
+
 // VDA: Gram into (am, bw) slots [B, H, F, d, d] (slot 0 = text), inverse in place
 // of am, scans into states [B, H, 2, J, d, d].
 cudaError_t launch_vda_states(const Layout& l, int dtype, const void* k, const void* v,
