@@ -4,7 +4,7 @@
 // over the U tokens of one frame (or of the text, slot 0), fp32 results.
 //
 // CTA = one (b, h, slot); 192 threads:
-//   warp 0     TMA producer: 64-token K and V tiles into a ring of stages
+//   warp 0     TMA producer: 32-token K and V tiles into a ring of stages
 //   warp 1     MMA issuer (one lane) and TMEM owner
 //   warps 2-5  scalers: write Kw = beta (.) K next to K as two bf16 parts,
 //              Kw_hi = bf16(beta k) and Kw_lo = bf16(beta k - Kw_hi), so that the
@@ -34,9 +34,9 @@ cudaError_t read_and_clear_gram_status(int* status) {
 
 namespace {
 
-constexpr int kTok = 64;        // tokens per tile
+constexpr int kTok = 32;        // tokens per tile (96 KB of stages: two CTAs per SM)
 constexpr int kThreads = 192;
-constexpr int kHalfBytes = kTok * 128;  // 64 tokens x 64 bf16 (one swizzle atom column)
+constexpr int kHalfBytes = kTok * 128;  // kTok tokens x 64 bf16 (one swizzle atom column)
 
 template <int D>
 struct GCfg {
@@ -83,7 +83,7 @@ struct GramSlots {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUtensorMap tm_vt,
                const Layout l, const GramSlots slots, const float* __restrict__ beta,
@@ -190,7 +190,7 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     }
   } else {
     // ---------------------------------------------------- scalers / epilogue
-    const int u = threadIdx.x - 64;  // token row within a tile, 0..127? only 0..63 used
+    const int u = threadIdx.x - 64;  // 0..127: (token row, d half) items below
     bool ok = true;
     for (int t = 0; t < n_tiles && ok; ++t) {
       const int s = t % C::kStages, use = t / C::kStages;

@@ -3,7 +3,7 @@
 // (project page "Local Softmax and Long-Range Linear Memory": both states are
 // read and their outputs added; boundary frames read nothing).
 //
-// CTA = up to 8 consecutive 128-row query tiles of one query group of one
+// CTA = up to 24 consecutive 128-row query tiles of one query group of one
 // (b, h); 192 threads:
 //   warp 0     TMA producer: Q tiles into two shared-memory stages
 //   warp 1     MMA issuer and TMEM owner: O = Q S_hi^T + Q S_lo^T into one of two
@@ -28,7 +28,7 @@ cudaError_t read_and_clear_readout_status(int* status) {
 namespace {
 
 constexpr int kRows = 128;
-constexpr int kTilesPerCta = 8;
+constexpr int kTilesPerCta = 24;
 constexpr int kThreads = 192;
 
 template <int D>

@@ -12,7 +12,8 @@
 //            F-2..rev_min, from S0 = 1/2 B_T M_T. Rows of S evolve independently
 //            (the update multiplies on the right), so each CTA owns 16 rows of
 //            one (b, h, direction) state and the chain needs no cross-CTA sync;
-//            M_f and B_f stream into shared memory two steps ahead.
+//            all CTAs are resident at once and M_f streams through a small
+//            cp.async ring.
 //            States read by each chunk are stored into [B, H, 2, J, d, d].
 #include "vdn_internal.cuh"
 
@@ -115,11 +116,14 @@ gram_kernel(Layout l, SlotMap sm_map, const T* __restrict__ k, const T* __restri
 
 // In-place inverse of (I + A) for one slot: Gauss-Jordan elimination without
 // pivoting (every pivot of an SPD matrix with eigenvalues >= 1 is >= 1).
-// Thread (tr, tc) of a 16 x 16 grid keeps the interleaved block of rows
-// tr + 16a and columns tc + 16c in registers; the pivot row and column of
-// each step go through double-buffered shared memory, one barrier per step.
+// Step k written as a rank-1 update: with row k and column k zeroed,
+//   a <- a - c r^T,  c = column k (c_k = -1),  r = row k / p (r_k = 1/p),
+// which yields the Gauss-Jordan result in every entry. Thread (tr, tc) of a
+// 16 x 16 grid keeps the interleaved block of rows tr + 16x and columns
+// tc + 16y in registers; the pivot row and column go through double-buffered
+// shared memory, one barrier per step.
 template <int D>
-__global__ void __launch_bounds__(NT)
+__global__ void __launch_bounds__(NT, 2)
 inverse_kernel(Layout l, SlotMap sm_map, float* __restrict__ am) {
   constexpr int RA = D / 16;
   __shared__ float rowk[2][D];
@@ -145,38 +149,35 @@ inverse_kernel(Layout l, SlotMap sm_map, float* __restrict__ am) {
     for (int kr = 0; kr < 16; ++kr) {
       const int k = 16 * kb + kr;
       const int buf = k & 1;
-      // owners publish row k and column k of the current matrix
+      // owners publish row k and column k, then zero them in their registers
       if (tr == kr) {
 #pragma unroll
-        for (int y = 0; y < RA; ++y) rowk[buf][tc + 16 * y] = a[kb][y];
+        for (int y = 0; y < RA; ++y) {
+          rowk[buf][tc + 16 * y] = a[kb][y];
+          a[kb][y] = 0.f;
+        }
       }
       if (tc == kr) {
 #pragma unroll
-        for (int x = 0; x < RA; ++x) colk[buf][tr + 16 * x] = a[x][kb];
+        for (int x = 0; x < RA; ++x) {
+          colk[buf][tr + 16 * x] = (x == kb && tr == kr) ? -1.f : a[x][kb];
+          a[x][kb] = 0.f;
+        }
       }
       __syncthreads();
       const float rp = 1.f / rowk[buf][k];
-      float rjs[RA];
+      float r[RA], c[RA];
 #pragma unroll
       for (int y = 0; y < RA; ++y) {
         const int j = tc + 16 * y;
-        rjs[y] = (j == k) ? rp : rowk[buf][j] * rp;
+        r[y] = (j == k) ? rp : rowk[buf][j] * rp;
       }
 #pragma unroll
-      for (int x = 0; x < RA; ++x) {
-        const int i = tr + 16 * x;
-        if (i == k) {
+      for (int x = 0; x < RA; ++x) c[x] = colk[buf][tr + 16 * x];
 #pragma unroll
-          for (int y = 0; y < RA; ++y) a[x][y] = rjs[y];
-        } else {
-          const float ci = colk[buf][i];
+      for (int x = 0; x < RA; ++x)
 #pragma unroll
-          for (int y = 0; y < RA; ++y) {
-            const int j = tc + 16 * y;
-            a[x][y] = fmaf(-ci, rjs[y], (j == k) ? 0.f : a[x][y]);
-          }
-        }
-      }
+        for (int y = 0; y < RA; ++y) a[x][y] = fmaf(-c[x], r[y], a[x][y]);
     }
   }
 #pragma unroll
@@ -185,33 +186,45 @@ inverse_kernel(Layout l, SlotMap sm_map, float* __restrict__ am) {
     for (int y = 0; y < RA; ++y) g[(tr + 16 * x) * D + tc + 16 * y] = a[x][y];
 }
 
-// Row-split scan. grid (D/16, 2, B*H); 16 rows of S per CTA, 2*D threads, each
-// owning a 2 x 4 block of those rows. One thread bulk-copies M_f (D x D) and
-// the CTA's 16 rows of B_f into double-buffered shared memory two steps ahead
-// (cp.async.bulk completing on an mbarrier); the first step is the text slot
-// (S0 = 1/2 B_T M_T) when there is text.
+// Row-split scan. grid (D/16, 2, B*H): 16 rows of S per CTA, so all
+// 2 (D/16) B H CTAs are resident at once (40 KB of shared memory each) and the
+// chain of dependent steps runs a single time. 128 threads (fewer for d < 32); thread (rg, cg)
+// owns rows 4rg..4rg+3 and columns 4cg..4cg+3 of the CTA's block (d = 128;
+// smaller d use fewer column groups and more rows per thread). Each step
+// S <- (S + B_f) M_f streams M_f through a 3-deep ring of 16-row chunks with
+// cp.async; the first step is the text slot (S0 = 1/2 B_T M_T) when there is text.
 template <int D>
-struct ScanSmem {
-  float m[2][D * D];
-  float bw[2][16 * D];
-  float x[16 * D];
-  unsigned long long full[2];
+struct ScanCfg {
+  static constexpr int kR = 16;                 // rows of S per CTA
+  static constexpr int kCG = D / 4;             // column groups of 4
+  static constexpr int kThreads = (kCG * 16 < 128) ? kCG * 16 : 128;
+  static constexpr int kRG = kThreads / kCG;    // row groups
+  static constexpr int kRR = kR / kRG;          // rows per thread
+  static constexpr int kChunk = 16;             // rows of M per chunk
+  static constexpr int kRing = 3;
 };
 
-__device__ __forceinline__ uint32_t scan_smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
 }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 template <int D>
-__global__ void __launch_bounds__(2 * D)
+__global__ void __launch_bounds__(128)
 scan_kernel(Layout l, int fwd_max, int rev_min, int has_text, const float* __restrict__ am,
             const float* __restrict__ bw, float* __restrict__ states) {
-  constexpr int R = 16;
-  constexpr int CG = D / 4;             // column groups of 4
-  extern __shared__ __align__(128) unsigned char scan_raw[];
-  ScanSmem<D>& sm = *reinterpret_cast<ScanSmem<D>*>(scan_raw);
+  using C = ScanCfg<D>;
+  constexpr int R = C::kR, RR = C::kRR, CH = C::kChunk, NCH = D / CH;
+  __shared__ __align__(16) float ring[C::kRing][CH * D];
+  __shared__ __align__(16) float brows[R * D];
+  __shared__ __align__(16) float x[R * D];
   const int tid = threadIdx.x;
-  const int cg = tid % CG, rg = tid / CG;   // rows 2rg, 2rg+1; cols 4cg..4cg+3
+  const int cg = tid % C::kCG, rg = tid / C::kCG;
   const int row0 = blockIdx.x * R;
   const int dir = blockIdx.y;
   const int bh = blockIdx.z;
@@ -221,34 +234,20 @@ scan_kernel(Layout l, int fwd_max, int rev_min, int has_text, const float* __res
   float* st_bh = states + (long long)bh * 2 * J * D * D + (long long)dir * J * D * D;
   const int nframes = dir == 0 ? fwd_max : (l.F - 1 - rev_min);
   const int nsteps = has_text + nframes;
-  auto frame_of = [&](int t) { return (has_text && t == 0) ? 0 : (dir == 0 ? 1 + (t - has_text) : l.F - 2 - (t - has_text)); };
-  constexpr uint32_t kBytes = (D * D + R * D) * 4;
-  auto issue = [&](int t) {
-    const int f = frame_of(t);
-    const int buf = t & 1;
-    const uint32_t bar = scan_smem_u32(&sm.full[buf]);
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(kBytes) : "memory");
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 ::"r"(scan_smem_u32(sm.m[buf])), "l"(am_bh + (long long)f * D * D), "r"(D * D * 4), "r"(bar)
-                 : "memory");
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 ::"r"(scan_smem_u32(sm.bw[buf])), "l"(bw_bh + (long long)f * D * D + (long long)row0 * D),
-                   "r"(R * D * 4), "r"(bar)
-                 : "memory");
+  auto frame_of = [&](int t) {
+    return (has_text && t == 0) ? 0 : (dir == 0 ? 1 + (t - has_text) : l.F - 2 - (t - has_text));
   };
-  if (tid == 0) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(scan_smem_u32(&sm.full[0])) : "memory");
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(scan_smem_u32(&sm.full[1])) : "memory");
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  __syncthreads();
-  if (tid == 0) {
-    if (nsteps > 0) issue(0);
-    if (nsteps > 1) issue(1);
-  }
-  float s[2][4];
+  // global chunk sequence q = t * NCH + c: rows 16c..16c+15 of M_{frame_of(t)}
+  auto load_chunk = [&](int q) {
+    const int t = q / NCH, c = q % NCH;
+    const float* src = am_bh + (long long)frame_of(t) * D * D + (long long)c * CH * D;
+    float* dst = ring[q % C::kRing];
+    for (int i = tid * 4; i < CH * D; i += C::kThreads * 4) cp_async16(dst + i, src + i);
+  };
+  const int nq = nsteps * NCH;
+  float s[RR][4];
 #pragma unroll
-  for (int r = 0; r < 2; ++r)
+  for (int r = 0; r < RR; ++r)
 #pragma unroll
     for (int c = 0; c < 4; ++c) s[r][c] = 0.f;
   auto store_for = [&](int idx) {
@@ -259,75 +258,70 @@ scan_kernel(Layout l, int fwd_max, int rev_min, int has_text, const float* __res
       if (want != idx) continue;
       float* dst = st_bh + (long long)j * D * D;
 #pragma unroll
-      for (int r = 0; r < 2; ++r)
-        *reinterpret_cast<float4*>(dst + (row0 + 2 * rg + r) * D + 4 * cg) =
+      for (int r = 0; r < RR; ++r)
+        *reinterpret_cast<float4*>(dst + (row0 + RR * rg + r) * D + 4 * cg) =
             make_float4(s[r][0], s[r][1], s[r][2], s[r][3]);
     }
   };
   if (!has_text) store_for(dir == 0 ? 0 : l.F - 1);
+  // prologue: two chunks in flight
+  for (int q = 0; q < 2; ++q) {
+    if (q < nq) load_chunk(q);
+    cp_async_commit();
+  }
   for (int t = 0; t < nsteps; ++t) {
-    const int buf = t & 1;
     const bool text = has_text && t == 0;
-    // the copy lands within microseconds; the spin is bounded anyway
-    {
-      const uint32_t bar = scan_smem_u32(&sm.full[buf]);
-      const uint32_t parity = (t >> 1) & 1;
-      uint32_t ok = 0;
-      for (uint32_t it = 0; it < (1u << 26) && !ok; ++it) {
-        asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-                     "selp.u32 %0, 1, 0, p;\n\t}\n"
-                     : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-      }
-      // (not reached in practice; if it were, the CTA carries on with stale
-      // shared memory rather than leave the others waiting at the barrier)
-    }
-    // X = S + B_f rows (text step: X = 1/2 B_T rows)
+    const int f = frame_of(t);
+    // X = S + B_f rows (text step: X = 1/2 B_T rows); B rows read straight from global
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const float4 bv = *reinterpret_cast<const float4*>(&sm.bw[buf][(2 * rg + r) * D + 4 * cg]);
-      float4 xv;
-      if (text) {
-        xv = make_float4(0.5f * bv.x, 0.5f * bv.y, 0.5f * bv.z, 0.5f * bv.w);
-      } else {
-        xv = make_float4(s[r][0] + bv.x, s[r][1] + bv.y, s[r][2] + bv.z, s[r][3] + bv.w);
-      }
-      *reinterpret_cast<float4*>(&sm.x[(2 * rg + r) * D + 4 * cg]) = xv;
+    for (int r = 0; r < RR; ++r) {
+      const float4 bv = *reinterpret_cast<const float4*>(bw_bh + (long long)f * D * D +
+                                                         (long long)(row0 + RR * rg + r) * D + 4 * cg);
+      const float4 xv = text ? make_float4(0.5f * bv.x, 0.5f * bv.y, 0.5f * bv.z, 0.5f * bv.w)
+                             : make_float4(s[r][0] + bv.x, s[r][1] + bv.y, s[r][2] + bv.z, s[r][3] + bv.w);
+      *reinterpret_cast<float4*>(&x[(RR * rg + r) * D + 4 * cg]) = xv;
     }
-    __syncthreads();
-    float acc[2][4];
+    float acc[RR][4];
 #pragma unroll
-    for (int r = 0; r < 2; ++r)
+    for (int r = 0; r < RR; ++r)
 #pragma unroll
       for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
-    const float* mb = sm.m[buf];
-#pragma unroll 4
-    for (int i = 0; i < D; i += 4) {
-      const float4 x0 = *reinterpret_cast<const float4*>(&sm.x[(2 * rg) * D + i]);
-      const float4 x1 = *reinterpret_cast<const float4*>(&sm.x[(2 * rg + 1) * D + i]);
-      const float xa[4] = {x0.x, x0.y, x0.z, x0.w};
-      const float xb[4] = {x1.x, x1.y, x1.z, x1.w};
+    for (int c = 0; c < NCH; ++c) {
+      const int q = t * NCH + c;
+      cp_async_wait<1>();   // chunk q has landed (q + 1 may still be in flight)
+      __syncthreads();      // ... for every thread; x is complete; slot (q + 2) % 3 is free
+      if (q + 2 < nq) load_chunk(q + 2);
+      cp_async_commit();
+      const float* mb = ring[q % C::kRing];
 #pragma unroll
-      for (int ii = 0; ii < 4; ++ii) {
-        const float4 m = *reinterpret_cast<const float4*>(&mb[(i + ii) * D + 4 * cg]);
-        acc[0][0] = fmaf(xa[ii], m.x, acc[0][0]);
-        acc[0][1] = fmaf(xa[ii], m.y, acc[0][1]);
-        acc[0][2] = fmaf(xa[ii], m.z, acc[0][2]);
-        acc[0][3] = fmaf(xa[ii], m.w, acc[0][3]);
-        acc[1][0] = fmaf(xb[ii], m.x, acc[1][0]);
-        acc[1][1] = fmaf(xb[ii], m.y, acc[1][1]);
-        acc[1][2] = fmaf(xb[ii], m.z, acc[1][2]);
-        acc[1][3] = fmaf(xb[ii], m.w, acc[1][3]);
+      for (int i4 = 0; i4 < CH; i4 += 4) {
+        float xr[RR][4];
+#pragma unroll
+        for (int r = 0; r < RR; ++r) {
+          const float4 v = *reinterpret_cast<const float4*>(&x[(RR * rg + r) * D + c * CH + i4]);
+          xr[r][0] = v.x; xr[r][1] = v.y; xr[r][2] = v.z; xr[r][3] = v.w;
+        }
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii) {
+          const float4 m = *reinterpret_cast<const float4*>(&mb[(i4 + ii) * D + 4 * cg]);
+#pragma unroll
+          for (int r = 0; r < RR; ++r) {
+            acc[r][0] = fmaf(xr[r][ii], m.x, acc[r][0]);
+            acc[r][1] = fmaf(xr[r][ii], m.y, acc[r][1]);
+            acc[r][2] = fmaf(xr[r][ii], m.z, acc[r][2]);
+            acc[r][3] = fmaf(xr[r][ii], m.w, acc[r][3]);
+          }
+        }
       }
     }
+    __syncthreads();  // all reads of x done before the next step rewrites it
 #pragma unroll
-    for (int r = 0; r < 2; ++r)
+    for (int r = 0; r < RR; ++r)
 #pragma unroll
       for (int c = 0; c < 4; ++c) s[r][c] = acc[r][c];
-    __syncthreads();  // everyone is done with buffer `buf` and with x
-    if (tid == 0 && t + 2 < nsteps) issue(t + 2);
-    if (text) store_for(dir == 0 ? 0 : l.F - 1);
-    else store_for(frame_of(t));
+    store_for(text ? (dir == 0 ? 0 : l.F - 1) : f);
   }
+  cp_async_wait<0>();
 }
 
 // Zero the chunk-table entries of chunks without non-boundary frames.
@@ -378,11 +372,8 @@ cudaError_t launch_states_t(const Layout& l, int dtype, const void* k, const voi
   }
   {
     dim3 grid(D / 16, 2, l.B * l.H);
-    const int smem = (int)sizeof(ScanSmem<D>);
-    cudaError_t e = cudaFuncSetAttribute(scan_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    scan_kernel<D><<<grid, 2 * D, smem, st>>>(l, fwd_max, rev_min, map.has_text, am, bw, states);
-    e = cudaGetLastError();
+    scan_kernel<D><<<grid, ScanCfg<D>::kThreads, 0, st>>>(l, fwd_max, rev_min, map.has_text, am, bw, states);
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     zero_unused_chunks<<<dim3(32, l.B * l.H), 256, 0, st>>>(l, states);
   }
