@@ -9,7 +9,8 @@
 //   warps 2-5  scalers: write Kw = beta (.) K next to K as two bf16 parts,
 //              Kw_hi = bf16(beta k) and Kw_lo = bf16(beta k - Kw_hi), so that the
 //              products keep ~16 significant bits of beta k (a single bf16 copy
-//              put the chunk states 1e-2 off); one token row per thread, beta = 0
+//              put the chunk states 1e-2 off); four threads per token row, beta
+//              fetched one tile ahead, beta = 0
 //              past the frame (which also masks the ragged last tile); then the
 //              epilogue reads A and B out of TMEM.
 // Both MMA operands are MN-major (token = K dimension, contiguous along d):
@@ -190,43 +191,49 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     }
   } else {
     // ---------------------------------------------------- scalers / epilogue
-    const int u = threadIdx.x - 64;  // 0..127: (token row, d half) items below
+    // 4 threads per token row, each scaling (D / 8) / 4 of the row's 16-byte chunks;
+    // beta of the next tile is fetched one tile ahead (it is a strided 4-byte read)
+    const int u = threadIdx.x - 64;
+    constexpr int kTpr = 128 / kTok;              // threads per token row
+    constexpr int kCpt = (D / 8) / kTpr;          // 16-byte chunks per thread
+    const int r = u / kTpr, part = u % kTpr;
+    auto beta_of = [&](int t) -> float {
+      const int tok = t * kTok + r;
+      if (tok >= U) return 0.f;
+      return text ? beta_t[((long long)b * l.T + tok) * l.H + h]
+                  : beta[((long long)b * l.L() + row0 + tok) * l.H + h];
+    };
+    float bnext = n_tiles > 0 ? beta_of(0) : 0.f;
     bool ok = true;
     for (int t = 0; t < n_tiles && ok; ++t) {
       const int s = t % C::kStages, use = t / C::kStages;
+      const float bu = bnext;
+      if (t + 1 < n_tiles) bnext = beta_of(t + 1);
       if (!__all_sync(0xffffffffu, gwait(&bars->full[s], use & 1, abort))) {
         ok = false;
         break;
       }
-      // 128 threads, 64 token rows x kHalves halves: thread -> (row, half pair)
       uint8_t* st = smem + s * C::kStageBytes;
-      for (int item = u; item < kTok * C::kHalves; item += 128) {
-        const int r = item % kTok, hf = item / kTok;
-        const int tok = t * kTok + r;
-        float bu = 0.f;
-        if (tok < U)
-          bu = text ? beta_t[((long long)b * l.T + tok) * l.H + h]
-                    : beta[((long long)b * l.L() + row0 + tok) * l.H + h];
-        const uint4* src = reinterpret_cast<const uint4*>(st + hf * kHalfBytes + r * 128);
-        uint4* dhi = reinterpret_cast<uint4*>(st + 2 * C::kTileBytes + hf * kHalfBytes + r * 128);
-        uint4* dlo = reinterpret_cast<uint4*>(st + 3 * C::kTileBytes + hf * kHalfBytes + r * 128);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint4 x = src[c];
-          uint32_t w[4] = {x.x, x.y, x.z, x.w};
-          uint32_t hi4[4], lo4[4];
+      for (int cc = 0; cc < kCpt; ++cc) {
+        const int chunk = part * kCpt + cc;       // 0 .. D/8 - 1 within the row
+        const int hf = chunk / 8, c = chunk % 8;  // (swizzle permutes chunks within a row;
+                                                  //  the scaling does not care which)
+        const int off = hf * kHalfBytes + r * 128 + c * 16;
+        const uint4 x = *reinterpret_cast<const uint4*>(st + off);
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        uint32_t hi4[4], lo4[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float p0 = __uint_as_float(w[e] << 16) * bu;       // even element
-            const float p1 = __uint_as_float(w[e] & 0xFFFF0000u) * bu;  // odd element
-            const float h0 = __bfloat162float(__float2bfloat16_rn(p0));
-            const float h1 = __bfloat162float(__float2bfloat16_rn(p1));
-            hi4[e] = pack_bf16(h0, h1);
-            lo4[e] = pack_bf16(p0 - h0, p1 - h1);
-          }
-          dhi[c] = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
-          dlo[c] = make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
+        for (int e = 0; e < 4; ++e) {
+          const float p0 = __uint_as_float(w[e] << 16) * bu;          // even element
+          const float p1 = __uint_as_float(w[e] & 0xFFFF0000u) * bu;  // odd element
+          const float h0 = __bfloat162float(__float2bfloat16_rn(p0));
+          const float h1 = __bfloat162float(__float2bfloat16_rn(p1));
+          hi4[e] = pack_bf16(h0, h1);
+          lo4[e] = pack_bf16(p0 - h0, p1 - h1);
         }
+        *reinterpret_cast<uint4*>(st + 2 * C::kTileBytes + off) = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
+        *reinterpret_cast<uint4*>(st + 3 * C::kTileBytes + off) = make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       mbar_arrive(&bars->scaled[s]);

@@ -126,6 +126,27 @@ struct HybridArgs {
   __nv_bfloat16* out_lin;          // nullable
 };
 
+// 2^x evaluated on the FMA pipe instead of the MUFU unit, used for a quarter
+// of the softmax exponentials so that the two pipes share the load: n =
+// round(x) via the 1.5 * 2^23 shifter, f = x - n in [-1/2, 1/2], 2^f by a
+// degree-3 polynomial (coefficients fitted for minimax relative error by
+// exp2_poly_fit.py; max relative error 7.5e-5, far below the bf16 rounding of
+// the weights), and 2^n added into the exponent bits. x >= -126 is enforced
+// (smaller results are below anything the bf16 weights keep).
+constexpr float kExp2C0 = 9.999280572e-01f;
+constexpr float kExp2C1 = 6.932609677e-01f;
+constexpr float kExp2C2 = 2.426111400e-01f;
+constexpr float kExp2C3 = 5.517166853e-02f;
+
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -126.f);
+  const float t = x + 12582912.f;
+  const float n = t - 12582912.f;
+  const float f = x - n;
+  const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 __device__ __forceinline__ float sigmoid_fast(float x) {
   return 1.f / (1.f + ex2(-1.4426950408889634f * x));
 }
@@ -401,8 +422,10 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int j = 0; j < 64; ++j) {
-        const float a = ex2(fmaf(s[2 * j], sl2, nm));
-        const float c = ex2(fmaf(s[2 * j + 1], sl2, nm));
+        // every fourth pair on the FMA pipe, the rest on MUFU
+        const float xa = fmaf(s[2 * j], sl2, nm), xc = fmaf(s[2 * j + 1], sl2, nm);
+        const float a = ((j & 3) == 3) ? exp2_fma(xa) : ex2(xa);
+        const float c = ((j & 3) == 3) ? exp2_fma(xc) : ex2(xc);
         rs4[j & 3] += a + c;
         p[j] = pack_bf16(a, c);
       }
