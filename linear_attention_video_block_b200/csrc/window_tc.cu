@@ -126,25 +126,31 @@ struct HybridArgs {
   __nv_bfloat16* out_lin;          // nullable
 };
 
-// 2^x evaluated on the FMA pipe instead of the MUFU unit, used for a quarter
-// of the softmax exponentials so that the two pipes share the load: n =
-// round(x) via the 1.5 * 2^23 shifter, f = x - n in [-1/2, 1/2], 2^f by a
-// degree-3 polynomial (coefficients fitted for minimax relative error by
-// exp2_poly_fit.py; max relative error 7.5e-5, far below the bf16 rounding of
-// the weights), and 2^n added into the exponent bits. x >= -126 is enforced
-// (smaller results are below anything the bf16 weights keep).
-constexpr float kExp2C0 = 9.999280572e-01f;
-constexpr float kExp2C1 = 6.932609677e-01f;
-constexpr float kExp2C2 = 2.426111400e-01f;
-constexpr float kExp2C3 = 5.517166853e-02f;
-
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -126.f);
-  const float t = x + 12582912.f;
-  const float n = t - 12582912.f;
-  const float f = x - n;
-  const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+// Packed fp32 pairs (sm_100 f32x2 arithmetic) and the 3-input max: they halve
+// the instruction count of the softmax's per-element work.
+__device__ __forceinline__ unsigned long long f2pack(float a, float b) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(unsigned long long r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ unsigned long long f2fma(unsigned long long a, unsigned long long b,
+                                                    unsigned long long c) {
+  unsigned long long r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ unsigned long long f2add(unsigned long long a, unsigned long long b) {
+  unsigned long long r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 __device__ __forceinline__ float sigmoid_fast(float x) {
@@ -380,7 +386,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
       tc_fence_after();
       uint32_t sr[128];
-      tmem_ld_x128(tS, sr);
+      tmem_ld_x128_split(tS, sr);
       float* s = reinterpret_cast<float*>(sr);
       const int valid = key_tile(G, l.T, t).valid;
       if (valid < kRows) {
@@ -388,15 +394,15 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int j = 0; j < kRows; ++j)
           if (j >= valid) s[j] = -INFINITY;
       }
-      float mx4[4] = {s[0], s[1], s[2], s[3]};
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int j = 4; j < kRows; j += 4) {
-        mx4[0] = fmaxf(mx4[0], s[j]);
-        mx4[1] = fmaxf(mx4[1], s[j + 1]);
-        mx4[2] = fmaxf(mx4[2], s[j + 2]);
-        mx4[3] = fmaxf(mx4[3], s[j + 3]);
+      for (int j = 0; j < kRows; j += 8) {
+        mx4[0] = fmax3(mx4[0], s[j], s[j + 1]);
+        mx4[1] = fmax3(mx4[1], s[j + 2], s[j + 3]);
+        mx4[2] = fmax3(mx4[2], s[j + 4], s[j + 5]);
+        mx4[3] = fmax3(mx4[3], s[j + 6], s[j + 7]);
       }
-      const float mc = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
+      const float mc = fmaxf(fmax3(mx4[0], mx4[1], mx4[2]), mx4[3]) * sl2;
       if (t == 0) {
         m = mc;
       } else {
@@ -418,19 +424,30 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
       }
       const float nm = -m;
-      uint32_t p[64];
-      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+      const unsigned long long sl2x2 = f2pack(sl2, sl2), nmx2 = f2pack(nm, nm);
+      unsigned long long sum2[2] = {0ull, 0ull};
+      // P goes to TMEM in four 16-column pieces as it is produced
 #pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        // every fourth pair on the FMA pipe, the rest on MUFU
-        const float xa = fmaf(s[2 * j], sl2, nm), xc = fmaf(s[2 * j + 1], sl2, nm);
-        const float a = ((j & 3) == 3) ? exp2_fma(xa) : ex2(xa);
-        const float c = ((j & 3) == 3) ? exp2_fma(xc) : ex2(xc);
-        rs4[j & 3] += a + c;
-        p[j] = pack_bf16(a, c);
+      for (int c4 = 0; c4 < 4; ++c4) {
+        uint32_t p[16];
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) {
+          const int j = 16 * c4 + jj;
+          float xa, xc;
+          f2unpack(f2fma(f2pack(s[2 * j], s[2 * j + 1]), sl2x2, nmx2), xa, xc);
+          const float a = ex2(xa), c = ex2(xc);
+          sum2[jj & 1] = f2add(sum2[jj & 1], f2pack(a, c));
+          p[jj] = pack_bf16(a, c);
+        }
+        tmem_st_x16_nowait(tS + 16 * c4, p);
       }
-      lsum += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
-      tmem_st_x64(tS, p);
+      {
+        float s0, s1, s2, s3;
+        f2unpack(sum2[0], s0, s1);
+        f2unpack(sum2[1], s2, s3);
+        lsum += (s0 + s1) + (s2 + s3);
+      }
+      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bars->p_full[w]);
     }
