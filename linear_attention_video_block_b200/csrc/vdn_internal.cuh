@@ -107,6 +107,60 @@ __host__ __device__ inline void tile_to_group(const Layout& l, int rows, int t, 
   r0 = 0;
 }
 
+// Key tile t of a query group (tiles of `keys` keys): video segments first,
+// then the text keys.
+struct KeyTile {
+  int text;   // 1: rows index the text tensor
+  int row;    // first key row of the tile
+  int valid;  // keys of the tile that belong to the segment (<= keys)
+};
+
+__host__ __device__ inline int key_tile_count(const Group& G, int T, int keys) {
+  int n = 0;
+  for (int s = 0; s < G.nseg; ++s) n += (G.segn[s] + keys - 1) / keys;
+  return n + (T + keys - 1) / keys;
+}
+
+__host__ __device__ inline KeyTile key_tile(const Group& G, int T, int t, int keys) {
+  for (int s = 0; s < G.nseg; ++s) {
+    const int n = (G.segn[s] + keys - 1) / keys;
+    if (t < n) {
+      KeyTile k{0, G.seg0[s] + t * keys, G.segn[s] - t * keys};
+      if (k.valid > keys) k.valid = keys;
+      return k;
+    }
+    t -= n;
+  }
+  KeyTile k{1, t * keys, T - t * keys};
+  if (k.valid > keys) k.valid = keys;
+  return k;
+}
+
+// Order in which the window kernel's K and V tiles fill its slot ring, the
+// same order in which its MMA issuer consumes them: K0, K1 (if any), then for
+// each key tile t: V_t followed by K_{t+2} when that tile exists.
+struct KvFillOrder {
+  int n;
+  __host__ __device__ int total() const { return 2 * n; }
+  __host__ __device__ void at(int i, int& tile, int& is_v) const {
+    const int lead = n < 2 ? n : 2;
+    if (i < lead) {
+      tile = i;
+      is_v = 0;
+      return;
+    }
+    const int j = i - lead;
+    const int paired = n > 2 ? n - 2 : 0;  // tiles t that are followed by K_{t+2}
+    if (j < 2 * paired) {
+      tile = (j & 1) ? j / 2 + 2 : j / 2;
+      is_v = (j & 1) ? 0 : 1;
+    } else {
+      tile = paired + (j - 2 * paired);
+      is_v = 1;
+    }
+  }
+};
+
 // Scan extents: forward scan runs frames 1..fwd_max, reverse scan frames
 // F-2 down to rev_min (rev_min = F-1 means no reverse frame).
 inline void scan_extent(const Layout& l, int& fwd_max, int& rev_min) {

@@ -22,6 +22,27 @@ int main(int argc, char** argv) {
     for (int s = 0; s < G.nseg; ++s) std::printf(" %d:%d", G.seg0[s], G.segn[s]);
     std::printf("\n");
   }
+  for (int g = 0; g < l.groups(); ++g) {
+    vdn::Group G = vdn::make_group(l, g);
+    if (G.nq == 0) continue;
+    const int nk = vdn::key_tile_count(G, l.T, 64);
+    std::printf("keytiles %d", g);
+    for (int t = 0; t < nk; ++t) {
+      vdn::KeyTile k = vdn::key_tile(G, l.T, t, 64);
+      std::printf(" %d:%d:%d", k.text, k.row, k.valid);
+    }
+    std::printf("\n");
+  }
+  for (int n = 1; n <= 9; ++n) {
+    vdn::KvFillOrder o{n};
+    std::printf("fill %d", n);
+    for (int i = 0; i < o.total(); ++i) {
+      int tile, is_v;
+      o.at(i, tile, is_v);
+      std::printf(" %c%d", is_v ? 'V' : 'K', tile);
+    }
+    std::printf("\n");
+  }
   const int nt = vdn::tiles_per_head(l, rows);
   for (int t = 0; t < nt; ++t) {
     int g, r0;
