@@ -136,31 +136,6 @@ __host__ __device__ inline KeyTile key_tile(const Group& G, int T, int t, int ke
   return k;
 }
 
-// Order in which the window kernel's K and V tiles fill its slot ring, the
-// same order in which its MMA issuer consumes them: K0, K1 (if any), then for
-// each key tile t: V_t followed by K_{t+2} when that tile exists.
-struct KvFillOrder {
-  int n;
-  __host__ __device__ int total() const { return 2 * n; }
-  __host__ __device__ void at(int i, int& tile, int& is_v) const {
-    const int lead = n < 2 ? n : 2;
-    if (i < lead) {
-      tile = i;
-      is_v = 0;
-      return;
-    }
-    const int j = i - lead;
-    const int paired = n > 2 ? n - 2 : 0;  // tiles t that are followed by K_{t+2}
-    if (j < 2 * paired) {
-      tile = (j & 1) ? j / 2 + 2 : j / 2;
-      is_v = (j & 1) ? 0 : 1;
-    } else {
-      tile = paired + (j - 2 * paired);
-      is_v = 1;
-    }
-  }
-};
-
 // Scan extents: forward scan runs frames 1..fwd_max, reverse scan frames
 // F-2 down to rev_min (rev_min = F-1 means no reverse frame).
 inline void scan_extent(const Layout& l, int& fwd_max, int& rev_min) {

@@ -6,14 +6,14 @@
 // for every video query, softmax(q K^T / sqrt(d)) V over the keys of its
 // chunk window, the boundary anchor frames and all text tokens, one
 // normaliser. Keys are visited per query group as merged token segments
-// (window/anchor intervals, then text) in 64-key tiles; only the last tile of
+// (window/anchor intervals, then text) in 128-key tiles; only the last tile of
 // each segment is partially masked.
 //
 // CTA = 256 query rows (two 128-row Q tiles) of one query group of one
 // (b, h); 384 threads:
 //   warps 0-3   softmax warpgroup of Q tile 0 (thread i owns row i = TMEM lane i)
 //   warps 4-7   softmax warpgroup of Q tile 1
-//   warp  8     TMA producer (one elected lane): Q once, then K and V tiles
+//   warp  8     TMA producer (one elected lane): Q once, then K_t, V_t tiles
 //               into a ring of shared-memory slots
 //   warp  9     MMA issuer (one elected lane) and TMEM owner
 //   warps 10-11 hybrid epilogue helpers (fused variant only): stage the chunk's
@@ -21,23 +21,18 @@
 //               K-major operand while the mainloop runs, in two parts
 //               S_hi = bf16(S_sum) and S_lo = bf16(S_sum - S_hi), so that the
 //               readout keeps about 16 significant bits of the fp32 state
-//
-// TMEM (512 columns): for Q tile w, two score buffers S_w[0], S_w[1] of 64
-// columns at 128w and 128w + 64, and the output O_w at 256 + d w. Key tile t of
-// Q tile w uses score buffer t mod 2; its bf16 weights P overwrite the first 32
-// columns of that buffer and are the A operand of P.V straight from TMEM.
-// MMA issue order: S0(0) S1(0) S0(1) S1(1), then per key tile t:
-//   PV0(t), PV1(t), S0(t+2), S1(t+2)
-// S_w(t+2) reuses the buffer of tile t right after PV_w(t) has read it
-// (tcgen05.mma runs in issue order), so the next score tile is ready before the
-// softmax of the current one ends and each softmax warpgroup runs from tile to
-// tile without waiting for its own P.V. O is rescaled lazily (only when the
-// running max grows by more than 2^8), after waiting for the previous P.V.
-//
 // Fused hybrid variant (project page, "Gating the Softmax and Linear Branch
 // Outputs"): after the last P.V the MMA issuer computes O_lin = Q S_hi^T +
-// Q S_lo^T into the score columns of TMEM, and each softmax thread, owning a
-// whole row, finishes out = sigmoid(g_s) o_soft + sigmoid(g_l) RMSNorm(o_lin).
+// Q S_lo^T into the freed S columns of TMEM, and each softmax thread, owning a whole row,
+// finishes out = sigmoid(g_s) o_soft + sigmoid(g_l) RMSNorm(o_lin) in registers.
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+d) O1 [256+d,256+2d).
+// P (bf16) overwrites the first 64 columns of S and is the A operand of P.V
+// straight from TMEM. MMA issue order per key tile t:
+//   PV0(t), S0(t+1), PV1(t), S1(t+1)
+// so softmax of one Q tile overlaps the tensor-core work of the other.
+// The tcgen05.commit after S_w(t) also covers PV_w(t-1), so when softmax w sees
+// S_w(t) its O accumulator is stable and can be rescaled in place (lazy
+// rescaling: only when the running max grows by more than 2^8).
 //
 // Every mbarrier wait is bounded (%globaltimer, 4 s); a timeout records
 // VDN_ERR_TIMEOUT in the status word, the roles leave their loops, the
@@ -59,33 +54,29 @@ cudaError_t read_and_clear_tc_status(int* status) {
 
 namespace {
 
-constexpr int kRows = 128;           // rows of a Q tile
-constexpr int kKeys = 64;            // keys of a K/V tile
+constexpr int kRows = 128;           // rows of a Q tile = keys of a K/V tile
 constexpr int kThreads = 384;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kTmemCols = 512;
-constexpr int kSlots = 8;
 
 template <int D>
 struct Cfg {
   static constexpr int kHalves = D / 64;               // 128-byte swizzle atoms per row
-  static constexpr int kQTileBytes = kRows * D * 2;    // one 128 x D bf16 Q tile
-  static constexpr int kQHalfBytes = kRows * 128;      // 128 rows x 64 columns
-  static constexpr int kKvTileBytes = kKeys * D * 2;   // one 64 x D bf16 K or V tile
-  static constexpr int kKvHalfBytes = kKeys * 128;     // 64 rows x 64 columns
-  static constexpr int kQBytes = 2 * kQTileBytes;
-  static constexpr int kSsumBytes = kRows * D * 2;     // bf16 S_sum (fused only)
-  static constexpr int kSmemBytes = 1024 + kQBytes + kSlots * kKvTileBytes + kSsumBytes + 256;
+  static constexpr int kTileBytes = kRows * D * 2;     // one 128 x D bf16 tile
+  static constexpr int kHalfBytes = kRows * 128;       // one 128-row x 64-column atom column
+  static constexpr int kSlots = (D == 128) ? 4 : 8;
+  static constexpr int kQBytes = 2 * kTileBytes;
+  static constexpr int kSsumBytes = kRows * D * 2;     // bf16 S_sum, 128 x D (fused only)
+  static constexpr int kSmemBytes = 1024 + kQBytes + kSlots * kTileBytes + kSsumBytes + 256;
 };
 
 struct Bars {
   unsigned long long q_full;
-  unsigned long long kv_full[kSlots];
-  unsigned long long kv_empty[kSlots];
-  unsigned long long s_full[2][2];   // [Q tile][score buffer]
-  unsigned long long p_full[2][2];
-  unsigned long long pv_done[2];     // one phase per P.V of each Q tile
+  unsigned long long kv_full[8];
+  unsigned long long kv_empty[8];
+  unsigned long long s_full[2];
+  unsigned long long p_full[2];
   unsigned long long o_full;
   unsigned long long ssum_ready;
   unsigned long long ssum_free;
@@ -156,7 +147,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = smem;
   uint8_t* sKV = smem + C::kQBytes;
-  uint8_t* sSsum = sKV + kSlots * C::kKvTileBytes;
+  uint8_t* sSsum = sKV + C::kSlots * C::kTileBytes;
   Bars* bars = reinterpret_cast<Bars*>(sSsum + (kFuse ? C::kSsumBytes : 0));
 
   const int warp = threadIdx.x / 32;
@@ -165,22 +156,18 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   int g, r0;
   tile_to_group(l, 2 * kRows, blockIdx.x, g, r0);
   const Group G = make_group(l, g < 0 ? 0 : g);
-  const int n_tiles = key_tile_count(G, l.T, kKeys);
+  const int n_tiles = key_tile_count(G, l.T, kRows);
   const bool has_lin = kFuse && G.chunk >= 0;
-  const KvFillOrder order{n_tiles};
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
-    for (int i = 0; i < kSlots; ++i) {
+    for (int i = 0; i < C::kSlots; ++i) {
       mbar_init(&bars->kv_full[i], 1);
       mbar_init(&bars->kv_empty[i], 1);
     }
     for (int w = 0; w < 2; ++w) {
-      for (int bf = 0; bf < 2; ++bf) {
-        mbar_init(&bars->s_full[w][bf], 1);
-        mbar_init(&bars->p_full[w][bf], 128);
-      }
-      mbar_init(&bars->pv_done[w], 1);
+      mbar_init(&bars->s_full[w], 1);
+      mbar_init(&bars->p_full[w], 128);
     }
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->ssum_ready, 64);
@@ -203,40 +190,43 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   if (warp == kProducerWarp) {
     if (lane == 0 && !*abort) {
       // ------------------------------------------------------- TMA producer
-      mbar_expect_tx(&bars->q_full, 2 * C::kQTileBytes);
+      mbar_expect_tx(&bars->q_full, 2 * C::kTileBytes);
       for (int qt = 0; qt < 2; ++qt)
         for (int hf = 0; hf < C::kHalves; ++hf)
-          tma_load_4d(sQ + qt * C::kQTileBytes + hf * C::kQHalfBytes, &tm_q, &bars->q_full, hf * 64,
+          tma_load_4d(sQ + qt * C::kTileBytes + hf * C::kHalfBytes, &tm_q, &bars->q_full, hf * 64,
                       h, r0 + qt * kRows, b);
-      const int total = order.total();
       int fill = 0;
-      for (; fill < total; ++fill) {
-        const int slot = fill % kSlots;
-        const int use = fill / kSlots;
-        if (use > 0 && !mbar_wait(&bars->kv_empty[slot], (use - 1) & 1, abort)) break;
-        int tile, is_v;
-        order.at(fill, tile, is_v);
-        const KeyTile kt = key_tile(G, l.T, tile, kKeys);
-        const CUtensorMap* map = kt.text ? (is_v ? &tm_vt : &tm_kt) : (is_v ? &tm_v : &tm_k);
-        mbar_expect_tx(&bars->kv_full[slot], C::kKvTileBytes);
-        for (int hf = 0; hf < C::kHalves; ++hf)
-          tma_load_4d(sKV + slot * C::kKvTileBytes + hf * C::kKvHalfBytes, map, &bars->kv_full[slot],
-                      hf * 64, h, kt.row, b);
+      bool ok = true;
+      for (int t = 0; t < n_tiles && ok; ++t) {
+        const KeyTile kt = key_tile(G, l.T, t, kRows);
+        for (int kv = 0; kv < 2; ++kv, ++fill) {
+          const int slot = fill % C::kSlots;
+          const int use = fill / C::kSlots;
+          if (use > 0 && !mbar_wait(&bars->kv_empty[slot], (use - 1) & 1, abort)) {
+            ok = false;
+            break;
+          }
+          const CUtensorMap* map = kt.text ? (kv ? &tm_vt : &tm_kt) : (kv ? &tm_v : &tm_k);
+          mbar_expect_tx(&bars->kv_full[slot], C::kTileBytes);
+          for (int hf = 0; hf < C::kHalves; ++hf)
+            tma_load_4d(sKV + slot * C::kTileBytes + hf * C::kHalfBytes, map, &bars->kv_full[slot],
+                        hf * 64, h, kt.row, b);
+        }
       }
-      if (fill < total) {
+      if (!ok) {
         // leave no copy in flight into this CTA's shared memory: the last fill
         // of slot s was number (fill - 1 - ((fill - 1 - s) mod kSlots))
         mbar_wait(&bars->q_full, 0, abort, false);
-        for (int s = 0; s < kSlots && s < fill; ++s) {
-          const int last = fill - 1 - ((fill - 1 - s) % kSlots);
-          mbar_wait(&bars->kv_full[s], (last / kSlots) & 1, abort, false);
+        for (int s = 0; s < C::kSlots && s < fill; ++s) {
+          const int last = fill - 1 - ((fill - 1 - s) % C::kSlots);
+          mbar_wait(&bars->kv_full[s], (last / C::kSlots) & 1, abort, false);
         }
       }
     }
   } else if (warp == kMmaWarp) {
     if (lane == 0 && !*abort) {
       // ------------------------------------------------------- MMA issuer
-      constexpr uint32_t idesc_s = make_idesc(kKeys, false);
+      constexpr uint32_t idesc_s = make_idesc(kRows, false);
       constexpr uint32_t idesc_o = make_idesc(D, true);
       constexpr uint32_t idesc_lin = make_idesc(D, false);
       const uint32_t q_addr = smem_u32(sQ);
@@ -244,64 +234,67 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       int use = 0;
       bool ok = mbar_wait(&bars->q_full, 0, abort);
       auto take_slot = [&](int& slot) -> bool {
-        slot = use % kSlots;
-        const bool r = mbar_wait(&bars->kv_full[slot], (use / kSlots) & 1, abort);
+        slot = use % C::kSlots;
+        const bool r = mbar_wait(&bars->kv_full[slot], (use / C::kSlots) & 1, abort);
         ++use;
         tc_fence_after();
         return r;
       };
-      // S_w(t) = Q_w K_t^T into score buffer t mod 2 of Q tile w
-      auto issue_s = [&](int w, int t, int slot) {
-        const uint32_t d_tmem = tmem + 128 * w + 64 * (t & 1);
+      auto issue_s = [&](int w, int slot) {
+        const uint32_t d_tmem = tmem + 128 * w;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t qoff = (uint32_t)((ks / 4) * C::kQHalfBytes + (ks % 4) * 32);
-          const uint32_t koff = (uint32_t)((ks / 4) * C::kKvHalfBytes + (ks % 4) * 32);
-          mma_ss(d_tmem, desc_k_sw128(q_addr + w * C::kQTileBytes + qoff),
-                 desc_k_sw128(kv_addr + slot * C::kKvTileBytes + koff), idesc_s, ks > 0 ? 1u : 0u);
+          const uint32_t off = (uint32_t)((ks / 4) * C::kHalfBytes + (ks % 4) * 32);
+          mma_ss(d_tmem, desc_k_sw128(q_addr + w * C::kTileBytes + off),
+                 desc_k_sw128(kv_addr + slot * C::kTileBytes + off), idesc_s, ks > 0 ? 1u : 0u);
         }
       };
-      // O_w += P_w(t) V_t, P from the first 32 columns of score buffer t mod 2
-      auto issue_pv = [&](int w, int t, int slot) {
+      auto issue_pv = [&](int w, int slot, bool acc) {
         const uint32_t d_tmem = tmem + 256 + D * w;
-        const uint32_t a_tmem = tmem + 128 * w + 64 * (t & 1);
+        const uint32_t a_tmem = tmem + 128 * w;
 #pragma unroll
-        for (int ks = 0; ks < kKeys / 16; ++ks) {
+        for (int ks = 0; ks < kRows / 16; ++ks) {
           mma_ts(d_tmem, a_tmem + ks * 8,
-                 desc_mn_sw128(kv_addr + slot * C::kKvTileBytes + ks * 16 * 128, C::kKvHalfBytes),
-                 idesc_o, (t > 0 || ks > 0) ? 1u : 0u);
+                 desc_mn_sw128(kv_addr + slot * C::kTileBytes + ks * 16 * 128, C::kHalfBytes),
+                 idesc_o, (acc || ks > 0) ? 1u : 0u);
         }
       };
-      auto issue_both_s = [&](int t) -> bool {
-        int ks;
-        if (!take_slot(ks)) return false;
-        issue_s(0, t, ks);
-        tc_commit(&bars->s_full[0][t & 1]);
-        issue_s(1, t, ks);
-        tc_commit(&bars->s_full[1][t & 1]);
-        tc_commit(&bars->kv_empty[ks]);
-        return true;
-      };
-      if (ok) ok = issue_both_s(0);
-      if (ok && n_tiles > 1) ok = issue_both_s(1);
+      int ks_cur = 0;
+      if (ok) ok = take_slot(ks_cur);
+      if (ok) {
+        issue_s(0, ks_cur);
+        tc_commit(&bars->s_full[0]);
+        issue_s(1, ks_cur);
+        tc_commit(&bars->s_full[1]);
+        tc_commit(&bars->kv_empty[ks_cur]);
+      }
       for (int t = 0; t < n_tiles && ok; ++t) {
-        int vs = 0;
+        int vs = 0, ks_next = 0;
         if (!take_slot(vs)) { ok = false; break; }
-        for (int w = 0; w < 2; ++w) {
-          if (!mbar_wait(&bars->p_full[w][t & 1], (t >> 1) & 1, abort)) { ok = false; break; }
-          tc_fence_after();
-          issue_pv(w, t, vs);
-          tc_commit(&bars->pv_done[w]);
+        if (!mbar_wait(&bars->p_full[0], t & 1, abort)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(0, vs, t > 0);
+        const bool more = t + 1 < n_tiles;
+        if (more) {
+          if (!take_slot(ks_next)) { ok = false; break; }
+          issue_s(0, ks_next);
+          tc_commit(&bars->s_full[0]);
         }
-        if (!ok) break;
+        if (!mbar_wait(&bars->p_full[1], t & 1, abort)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(1, vs, t > 0);
         tc_commit(&bars->kv_empty[vs]);
-        if (t + 2 < n_tiles && !issue_both_s(t + 2)) { ok = false; break; }
+        if (more) {
+          issue_s(1, ks_next);
+          tc_commit(&bars->s_full[1]);
+          tc_commit(&bars->kv_empty[ks_next]);
+        }
       }
       if (ok && has_lin) {
-        // O_lin_w = Q_w S_hi^T + Q_w S_lo^T into the score columns of Q tile w
-        // (issued after the last P.V, which reads P from those columns). The
-        // helpers restage S_lo into the same buffer once the S_hi products
-        // have completed.
+        // O_lin_w = Q_w S_hi^T + Q_w S_lo^T into the S columns of TMEM (issued after
+        // the last P.V, which reads P from those columns; tcgen05.mma runs in
+        // issue order). The helpers restage S_lo into the same buffer once the
+        // S_hi products have completed.
         const uint32_t s_addr = smem_u32(sSsum);
         for (int part = 0; part < 2 && ok; ++part) {
           ok = mbar_wait(&bars->ssum_ready, part, abort);
@@ -310,8 +303,8 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           for (int w = 0; w < 2; ++w) {
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
-              const uint32_t off = (uint32_t)((ks / 4) * C::kQHalfBytes + (ks % 4) * 32);
-              mma_ss(tmem + 128 * w, desc_k_sw128(q_addr + w * C::kQTileBytes + off),
+              const uint32_t off = (uint32_t)((ks / 4) * C::kHalfBytes + (ks % 4) * 32);
+              mma_ss(tmem + 128 * w, desc_k_sw128(q_addr + w * C::kTileBytes + off),
                      desc_k_sw128(s_addr + off), idesc_lin, (part > 0 || ks > 0) ? 1u : 0u);
             }
           }
@@ -334,7 +327,6 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (part == 1 && !mbar_wait(&bars->ssum_free, 0, abort)) break;
         for (int ch = t; ch < kRows * kChunks; ch += 64) {
           const int n = ch / kChunks, kc = ch % kChunks;
-          if (n >= D) continue;  // the readout MMA reads N = d rows of S_sum
           const float4 a0 = *reinterpret_cast<const float4*>(sf + n * D + kc * 8);
           const float4 a1 = *reinterpret_cast<const float4*>(sf + n * D + kc * 8 + 4);
           const float4 b0 = *reinterpret_cast<const float4*>(sr + n * D + kc * 8);
@@ -348,7 +340,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           const uint4 v = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]),
                                      pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
           const int half = kc / 8, c16 = kc % 8;
-          *reinterpret_cast<uint4*>(sSsum + half * C::kQHalfBytes + n * 128 + ((c16 ^ (n & 7)) * 16)) = v;
+          *reinterpret_cast<uint4*>(sSsum + half * C::kHalfBytes + n * 128 + ((c16 ^ (n & 7)) * 16)) = v;
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_arrive(&bars->ssum_ready);
@@ -359,31 +351,30 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int w = warp / 4;
     const int row = threadIdx.x & 127;
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-    const uint32_t tSw = tmem + lane_base + 128 * w;     // score buffers of Q tile w
+    const uint32_t tS = tmem + lane_base + 128 * w;
     const uint32_t tO = tmem + lane_base + 256 + D * w;
     const float sl2 = 1.4426950408889634f / sqrtf((float)D);  // log2(e) / sqrt(d)
     float m = -INFINITY, lsum = 0.f;
     bool ok = !*abort;
     for (int t = 0; t < n_tiles && ok; ++t) {
-      const uint32_t tS = tSw + 64 * (t & 1);
       // the TMEM loads below are warp-collective: leave only as a whole warp
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[w][t & 1], (t >> 1) & 1, abort))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[w], t & 1, abort))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t sr[64];
-      tmem_ld_x64(tS, sr);
+      uint32_t sr[128];
+      tmem_ld_x128_split(tS, sr);
       float* s = reinterpret_cast<float*>(sr);
-      const int valid = key_tile(G, l.T, t, kKeys).valid;
-      if (valid < kKeys) {
+      const int valid = key_tile(G, l.T, t, kRows).valid;
+      if (valid < kRows) {
 #pragma unroll
-        for (int j = 0; j < kKeys; ++j)
+        for (int j = 0; j < kRows; ++j)
           if (j >= valid) s[j] = -INFINITY;
       }
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int j = 0; j < kKeys; j += 8) {
+      for (int j = 0; j < kRows; j += 8) {
         mx4[0] = fmax3(mx4[0], s[j], s[j + 1]);
         mx4[1] = fmax3(mx4[1], s[j + 2], s[j + 3]);
         mx4[2] = fmax3(mx4[2], s[j + 4], s[j + 5]);
@@ -395,13 +386,6 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       } else {
         const bool need = mc > m + 8.f;
         if (__any_sync(0xffffffffu, need)) {
-          // O must be stable: P.V of tile t - 1 complete (tile t's is not issued
-          // before this thread publishes P(t))
-          if (!__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[w], (t - 1) & 1, abort))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
           const float f = need ? ex2(m - mc) : 1.f;
 #pragma unroll 1
           for (int c0 = 0; c0 < D; c0 += 32) {
@@ -420,20 +404,20 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const float nm = -m;
       const unsigned long long sl2x2 = f2pack(sl2, sl2), nmx2 = f2pack(nm, nm);
       unsigned long long sum2[2] = {0ull, 0ull};
-      // P goes to TMEM in two 16-column pieces as it is produced
+      // P goes to TMEM in four 16-column pieces as it is produced
 #pragma unroll
-      for (int c2 = 0; c2 < 2; ++c2) {
+      for (int c4 = 0; c4 < 4; ++c4) {
         uint32_t p[16];
 #pragma unroll
         for (int jj = 0; jj < 16; ++jj) {
-          const int j = 16 * c2 + jj;
+          const int j = 16 * c4 + jj;
           float xa, xc;
           f2unpack(f2fma(f2pack(s[2 * j], s[2 * j + 1]), sl2x2, nmx2), xa, xc);
           const float a = ex2(xa), c = ex2(xc);
           sum2[jj & 1] = f2add(sum2[jj & 1], f2pack(a, c));
           p[jj] = pack_bf16(a, c);
         }
-        tmem_st_x16_nowait(tS + 16 * c2, p);
+        tmem_st_x16_nowait(tS + 16 * c4, p);
       }
       {
         float s0, s1, s2, s3;
@@ -443,7 +427,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars->p_full[w][t & 1]);
+      mbar_arrive(&bars->p_full[w]);
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_full, 0, abort));
     if (ok) {
@@ -484,7 +468,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll 1
           for (int c0 = 0; c0 < D; c0 += 32) {
             uint32_t o[32];
-            tmem_ld_x32(tSw + c0, o);
+            tmem_ld_x32(tS + c0, o);
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               const float x = __uint_as_float(o[i]);
@@ -497,7 +481,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t os[32], ol[32];
           tmem_ld_x32(tO + c0, os);
-          if (has_lin) tmem_ld_x32(tSw + c0, ol);
+          if (has_lin) tmem_ld_x32(tS + c0, ol);
           if (store) {
             const uint4* gsp = reinterpret_cast<const uint4*>(hy.g_soft + base + c0);
             const uint4* glp = reinterpret_cast<const uint4*>(hy.g_lin + base + c0);
@@ -550,17 +534,19 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   }
 }
 
+// ------------------------------------------------------------------- host
+
 template <int D, bool kFuse>
 cudaError_t launch_tc_t(const Layout& l, const void* q, const void* k, const void* v,
                         const void* kt, const void* vt, void* o, bool out_f32, float* lse,
                         const HybridArgs& hy, cudaStream_t st) {
   CUtensorMap mq, mk, mv, mkt, mvt;
   const long long L = l.L();
-  if (!make_map(&mq, q, D, l.H, L, l.B, kRows) || !make_map(&mk, k, D, l.H, L, l.B, kKeys) ||
-      !make_map(&mv, v, D, l.H, L, l.B, kKeys))
+  if (!make_map(&mq, q, D, l.H, L, l.B) || !make_map(&mk, k, D, l.H, L, l.B) ||
+      !make_map(&mv, v, D, l.H, L, l.B))
     return cudaErrorInvalidValue;
   if (l.T > 0) {
-    if (!make_map(&mkt, kt, D, l.H, l.T, l.B, kKeys) || !make_map(&mvt, vt, D, l.H, l.T, l.B, kKeys))
+    if (!make_map(&mkt, kt, D, l.H, l.T, l.B) || !make_map(&mvt, vt, D, l.H, l.T, l.B))
       return cudaErrorInvalidValue;
   } else {
     mkt = mk;  // never read: no text tiles

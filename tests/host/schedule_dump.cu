@@ -25,21 +25,11 @@ int main(int argc, char** argv) {
   for (int g = 0; g < l.groups(); ++g) {
     vdn::Group G = vdn::make_group(l, g);
     if (G.nq == 0) continue;
-    const int nk = vdn::key_tile_count(G, l.T, 64);
+    const int nk = vdn::key_tile_count(G, l.T, 128);
     std::printf("keytiles %d", g);
     for (int t = 0; t < nk; ++t) {
-      vdn::KeyTile k = vdn::key_tile(G, l.T, t, 64);
+      vdn::KeyTile k = vdn::key_tile(G, l.T, t, 128);
       std::printf(" %d:%d:%d", k.text, k.row, k.valid);
-    }
-    std::printf("\n");
-  }
-  for (int n = 1; n <= 9; ++n) {
-    vdn::KvFillOrder o{n};
-    std::printf("fill %d", n);
-    for (int i = 0; i < o.total(); ++i) {
-      int tile, is_v;
-      o.at(i, tile, is_v);
-      std::printf(" %c%d", is_v ? 'V' : 'K', tile);
     }
     std::printf("\n");
   }

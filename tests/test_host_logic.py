@@ -92,7 +92,7 @@ def _parse(text, extras=None):
     extent = None
     for line in text.splitlines():
         t = line.split()
-        if extras is not None and t[0] in ("keytiles", "fill"):
+        if extras is not None and t[0] == "keytiles":
             extras.setdefault(t[0], {})[int(t[1])] = t[2:]
             continue
         if t[0] == "extent":
@@ -150,7 +150,7 @@ def test_cuda_schedule_matches_oracle_key_sets(schedule_dump, F, c):
 
 @pytest.mark.parametrize("F,c,N,T", [(7, 2, 70, 130), (36, 5, 100, 64), (3, 1, 50, 0), (1, 3, 200, 7)])
 def test_key_tiles_cover_segments_exactly(schedule_dump, F, c, N, T):
-    """64-key tiles of the window kernel: video segments in order, then text;
+    """128-key tiles of the window kernel: video segments in order, then text;
     every key of the group's key set appears in exactly one tile, only the last
     tile of a segment is partial."""
     r = subprocess.run([schedule_dump, str(F), str(N), str(c), "4"], check=True, capture_output=True,
@@ -166,23 +166,9 @@ def test_key_tiles_cover_segments_exactly(schedule_dump, F, c, N, T):
         text_tiles = [(row, valid) for text, row, valid in tiles if text == 1]
         keys = []
         for row, valid in video:
-            assert 1 <= valid <= 64
+            assert 1 <= valid <= 128
             keys += list(range(row, row + valid))
         assert sorted(keys) == sorted(k for s0, sn in G["segs"] for k in range(s0, s0 + sn))
         assert len(keys) == len(set(keys))
         assert [v for _, v in text_tiles] == [1]  # the dump program uses one text token
 
-
-def test_kv_fill_order_matches_mma_consumption(schedule_dump):
-    """The producer's fill order equals the order in which the MMA issuer takes
-    tiles: K0, K1, then per key tile t: V_t and K_{t+2} when it exists."""
-    r = subprocess.run([schedule_dump, "4", "3", "2", "4"], check=True, capture_output=True, text=True)
-    extras = {}
-    _parse(r.stdout, extras)
-    for n in range(1, 10):
-        want = ["K0"] + (["K1"] if n > 1 else [])
-        for t in range(n):
-            want.append(f"V{t}")
-            if t + 2 < n:
-                want.append(f"K{t + 2}")
-        assert extras["fill"][n] == want, n
