@@ -48,7 +48,8 @@
  * Ownership and execution. Every pointer is caller-owned device memory, except
  * the layout struct which is read on the host during the call. The library
  * allocates no memory and keeps no state between calls besides a device-side
- * status word (vdn_device_status). Calls are asynchronous on `stream`;
+ * status word (vdn_device_status) and the static scratch array used by
+ * vdn_vda_scan_fwd_noalloc. Calls are asynchronous on `stream`;
  * the return code reports host-detectable errors (VDN_ERR_INVALID for a bad
  * layout or a NULL required pointer, VDN_ERR_UNSUPPORTED for a dtype/d
  * combination not built or a pointer not 16-byte aligned, VDN_ERR_WORKSPACE
@@ -125,6 +126,31 @@ int vdn_hybrid_attn_fwd(const vdn_layout_t* layout, int dtype,
                         const float* rms_weight, float rms_eps,
                         void* out, void* out_soft, void* out_lin,
                         void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Size of the device scratch array behind vdn_vda_scan_fwd_noalloc: 64 MiB. */
+#define VDN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+/* The linear-branch entry point for callers that cannot allocate device
+ * memory where they run this op (for example a plugin inside an inference
+ * engine that owns all device memory and hands plugins no workspace, or a
+ * serving loop that forbids device allocations after start-up because
+ * cudaMalloc and cudaFree can synchronise the device). The pages have no
+ * counterpart to it; it is an interface variant, not a different computation.
+ * Same arguments and results as vdn_vda_scan_fwd without the workspace: the
+ * scratch lives in a static device array of VDN_NOALLOC_SCRATCH_BYTES that
+ * every GPU loading the library holds until the process exits. It needs
+ * 2 B H F d^2 4 bytes, plus B H 2 ceil(F/c) d^2 4 bytes when chunk_states is
+ * NULL (each part rounded up to 256); a layout needing more returns
+ * VDN_ERR_WORKSPACE and launches nothing. The call allocates nothing. The
+ * first call on each device looks up the array's device address; make that
+ * first call before any stream capture. All calls share the array and it
+ * keeps the last call's contents (nothing in it needs to start at zero):
+ * calls that overlap on the GPU race with each other and must be serialised. */
+int vdn_vda_scan_fwd_noalloc(const vdn_layout_t* layout, int dtype,
+                             const void* q, const void* k, const void* v,
+                             const void* k_text, const void* v_text,
+                             const float* beta, const float* beta_text,
+                             void* o_lin, float* chunk_states, cudaStream_t stream);
 
 /* Reads and clears the device-side status word on the current device
  * (synchronises the device). VDN_ERR_TIMEOUT means a kernel gave up a bounded

@@ -183,6 +183,28 @@ def hybrid_attn_fwd(layout: Layout, q, k, v, k_text, v_text, beta, beta_text, g_
     return out
 
 
+NOALLOC_SCRATCH_BYTES = 64 << 20
+
+
+def vda_scan_fwd_noalloc(layout: Layout, q, k, v, k_text, v_text, beta, beta_text, o_lin,
+                         chunk_states=None):
+    """Linear branch without a workspace and without allocating: for callers
+    that cannot allocate device memory where they run the op. Scratch comes
+    from a static 64 MiB device array inside the library (shared by all calls;
+    overlapping calls race). o_lin (and chunk_states, if wanted) are
+    caller-provided device tensors."""
+    _require_cuda()
+    f = lib().vdn_vda_scan_fwd_noalloc
+    if f.argtypes is None:
+        f.argtypes = [ctypes.POINTER(_CLayout), ctypes.c_int] + [ctypes.c_void_p] * 10
+        f.restype = ctypes.c_int
+    code = f(ctypes.byref(_clayout(layout)), _dtype_code(q), _ptr(q), _ptr(k), _ptr(v),
+             _ptr(k_text), _ptr(v_text), _ptr(beta), _ptr(beta_text), _ptr(o_lin),
+             _ptr(chunk_states), _stream(q.device))
+    _check(code, "vdn_vda_scan_fwd_noalloc")
+    return o_lin
+
+
 def device_status() -> int:
     """Reads and clears libvdn's device status word (synchronises the device)."""
     return int(lib().vdn_device_status())
