@@ -80,7 +80,6 @@ struct Bars {
   unsigned long long o_full;
   unsigned long long ssum_ready;
   unsigned long long ssum_free;
-  unsigned long long seq[2];   // exp-phase turns: [0] Q tile 1 done (tile t), [1] Q tile 0 done
   uint32_t tmem_base;
   int abort;
 };
@@ -173,8 +172,6 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->ssum_ready, 64);
     mbar_init(&bars->ssum_free, 1);
-    mbar_init(&bars->seq[0], 128);
-    mbar_init(&bars->seq[1], 128);
     bars->abort = (g < 0) ? 1 : 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -404,18 +401,6 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           }
         }
       }
-      // The two softmax warpgroups take turns for the exponentials (they share
-      // the MUFU units): Q tile 0 computes tile t, then Q tile 1 tile t, then
-      // Q tile 0 tile t + 1, ... Loading S and the row max above overlap the
-      // other warpgroup's turn.
-      {
-        const bool turn = (w == 0) ? (t == 0 || mbar_wait(&bars->seq[0], (t - 1) & 1, abort))
-                                   : mbar_wait(&bars->seq[1], t & 1, abort);
-        if (!__all_sync(0xffffffffu, turn)) {
-          ok = false;
-          break;
-        }
-      }
       const float nm = -m;
       const unsigned long long sl2x2 = f2pack(sl2, sl2), nmx2 = f2pack(nm, nm);
       unsigned long long sum2[2] = {0ull, 0ull};
@@ -434,7 +419,6 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         tmem_st_x16_nowait(tS + 16 * c4, p);
       }
-      mbar_arrive(&bars->seq[w == 0 ? 1 : 0]);  // the other warpgroup's turn
       {
         float s0, s1, s2, s3;
         f2unpack(sum2[0], s0, s1);
