@@ -168,6 +168,15 @@ __device__ __forceinline__ void tmem_st_x16_nowait(uint32_t taddr, const uint32_
                : "memory");
 }
 
+// Stores 8 consecutive 32-bit TMEM columns of this thread's lane without
+// waiting (pair with tmem_st_wait before the data is consumed).
+__device__ __forceinline__ void tmem_st_x8_nowait(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};\n"
+               :
+               : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }

@@ -115,23 +115,35 @@ struct KeyTile {
   int valid;  // keys of the tile that belong to the segment (<= keys)
 };
 
+// (The loops below run over the at most 3 video segments with compile-time
+// indices, so a Group stays in registers on the device.)
 __host__ __device__ inline int key_tile_count(const Group& G, int T, int keys) {
   int n = 0;
-  for (int s = 0; s < G.nseg; ++s) n += (G.segn[s] + keys - 1) / keys;
+#pragma unroll
+  for (int s = 0; s < 3; ++s)
+    if (s < G.nseg) n += (G.segn[s] + keys - 1) / keys;
   return n + (T + keys - 1) / keys;
 }
 
 __host__ __device__ inline KeyTile key_tile(const Group& G, int T, int t, int keys) {
-  for (int s = 0; s < G.nseg; ++s) {
-    const int n = (G.segn[s] + keys - 1) / keys;
-    if (t < n) {
-      KeyTile k{0, G.seg0[s] + t * keys, G.segn[s] - t * keys};
-      if (k.valid > keys) k.valid = keys;
-      return k;
+  KeyTile k{1, 0, 0};
+  bool found = false;
+  int first = 0;  // first tile index of segment s
+#pragma unroll
+  for (int s = 0; s < 3; ++s) {
+    const int n = (s < G.nseg) ? (G.segn[s] + keys - 1) / keys : 0;
+    if (!found && t < first + n) {
+      k.text = 0;
+      k.row = G.seg0[s] + (t - first) * keys;
+      k.valid = G.segn[s] - (t - first) * keys;
+      found = true;
     }
-    t -= n;
+    first += n;
   }
-  KeyTile k{1, t * keys, T - t * keys};
+  if (!found) {
+    k.row = (t - first) * keys;
+    k.valid = T - (t - first) * keys;
+  }
   if (k.valid > keys) k.valid = keys;
   return k;
 }

@@ -10,17 +10,16 @@
 // each segment is partially masked.
 //
 // CTA = 256 query rows (two 128-row Q tiles) of one query group of one
-// (b, h); 384 threads:
+// (b, h); 320 threads (at most 200 registers each):
 //   warps 0-3   softmax warpgroup of Q tile 0 (thread i owns row i = TMEM lane i)
 //   warps 4-7   softmax warpgroup of Q tile 1
-//   warp  8     TMA producer (one elected lane): Q once, then K_t, V_t tiles
-//               into a ring of shared-memory slots
+//   warp  8     lane 0: TMA producer (Q once, then K_t, V_t tiles into a ring
+//               of shared-memory slots); lanes 1-31 (fused variant only) stage
+//               the chunk's VDA read state S_sum = S_fwd + S_rev in shared
+//               memory as a bf16 K-major operand while the mainloop runs, in
+//               two parts S_hi = bf16(S_sum) and S_lo = bf16(S_sum - S_hi), so
+//               that the readout keeps about 16 significant bits of the state
 //   warp  9     MMA issuer (one elected lane) and TMEM owner
-//   warps 10-11 hybrid epilogue helpers (fused variant only): stage the chunk's
-//               VDA read state S_sum = S_fwd + S_rev in shared memory as a bf16
-//               K-major operand while the mainloop runs, in two parts
-//               S_hi = bf16(S_sum) and S_lo = bf16(S_sum - S_hi), so that the
-//               readout keeps about 16 significant bits of the fp32 state
 // Fused hybrid variant (project page, "Gating the Softmax and Linear Branch
 // Outputs"): after the last P.V the MMA issuer computes O_lin = Q S_hi^T +
 // Q S_lo^T into the freed S columns of TMEM, and each softmax thread, owning a whole row,
@@ -55,7 +54,7 @@ cudaError_t read_and_clear_tc_status(int* status) {
 namespace {
 
 constexpr int kRows = 128;           // rows of a Q tile = keys of a K/V tile
-constexpr int kThreads = 384;
+constexpr int kThreads = 320;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kTmemCols = 512;
@@ -170,7 +169,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       mbar_init(&bars->p_full[w], 128);
     }
     mbar_init(&bars->o_full, 1);
-    mbar_init(&bars->ssum_ready, 64);
+    mbar_init(&bars->ssum_ready, 31);
     mbar_init(&bars->ssum_free, 1);
     bars->abort = (g < 0) ? 1 : 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -188,6 +187,36 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   volatile int* abort = &bars->abort;
 
   if (warp == kProducerWarp) {
+    // ---------------------------------------------- S_sum staging (fused)
+    if (lane > 0 && has_lin && !*abort) {
+      const int t = lane - 1;  // 31 staging lanes
+      const int J = l.J();
+      const float* sf = hy.states + ((((long long)b * l.H + h) * 2 + 0) * J + G.chunk) * D * D;
+      const float* sr = hy.states + ((((long long)b * l.H + h) * 2 + 1) * J + G.chunk) * D * D;
+      constexpr int kChunks = D / 8;  // 16-byte chunks per row
+      for (int part = 0; part < 2; ++part) {
+        if (part == 1 && !mbar_wait(&bars->ssum_free, 0, abort)) break;
+        for (int ch = t; ch < kRows * kChunks; ch += 31) {
+          const int n = ch / kChunks, kc = ch % kChunks;
+          const float4 a0 = *reinterpret_cast<const float4*>(sf + n * D + kc * 8);
+          const float4 a1 = *reinterpret_cast<const float4*>(sf + n * D + kc * 8 + 4);
+          const float4 b0 = *reinterpret_cast<const float4*>(sr + n * D + kc * 8);
+          const float4 b1 = *reinterpret_cast<const float4*>(sr + n * D + kc * 8 + 4);
+          float x[8] = {a0.x + b0.x, a0.y + b0.y, a0.z + b0.z, a0.w + b0.w,
+                        a1.x + b1.x, a1.y + b1.y, a1.z + b1.z, a1.w + b1.w};
+          if (part == 1) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] -= __bfloat162float(__float2bfloat16_rn(x[e]));
+          }
+          const uint4 v = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]),
+                                     pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
+          const int half = kc / 8, c16 = kc % 8;
+          *reinterpret_cast<uint4*>(sSsum + half * C::kHalfBytes + n * 128 + ((c16 ^ (n & 7)) * 16)) = v;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive(&bars->ssum_ready);
+      }
+    }
     if (lane == 0 && !*abort) {
       // ------------------------------------------------------- TMA producer
       mbar_expect_tx(&bars->q_full, 2 * C::kTileBytes);
@@ -315,37 +344,6 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       // every MMA issued must finish before TMEM is freed
       if (!ok) mbar_wait(&bars->o_full, 0, abort, false);
     }
-  } else if (warp >= 10) {
-    // ---------------------------------------------- S_sum staging (fused)
-    if (has_lin && !*abort) {
-      const int t = threadIdx.x - 320;
-      const int J = l.J();
-      const float* sf = hy.states + ((((long long)b * l.H + h) * 2 + 0) * J + G.chunk) * D * D;
-      const float* sr = hy.states + ((((long long)b * l.H + h) * 2 + 1) * J + G.chunk) * D * D;
-      constexpr int kChunks = D / 8;  // 16-byte chunks per row
-      for (int part = 0; part < 2; ++part) {
-        if (part == 1 && !mbar_wait(&bars->ssum_free, 0, abort)) break;
-        for (int ch = t; ch < kRows * kChunks; ch += 64) {
-          const int n = ch / kChunks, kc = ch % kChunks;
-          const float4 a0 = *reinterpret_cast<const float4*>(sf + n * D + kc * 8);
-          const float4 a1 = *reinterpret_cast<const float4*>(sf + n * D + kc * 8 + 4);
-          const float4 b0 = *reinterpret_cast<const float4*>(sr + n * D + kc * 8);
-          const float4 b1 = *reinterpret_cast<const float4*>(sr + n * D + kc * 8 + 4);
-          float x[8] = {a0.x + b0.x, a0.y + b0.y, a0.z + b0.z, a0.w + b0.w,
-                        a1.x + b1.x, a1.y + b1.y, a1.z + b1.z, a1.w + b1.w};
-          if (part == 1) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] -= __bfloat162float(__float2bfloat16_rn(x[e]));
-          }
-          const uint4 v = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]),
-                                     pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
-          const int half = kc / 8, c16 = kc % 8;
-          *reinterpret_cast<uint4*>(sSsum + half * C::kHalfBytes + n * 128 + ((c16 ^ (n & 7)) * 16)) = v;
-        }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_arrive(&bars->ssum_ready);
-      }
-    }
   } else {
     // ----------------------------------------------------------- softmax
     const int w = warp / 4;
@@ -356,6 +354,21 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const float sl2 = 1.4426950408889634f / sqrtf((float)D);  // log2(e) / sqrt(d)
     float m = -INFINITY, lsum = 0.f;
     bool ok = !*abort;
+    // The only partially valid key tiles are the last tile of each segment
+    // (3 video segments at most, then the text): (tile index << 8) | valid
+    // count for each (valid <= 128 fits in 8 bits; -1 when a segment is empty).
+    int edge[4];
+    {
+      int first = 0;
+#pragma unroll
+      for (int sgi = 0; sgi < 4; ++sgi) {
+        const int len = (sgi < 3) ? ((sgi < G.nseg) ? G.segn[sgi] : 0) : l.T;
+        const int n = (len + kRows - 1) / kRows;
+        edge[sgi] = (n > 0) ? (((first + n - 1) << 8) | (len - (n - 1) * kRows)) : -1;
+        first += n;
+      }
+    }
+    const int q_end = G.q0 + G.nq;
     for (int t = 0; t < n_tiles && ok; ++t) {
       // the TMEM loads below are warp-collective: leave only as a whole warp
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[w], t & 1, abort))) {
@@ -366,7 +379,10 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       uint32_t sr[128];
       tmem_ld_x128_split(tS, sr);
       float* s = reinterpret_cast<float*>(sr);
-      const int valid = key_tile(G, l.T, t, kRows).valid;
+      int valid = kRows;
+#pragma unroll
+      for (int sgi = 0; sgi < 4; ++sgi)
+        if (edge[sgi] >= 0 && (edge[sgi] >> 8) == t) valid = edge[sgi] & 255;
       if (valid < kRows) {
 #pragma unroll
         for (int j = 0; j < kRows; ++j)
@@ -404,20 +420,20 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const float nm = -m;
       const unsigned long long sl2x2 = f2pack(sl2, sl2), nmx2 = f2pack(nm, nm);
       unsigned long long sum2[2] = {0ull, 0ull};
-      // P goes to TMEM in four 16-column pieces as it is produced
+      // P goes to TMEM in eight 8-column pieces as it is produced
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        uint32_t p[16];
+      for (int c4 = 0; c4 < 8; ++c4) {
+        uint32_t p[8];
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-          const int j = 16 * c4 + jj;
+        for (int jj = 0; jj < 8; ++jj) {
+          const int j = 8 * c4 + jj;
           float xa, xc;
           f2unpack(f2fma(f2pack(s[2 * j], s[2 * j + 1]), sl2x2, nmx2), xa, xc);
           const float a = ex2(xa), c = ex2(xc);
           sum2[jj & 1] = f2add(sum2[jj & 1], f2pack(a, c));
           p[jj] = pack_bf16(a, c);
         }
-        tmem_st_x16_nowait(tS + 16 * c4, p);
+        tmem_st_x8_nowait(tS + 8 * c4, p);
       }
       {
         float s0, s1, s2, s3;
@@ -433,7 +449,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (ok) {
       tc_fence_after();
       const int grow = r0 + kRows * w + row;
-      const bool store = grow < G.q0 + G.nq;
+      const bool store = grow < q_end;
       const float inv = 1.f / lsum;
       const long long base = (((long long)b * l.L() + grow) * l.H + h) * D;
       if constexpr (!kFuse) {
