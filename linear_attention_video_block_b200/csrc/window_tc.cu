@@ -75,7 +75,7 @@ struct Bars {
   unsigned long long kv_full[8];
   unsigned long long kv_empty[8];
   unsigned long long s_full[2];
-  unsigned long long p_full[2];
+  unsigned long long p_full[2][2];   // [Q tile][key half]: P of keys 0..63 / 64..127
   unsigned long long o_full;
   unsigned long long ssum_ready;
   unsigned long long ssum_free;
@@ -166,7 +166,8 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(&bars->s_full[w], 1);
-      mbar_init(&bars->p_full[w], 128);
+      mbar_init(&bars->p_full[w][0], 128);
+      mbar_init(&bars->p_full[w][1], 128);
     }
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->ssum_ready, 31);
@@ -278,15 +279,27 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                  desc_k_sw128(kv_addr + slot * C::kTileBytes + off), idesc_s, ks > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int w, int slot, bool acc) {
+      // O_w += P_w V for one half of the key tile (keys 64 half .. 64 half + 63)
+      auto issue_pv_half = [&](int w, int slot, bool acc, int half) {
         const uint32_t d_tmem = tmem + 256 + D * w;
         const uint32_t a_tmem = tmem + 128 * w;
 #pragma unroll
-        for (int ks = 0; ks < kRows / 16; ++ks) {
+        for (int kk = 0; kk < kRows / 32; ++kk) {
+          const int ks = 4 * half + kk;
           mma_ts(d_tmem, a_tmem + ks * 8,
                  desc_mn_sw128(kv_addr + slot * C::kTileBytes + ks * 16 * 128, C::kHalfBytes),
                  idesc_o, (acc || ks > 0) ? 1u : 0u);
         }
+      };
+      // P_w(t) is published in two halves; the first half's P.V runs while the
+      // softmax computes the second
+      auto issue_pv = [&](int w, int slot, bool acc, int t) -> bool {
+        for (int half = 0; half < 2; ++half) {
+          if (!mbar_wait(&bars->p_full[w][half], t & 1, abort)) return false;
+          tc_fence_after();
+          issue_pv_half(w, slot, acc, half);
+        }
+        return true;
       };
       int ks_cur = 0;
       if (ok) ok = take_slot(ks_cur);
@@ -300,18 +313,14 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       for (int t = 0; t < n_tiles && ok; ++t) {
         int vs = 0, ks_next = 0;
         if (!take_slot(vs)) { ok = false; break; }
-        if (!mbar_wait(&bars->p_full[0], t & 1, abort)) { ok = false; break; }
-        tc_fence_after();
-        issue_pv(0, vs, t > 0);
+        if (!issue_pv(0, vs, t > 0, t)) { ok = false; break; }
         const bool more = t + 1 < n_tiles;
         if (more) {
           if (!take_slot(ks_next)) { ok = false; break; }
           issue_s(0, ks_next);
           tc_commit(&bars->s_full[0]);
         }
-        if (!mbar_wait(&bars->p_full[1], t & 1, abort)) { ok = false; break; }
-        tc_fence_after();
-        issue_pv(1, vs, t > 0);
+        if (!issue_pv(1, vs, t > 0, t)) { ok = false; break; }
         tc_commit(&bars->kv_empty[vs]);
         if (more) {
           issue_s(1, ks_next);
@@ -420,20 +429,28 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const float nm = -m;
       const unsigned long long sl2x2 = f2pack(sl2, sl2), nmx2 = f2pack(nm, nm);
       unsigned long long sum2[2] = {0ull, 0ull};
-      // P goes to TMEM in eight 8-column pieces as it is produced
+      // P goes to TMEM in 8-column pieces as it is produced; each half of the
+      // key tile (P columns 0..31 = keys 0..63, 32..63 = keys 64..127) is
+      // published as soon as it is complete
 #pragma unroll
-      for (int c4 = 0; c4 < 8; ++c4) {
-        uint32_t p[8];
+      for (int half = 0; half < 2; ++half) {
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-          const int j = 8 * c4 + jj;
-          float xa, xc;
-          f2unpack(f2fma(f2pack(s[2 * j], s[2 * j + 1]), sl2x2, nmx2), xa, xc);
-          const float a = ex2(xa), c = ex2(xc);
-          sum2[jj & 1] = f2add(sum2[jj & 1], f2pack(a, c));
-          p[jj] = pack_bf16(a, c);
+        for (int c4 = 0; c4 < 4; ++c4) {
+          uint32_t p[8];
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {
+            const int j = 32 * half + 8 * c4 + jj;
+            float xa, xc;
+            f2unpack(f2fma(f2pack(s[2 * j], s[2 * j + 1]), sl2x2, nmx2), xa, xc);
+            const float a = ex2(xa), c = ex2(xc);
+            sum2[jj & 1] = f2add(sum2[jj & 1], f2pack(a, c));
+            p[jj] = pack_bf16(a, c);
+          }
+          tmem_st_x8_nowait(tS + 32 * half + 8 * c4, p);
         }
-        tmem_st_x8_nowait(tS + 8 * c4, p);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bars->p_full[w][half]);
       }
       {
         float s0, s1, s2, s3;
@@ -441,9 +458,6 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         f2unpack(sum2[1], s2, s3);
         lsum += (s0 + s1) + (s2 + s3);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&bars->p_full[w]);
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_full, 0, abort));
     if (ok) {
