@@ -75,7 +75,7 @@ struct Bars {
   unsigned long long kv_full[8];
   unsigned long long kv_empty[8];
   unsigned long long s_full[2];
-  unsigned long long p_full[2][4];   // [Q tile][key quarter]: P of keys 32q .. 32q + 31
+  unsigned long long p_full[2][2];   // [Q tile][key half]: P of keys 0..63 / 64..127
   unsigned long long o_full;
   unsigned long long ssum_ready;
   unsigned long long ssum_free;
@@ -166,7 +166,8 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(&bars->s_full[w], 1);
-      for (int qq = 0; qq < 4; ++qq) mbar_init(&bars->p_full[w][qq], 128);
+      mbar_init(&bars->p_full[w][0], 128);
+      mbar_init(&bars->p_full[w][1], 128);
     }
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->ssum_ready, 31);
@@ -278,25 +279,25 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                  desc_k_sw128(kv_addr + slot * C::kTileBytes + off), idesc_s, ks > 0 ? 1u : 0u);
         }
       };
-      // O_w += P_w V for one quarter of the key tile (keys 32 qq .. 32 qq + 31)
-      auto issue_pv_part = [&](int w, int slot, bool acc, int qq) {
+      // O_w += P_w V for one half of the key tile (keys 64 half .. 64 half + 63)
+      auto issue_pv_half = [&](int w, int slot, bool acc, int half) {
         const uint32_t d_tmem = tmem + 256 + D * w;
         const uint32_t a_tmem = tmem + 128 * w;
 #pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-          const int ks = 2 * qq + kk;
+        for (int kk = 0; kk < kRows / 32; ++kk) {
+          const int ks = 4 * half + kk;
           mma_ts(d_tmem, a_tmem + ks * 8,
                  desc_mn_sw128(kv_addr + slot * C::kTileBytes + ks * 16 * 128, C::kHalfBytes),
                  idesc_o, (acc || ks > 0) ? 1u : 0u);
         }
       };
-      // P_w(t) is published in four parts; each part's P.V runs while the
-      // softmax computes the next
+      // P_w(t) is published in two halves; the first half's P.V runs while the
+      // softmax computes the second
       auto issue_pv = [&](int w, int slot, bool acc, int t) -> bool {
-        for (int qq = 0; qq < 4; ++qq) {
-          if (!mbar_wait(&bars->p_full[w][qq], t & 1, abort)) return false;
+        for (int half = 0; half < 2; ++half) {
+          if (!mbar_wait(&bars->p_full[w][half], t & 1, abort)) return false;
           tc_fence_after();
-          issue_pv_part(w, slot, acc, qq);
+          issue_pv_half(w, slot, acc, half);
         }
         return true;
       };
@@ -428,28 +429,28 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const float nm = -m;
       const unsigned long long sl2x2 = f2pack(sl2, sl2), nmx2 = f2pack(nm, nm);
       unsigned long long sum2[2] = {0ull, 0ull};
-      // P goes to TMEM in 8-column pieces as it is produced; each quarter of
-      // the key tile (P columns 16 qq .. 16 qq + 15 = keys 32 qq .. 32 qq + 31)
-      // is published as soon as it is complete
+      // P goes to TMEM in 8-column pieces as it is produced; each half of the
+      // key tile (P columns 0..31 = keys 0..63, 32..63 = keys 64..127) is
+      // published as soon as it is complete
 #pragma unroll
-      for (int qq = 0; qq < 4; ++qq) {
+      for (int half = 0; half < 2; ++half) {
 #pragma unroll
-        for (int c4 = 0; c4 < 2; ++c4) {
+        for (int c4 = 0; c4 < 4; ++c4) {
           uint32_t p[8];
 #pragma unroll
           for (int jj = 0; jj < 8; ++jj) {
-            const int j = 16 * qq + 8 * c4 + jj;
+            const int j = 32 * half + 8 * c4 + jj;
             float xa, xc;
             f2unpack(f2fma(f2pack(s[2 * j], s[2 * j + 1]), sl2x2, nmx2), xa, xc);
             const float a = ex2(xa), c = ex2(xc);
             sum2[jj & 1] = f2add(sum2[jj & 1], f2pack(a, c));
             p[jj] = pack_bf16(a, c);
           }
-          tmem_st_x8_nowait(tS + 16 * qq + 8 * c4, p);
+          tmem_st_x8_nowait(tS + 32 * half + 8 * c4, p);
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&bars->p_full[w][qq]);
+        mbar_arrive(&bars->p_full[w][half]);
       }
       {
         float s0, s1, s2, s3;
