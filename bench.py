@@ -68,10 +68,12 @@ def window_flops(lay) -> float:
     return 4.0 * lay.d * window_pairs(lay) * lay.H * lay.B
 
 
-def launches_per_step(lay) -> int:
-    """Kernels of one vdn_hybrid_attn_fwd call: window softmax, gram, inverse,
-    scan, zero-fill of unused chunk entries, readout/combine."""
-    return 6
+def launches_per_step(lay, dtype) -> int:
+    """Kernels of one vdn_hybrid_attn_fwd call: gram, inverse, scan, zero-fill of
+    unused chunk entries, and the window softmax with the readout, norm and
+    gates fused (bf16, d in {64, 128}); the CUDA-core path adds a separate
+    readout/combine kernel."""
+    return 5 if (dtype == "bf16" and lay.d in (64, 128)) else 6
 
 
 # ----------------------------------------------------------------- clocks
@@ -372,7 +374,7 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps},
         "clocks": clk,
-        "gpu_launches": launches_per_step(lay) * args.steps * world,
+        "gpu_launches": launches_per_step(lay, dtype) * args.steps * world,
         "when": datetime.datetime.now(datetime.timezone.utc).isoformat(timespec="seconds"),
     }
     print(json.dumps(line), flush=True)
