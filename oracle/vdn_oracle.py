@@ -26,7 +26,11 @@ B = V^T Diag(beta) K, state S of shape (d_v, d_k) so that S k ~ v.
 Readings of points the pages leave open (the CUDA path uses the same ones):
   R1  Joint objective: min_S 1/2 sum_u beta_u ||S k_u - v_u||^2 + 1/2 ||S - S_bar||_F^2,
       whose stationarity condition S (I + A) = S_bar + B is the printed closed form.
-  R2  No decay: S_bar = previous state (the KDA decay alpha is not used).
+  R2  No decay by default: S_bar = previous state. With a decay (the KDA gate,
+      VDN "Video Delta Attention": S_bar = S_{t-1} Diag(alpha)), alpha_f in
+      [0, 1]^{d_k} is given per frame, head and key channel and scales the
+      columns (key dimension) of the state before frame f is written, in both
+      scans; the text init has no decay.
   R3  Chunks: ch(f) = floor(f / c); the last chunk is partial when c does not
       divide F. Window of a non-boundary frame: chunks ch(f)-1 .. ch(f)+1 that
       exist. Boundary frames 0 and F-1 see every frame.
@@ -239,22 +243,30 @@ def text_init(K_T, V_T, beta_T, d_v, d_k):
     return 0.5 * frame_update(np.zeros((d_v, d_k)), K_T, V_T, beta_T)
 
 
-def scan_states(Kf, Vf, betaf, S0, F):
+def decayed(S, alpha_f):
+    """S_bar = S Diag(alpha_f): the KDA channel-wise decay of the inherited state
+    (VDN "Video Delta Attention"), alpha_f over the key channels (columns)."""
+    return S if alpha_f is None else S * alpha_f[None, :]
+
+
+def scan_states(Kf, Vf, betaf, S0, F, alphaf=None):
     """Forward and reverse VDA recurrences over frames 1 .. F-2 (R6).
 
-    Kf, Vf: [F, N, d] per-frame keys/values of one (b, h); betaf: [F, N].
+    Kf, Vf: [F, N, d] per-frame keys/values of one (b, h); betaf: [F, N];
+    alphaf: optional [F, d_k] decay per frame (R2).
     Returns (fwd, rev): fwd[s] = state after frames 1..s (fwd[0] = S0, s <= F-2);
     rev[s] = state after frames F-2 down to s (rev[F-1] = S0, s >= 1).
     """
+    a = (lambda f: None) if alphaf is None else (lambda f: alphaf[f])
     fwd = {0: S0}
     S = S0
     for f in range(1, F - 1):
-        S = frame_update(S, Kf[f], Vf[f], betaf[f])
+        S = frame_update(decayed(S, a(f)), Kf[f], Vf[f], betaf[f])
         fwd[f] = S
     rev = {F - 1: S0}
     S = S0
     for f in range(F - 2, 0, -1):
-        S = frame_update(S, Kf[f], Vf[f], betaf[f])
+        S = frame_update(decayed(S, a(f)), Kf[f], Vf[f], betaf[f])
         rev[f] = S
     return fwd, rev
 
@@ -269,13 +281,13 @@ def read_states(f, F, c, fwd, rev, S0):
 
 
 def linear_branch(q, k, v, k_text, v_text, beta, beta_text, F, N, c, heads=None,
-                  return_states=False):
+                  return_states=False, alpha=None):
     """VDA branch readout o_lin [B, L, H, d], ungated and before RMSNorm.
 
     Computed per frame (not per chunk): every non-boundary query frame reads
     its own (S_fwd + S_rev) and o_lin = (S_fwd + S_rev) q (R8); boundary frames
     read nothing (R7). With return_states, also returns per (b, h) the dicts
-    (S0, fwd, rev).
+    (S0, fwd, rev). alpha: optional decay [B, F, H, d] (R2).
     """
     Bn, L, H, d = q.shape
     heads = range(H) if heads is None else heads
@@ -288,7 +300,8 @@ def linear_branch(q, k, v, k_text, v_text, beta, beta_text, F, N, c, heads=None,
             bf = beta[b, :, h].reshape(F, N)
             S0 = text_init(k_text[b, :, h, :], v_text[b, :, h, :],
                            beta_text[b, :, h], d, d)
-            fwd, rev = scan_states(Kf, Vf, bf, S0, F)
+            af = None if alpha is None else alpha[b, :, h, :]
+            fwd, rev = scan_states(Kf, Vf, bf, S0, F, af)
             states[(b, h)] = (S0, fwd, rev)
             for f in range(F):
                 sl = slice(f * N, (f + 1) * N)
@@ -324,14 +337,15 @@ def combine(o_soft, o_lin, g_s, g_l, eps=RMS_EPS, weight=None):
 
 
 def hybrid(q, k, v, k_text, v_text, beta, beta_text, g_s, g_l, F, N, c,
-           rows=None, heads=None, eps=RMS_EPS, weight=None):
+           rows=None, heads=None, eps=RMS_EPS, weight=None, alpha=None):
     """The whole hybrid video-video attention forward for the given rows/heads.
 
     Returns dict with out, out_soft (gated), out_lin (gated), o_soft, o_lin.
     Elements outside the requested rows/heads are NaN.
     """
     o_soft = softmax_branch(q, k, v, k_text, v_text, F, N, c, rows=rows, heads=heads)
-    o_lin = linear_branch(q, k, v, k_text, v_text, beta, beta_text, F, N, c, heads=heads)
+    o_lin = linear_branch(q, k, v, k_text, v_text, beta, beta_text, F, N, c, heads=heads,
+                          alpha=alpha)
     out, gs, gl = combine(o_soft, o_lin, g_s, g_l, eps, weight)
     return {"out": out, "out_soft": gs, "out_lin": gl, "o_soft": o_soft, "o_lin": o_lin}
 

@@ -486,3 +486,62 @@ def test_no_text_tokens():
     assert np.isfinite(r["out"]).all()
     _, st = O.linear_branch(q, k, v, kt, vt, beta, bt, F, N, c, return_states=True)
     assert np.all(st[(0, 0)][0] == 0)
+
+
+# ------------------------------------------------ KDA channel decay (option)
+
+def test_decay_without_writes_is_a_product_of_diagonals():
+    """With every write strength zero (A = B = 0) the update reduces to the decay
+    alone: the forward state after frames 1..f is S0 Diag(prod_{g<=f} alpha_g),
+    the reverse one after F-2..f is S0 Diag(prod_{g>=f} alpha_g) (the decay acts on
+    the key channels, the columns of S)."""
+    rng = np.random.default_rng(30)
+    B, F, N, T, H, d, c = 1, 9, 3, 4, 1, 5, 2
+    q, k, v, kt, vt, beta, bt, *_ = _rand_inputs(rng, B, F, N, T, H, d)
+    beta[:] = 0.0
+    alpha = rng.uniform(0.3, 1.0, (B, F, H, d))
+    _, st = O.linear_branch(q, k, v, kt, vt, beta, bt, F, N, c, return_states=True, alpha=alpha)
+    S0, fwd, rev = st[(0, 0)]
+    for f in range(1, F - 1):
+        np.testing.assert_allclose(fwd[f], S0 * np.prod(alpha[0, 1:f + 1, 0], axis=0)[None, :], atol=1e-13)
+        np.testing.assert_allclose(rev[f], S0 * np.prod(alpha[0, f:F - 1, 0], axis=0)[None, :], atol=1e-13)
+
+
+def test_decay_one_token_frames_match_the_decayed_delta_step():
+    """One-token frames with decay: S <- S_bar + beta (v - S_bar k) k^T / (1 + beta |k|^2)
+    with S_bar = S Diag(alpha_f), frame by frame (Sherman-Morrison again)."""
+    rng = np.random.default_rng(31)
+    B, F, N, T, H, d, c = 1, 8, 1, 2, 1, 6, 2
+    q, k, v, kt, vt, beta, bt, *_ = _rand_inputs(rng, B, F, N, T, H, d)
+    alpha = rng.uniform(0.5, 1.0, (B, F, H, d))
+    _, st = O.linear_branch(q, k, v, kt, vt, beta, bt, F, N, c, return_states=True, alpha=alpha)
+    S0, fwd, _ = st[(0, 0)]
+    S = S0.copy()
+    for f in range(1, F - 1):
+        Sb = S @ np.diag(alpha[0, f, 0])
+        kk, vv, bb = k[0, f, 0], v[0, f, 0], beta[0, f, 0]
+        S = Sb + bb * np.outer(vv - Sb @ kk, kk) / (1 + bb * kk @ kk)
+        np.testing.assert_allclose(fwd[f], S, rtol=1e-11, atol=1e-12)
+
+
+def test_decay_keeps_the_transition_non_expansive():
+    """Project page, 'Stability of the Inherited State': with 0 <= alpha <= 1 the
+    inherited component passes through Diag(alpha)(I + A)^-1, of norm <= 1."""
+    rng = np.random.default_rng(32)
+    d, U = 7, 40
+    K = _unit_rows(rng, U, d)
+    beta = rng.uniform(0, 1, U)
+    for _ in range(5):
+        alpha = rng.uniform(0, 1, d)
+        Sb = rng.standard_normal((d, d))
+        out = O.frame_update(O.decayed(Sb, alpha), K, np.zeros((U, d)), beta)
+        assert np.linalg.norm(out, 2) <= np.linalg.norm(Sb, 2) + 1e-12
+
+
+def test_unit_decay_is_no_decay():
+    rng = np.random.default_rng(33)
+    B, F, N, T, H, d, c = 1, 10, 2, 3, 2, 4, 3
+    q, k, v, kt, vt, beta, bt, gs, gl = _rand_inputs(rng, B, F, N, T, H, d)
+    a = O.hybrid(q, k, v, kt, vt, beta, bt, gs, gl, F, N, c)["out"]
+    b = O.hybrid(q, k, v, kt, vt, beta, bt, gs, gl, F, N, c, alpha=np.ones((B, F, H, d)))["out"]
+    np.testing.assert_array_equal(a, b)
