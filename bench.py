@@ -1,7 +1,8 @@
 """Benchmark of the VDN hybrid video-video attention forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload 768p-bf16] [--entry hybrid|window|vda]
+                    [--workload 768p-bf16]
+                    [--entry hybrid|window|vda|vda-decay|hybrid-decay]
 
 A step is one vdn_hybrid_attn_fwd call (window softmax + VDA scans + readout,
 norm, gates) over one 768p-like layer input (B=1, H=40, d=128, F=36 frames of
@@ -16,7 +17,8 @@ reported time is the maximum over ranks.
 --entry selects the public entry point that forms the step: the hybrid
 forward (default, the headline), or the softmax branch or the linear branch
 alone (vdn_window_softmax_fwd / vdn_vda_scan_fwd), for per-branch numbers and
-for profiling one kernel family at a time.
+for profiling one kernel family at a time, or the KDA-decayed forms
+(vdn_vda_scan_fwd_decay / vdn_hybrid_attn_fwd_decay, alpha in (0.8, 1]).
 
 Printed on rank 0: one JSON line with the throughput (video tokens/s over all
 ranks), the roofline of the dominant kernel (window softmax, tensor-core bound),
@@ -419,26 +421,41 @@ def vda_bytes(lay) -> float:
     return float(per_bh * H * B)
 
 
+def decay_bytes(lay) -> float:
+    """Extra algorithmic bytes of the decayed scans: alpha [B, F, H, d] fp32 of
+    the non-boundary frames, read once."""
+    return float(lay.B * max(lay.F - 2, 0) * lay.H * lay.d * 4)
+
+
 def run_entry(args, rank, world, local_rank):
-    """One branch entry point as the step (no e2e / CPU baseline legs)."""
+    """One entry point as the step (no e2e / CPU baseline legs): a branch alone,
+    or the _decay forms of the linear branch and the hybrid forward."""
     import torch
     from linear_attention_video_block_b200 import vdn
-    from linear_attention_video_block_b200.synth import WORKLOADS, make_inputs
+    from linear_attention_video_block_b200.synth import WORKLOADS, make_decay, make_inputs
 
     lay, dtype, seed = WORKLOADS[args.workload]
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     inp = make_inputs(lay, dtype, rank_seed(seed, rank), device=str(dev))
+    alpha = make_decay(lay, rank_seed(seed, rank) + 1, device=str(dev))
     out = torch.empty_like(inp["q"])
     ws = torch.empty(vdn.workspace_bytes(lay, inp["q"].dtype), dtype=torch.uint8, device=dev)
     if args.entry == "window":
         def step():
             vdn.window_softmax_fwd(lay, inp["q"], inp["k"], inp["v"], inp["k_text"], inp["v_text"],
                                    o_soft=out)
+    elif args.entry == "hybrid-decay":
+        def step():
+            vdn.hybrid_attn_fwd(lay, inp["q"], inp["k"], inp["v"], inp["k_text"], inp["v_text"],
+                                inp["beta"], inp["beta_text"], inp["g_s"], inp["g_l"], out=out,
+                                workspace=ws, alpha=alpha)
     else:
+        a = alpha if args.entry == "vda-decay" else None
+
         def step():
             vdn.vda_scan_fwd(lay, inp["q"], inp["k"], inp["v"], inp["k_text"], inp["v_text"],
-                             inp["beta"], inp["beta_text"], o_lin=out, workspace=ws)
+                             inp["beta"], inp["beta_text"], o_lin=out, workspace=ws, alpha=a)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
@@ -458,17 +475,22 @@ def run_entry(args, rank, world, local_rank):
     if args.entry == "window":
         work, unit, peak = window_flops(lay) / 1e12, "TFLOP/s", float(peaks["bf16_tflops"])
         bound = "tensor"
+    elif args.entry == "hybrid-decay":
+        work, unit, peak, bound = None, None, None, None
     else:
-        work, unit, peak = vda_bytes(lay) / 1e9, "GB/s", float(peaks["hbm_gbs"])
+        extra = decay_bytes(lay) if args.entry == "vda-decay" else 0.0
+        work, unit, peak = (vda_bytes(lay) + extra) / 1e9, "GB/s", float(peaks["hbm_gbs"])
         bound = "hbm"
-    ach = work / (ms * 1e-3)
+    roof = None
+    if work is not None:
+        ach = work / (ms * 1e-3)
+        roof = {"bound": bound, "achieved": ach, "peak": peak, "unit": unit,
+                "frac": ach / peak, "peak_source": kind}
     print(json.dumps({
         "impl": "ours", "entry": args.entry, "metric": f"{args.entry} fwd video tokens/s",
         "value": lay.L * lay.B / (ms * 1e-3), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "dtype": dtype,
-        "config": config_of(args.workload, lay),
-        "roofline": {"bound": bound, "achieved": ach, "peak": peak, "unit": unit,
-                     "frac": ach / peak, "peak_source": kind},
+        "config": config_of(args.workload, lay), "roofline": roof,
     }), flush=True)
 
 
@@ -479,7 +501,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="768p-bf16")
-    ap.add_argument("--entry", choices=["hybrid", "window", "vda"], default="hybrid")
+    ap.add_argument("--entry", choices=["hybrid", "window", "vda", "vda-decay", "hybrid-decay"],
+                    default="hybrid")
     ap.add_argument("--ref-rows", type=int, default=96,
                     help="query rows per frame in the oracle's bounded sample")
     args = ap.parse_args()

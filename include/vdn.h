@@ -88,8 +88,9 @@ typedef enum {
   VDN_ERR_TIMEOUT = 5
 } vdn_status_t;
 
-/* Bytes of device workspace that vdn_vda_scan_fwd and vdn_hybrid_attn_fwd need
- * for this layout and dtype (the maximum of the two). 0 for an invalid layout. */
+/* Bytes of device workspace that vdn_vda_scan_fwd and vdn_hybrid_attn_fwd (and
+ * their _decay forms) need for this layout and dtype (the maximum of the two).
+ * 0 for an invalid layout. */
 size_t vdn_workspace_bytes(const vdn_layout_t* layout, int dtype);
 
 /* Softmax branch alone (project page, "Local Softmax and Long-Range Linear
@@ -126,6 +127,35 @@ int vdn_hybrid_attn_fwd(const vdn_layout_t* layout, int dtype,
                         const float* rms_weight, float rms_eps,
                         void* out, void* out_soft, void* out_lin,
                         void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Linear branch with KDA channel decay (project page "Video DeltaNet", section
+ * "Video Delta Attention: A Frame-Wise Solution": the inherited state is decayed
+ * per key channel before a frame is written, S_bar = S Diag(alpha)). Same as
+ * vdn_vda_scan_fwd except that every scan step over video frame f computes
+ * S <- (S Diag(alpha_f) + B_f)(I + A_f)^-1; the text write that makes S0 is not
+ * decayed. alpha: [B, F, H, d] float32, required (VDN_ERR_INVALID if NULL),
+ * 16-byte aligned, indexed by the key dim (columns of S); values are used as
+ * given (the pages take them in (0, 1]; 1 everywhere gives vdn_vda_scan_fwd's
+ * result). Entries of the boundary frames 0 and F-1 are never read. */
+int vdn_vda_scan_fwd_decay(const vdn_layout_t* layout, int dtype,
+                           const void* q, const void* k, const void* v,
+                           const void* k_text, const void* v_text,
+                           const float* beta, const float* beta_text,
+                           const float* alpha,
+                           void* o_lin, float* chunk_states,
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* The whole hybrid forward with the KDA-decayed linear branch of
+ * vdn_vda_scan_fwd_decay (alpha as there); everything else as vdn_hybrid_attn_fwd. */
+int vdn_hybrid_attn_fwd_decay(const vdn_layout_t* layout, int dtype,
+                              const void* q, const void* k, const void* v,
+                              const void* k_text, const void* v_text,
+                              const float* beta, const float* beta_text,
+                              const float* alpha,
+                              const void* g_soft, const void* g_lin,
+                              const float* rms_weight, float rms_eps,
+                              void* out, void* out_soft, void* out_lin,
+                              void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* Size of the device scratch array behind vdn_vda_scan_fwd_noalloc: 64 MiB. */
 #define VDN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)

@@ -8,7 +8,7 @@
 //            tensor-core kernel in gram_tc.cu; fp32 inputs: CUDA-core kernel here).
 //   inverse  M_f = (I + A_f)^-1 in place of A_f (register-blocked Gauss-Jordan;
 //            I + A_f is SPD with every pivot >= 1, so no pivoting is needed).
-//   scan     S <- (S + B_f) M_f, forward over 1..fwd_max and reverse over
+//   scan     S <- (S Diag(alpha_f) + B_f) M_f (alpha: optional KDA decay), forward over 1..fwd_max and reverse over
 //            F-2..rev_min, from S0 = 1/2 B_T M_T. Rows of S evolve independently
 //            (the update multiplies on the right), so each CTA owns 16 rows of
 //            one (b, h, direction) state and the chain needs no cross-CTA sync;
@@ -217,7 +217,7 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 template <int D>
 __global__ void __launch_bounds__(128)
 scan_kernel(Layout l, int fwd_max, int rev_min, int has_text, const float* __restrict__ am,
-            const float* __restrict__ bw, float* __restrict__ states) {
+            const float* __restrict__ bw, const float* __restrict__ alpha, float* __restrict__ states) {
   using C = ScanCfg<D>;
   constexpr int R = C::kR, RR = C::kRR, CH = C::kChunk, NCH = D / CH;
   __shared__ __align__(16) float ring[C::kRing][CH * D];
@@ -272,13 +272,19 @@ scan_kernel(Layout l, int fwd_max, int rev_min, int has_text, const float* __res
   for (int t = 0; t < nsteps; ++t) {
     const bool text = has_text && t == 0;
     const int f = frame_of(t);
-    // X = S + B_f rows (text step: X = 1/2 B_T rows); B rows read straight from global
+    // X = S Diag(alpha_f) + B_f rows (text step: X = 1/2 B_T rows); B rows read
+    // straight from global; alpha_f (KDA channel decay, optional) over columns
+    float4 av = make_float4(1.f, 1.f, 1.f, 1.f);
+    if (alpha != nullptr && !text)
+      av = *reinterpret_cast<const float4*>(
+          alpha + (((long long)(bh / l.H) * l.F + f) * l.H + bh % l.H) * D + 4 * cg);
 #pragma unroll
     for (int r = 0; r < RR; ++r) {
       const float4 bv = *reinterpret_cast<const float4*>(bw_bh + (long long)f * D * D +
                                                          (long long)(row0 + RR * rg + r) * D + 4 * cg);
       const float4 xv = text ? make_float4(0.5f * bv.x, 0.5f * bv.y, 0.5f * bv.z, 0.5f * bv.w)
-                             : make_float4(s[r][0] + bv.x, s[r][1] + bv.y, s[r][2] + bv.z, s[r][3] + bv.w);
+                             : make_float4(fmaf(s[r][0], av.x, bv.x), fmaf(s[r][1], av.y, bv.y),
+                                           fmaf(s[r][2], av.z, bv.z), fmaf(s[r][3], av.w, bv.w));
       *reinterpret_cast<float4*>(&x[(RR * rg + r) * D + 4 * cg]) = xv;
     }
     float acc[RR][4];
@@ -343,8 +349,9 @@ __global__ void zero_unused_chunks(Layout l, float* __restrict__ states) {
 
 template <typename T, int D>
 cudaError_t launch_states_t(const Layout& l, int dtype, const void* k, const void* v, const void* kt,
-                            const void* vt, const float* beta, const float* beta_t, float* am,
-                            float* bw, float* states, cudaStream_t st) {
+                            const void* vt, const float* beta, const float* beta_t,
+                            const float* alpha, float* am, float* bw, float* states,
+                            cudaStream_t st) {
   int fwd_max, rev_min;
   scan_extent(l, fwd_max, rev_min);
   SlotMap map;
@@ -372,7 +379,7 @@ cudaError_t launch_states_t(const Layout& l, int dtype, const void* k, const voi
   }
   {
     dim3 grid(D / 16, 2, l.B * l.H);
-    scan_kernel<D><<<grid, ScanCfg<D>::kThreads, 0, st>>>(l, fwd_max, rev_min, map.has_text, am, bw, states);
+    scan_kernel<D><<<grid, ScanCfg<D>::kThreads, 0, st>>>(l, fwd_max, rev_min, map.has_text, am, bw, alpha, states);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     zero_unused_chunks<<<dim3(32, l.B * l.H), 256, 0, st>>>(l, states);
@@ -384,19 +391,19 @@ cudaError_t launch_states_t(const Layout& l, int dtype, const void* k, const voi
 
 cudaError_t launch_vda_states(const Layout& l, int dtype, const void* k, const void* v,
                               const void* kt, const void* vt, const float* beta,
-                              const float* beta_text, float* am, float* bw, float* states,
-                              cudaStream_t st) {
+                              const float* beta_text, const float* alpha, float* am, float* bw,
+                              float* states, cudaStream_t st) {
   if (dtype == VDN_F32) {
     switch (l.d) {
-      case 16: return launch_states_t<float, 16>(l, dtype, k, v, kt, vt, beta, beta_text, am, bw, states, st);
-      case 32: return launch_states_t<float, 32>(l, dtype, k, v, kt, vt, beta, beta_text, am, bw, states, st);
-      case 64: return launch_states_t<float, 64>(l, dtype, k, v, kt, vt, beta, beta_text, am, bw, states, st);
-      case 128: return launch_states_t<float, 128>(l, dtype, k, v, kt, vt, beta, beta_text, am, bw, states, st);
+      case 16: return launch_states_t<float, 16>(l, dtype, k, v, kt, vt, beta, beta_text, alpha, am, bw, states, st);
+      case 32: return launch_states_t<float, 32>(l, dtype, k, v, kt, vt, beta, beta_text, alpha, am, bw, states, st);
+      case 64: return launch_states_t<float, 64>(l, dtype, k, v, kt, vt, beta, beta_text, alpha, am, bw, states, st);
+      case 128: return launch_states_t<float, 128>(l, dtype, k, v, kt, vt, beta, beta_text, alpha, am, bw, states, st);
     }
   } else {
     switch (l.d) {
-      case 64: return launch_states_t<__nv_bfloat16, 64>(l, dtype, k, v, kt, vt, beta, beta_text, am, bw, states, st);
-      case 128: return launch_states_t<__nv_bfloat16, 128>(l, dtype, k, v, kt, vt, beta, beta_text, am, bw, states, st);
+      case 64: return launch_states_t<__nv_bfloat16, 64>(l, dtype, k, v, kt, vt, beta, beta_text, alpha, am, bw, states, st);
+      case 128: return launch_states_t<__nv_bfloat16, 128>(l, dtype, k, v, kt, vt, beta, beta_text, alpha, am, bw, states, st);
     }
   }
   return cudaErrorInvalidValue;

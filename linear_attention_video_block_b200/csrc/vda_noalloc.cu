@@ -108,7 +108,7 @@ extern "C" int vdn_vda_scan_fwd_noalloc(const vdn_layout_t* layout, int dtype, c
   const void* kt = layout->T ? k_text : nullptr;
   const void* vt = layout->T ? v_text : nullptr;
   const float* bt = layout->T ? beta_text : nullptr;
-  if (vdn::launch_vda_states(l, dtype, k, v, kt, vt, beta, bt, am, bw, states, stream) != cudaSuccess)
+  if (vdn::launch_vda_states(l, dtype, k, v, kt, vt, beta, bt, nullptr, am, bw, states, stream) != cudaSuccess)
     return VDN_ERR_CUDA;
   cudaError_t e;
   if (vdn::readout_tc_supported(l, dtype))

@@ -100,15 +100,19 @@ int vdn_window_softmax_fwd(const vdn_layout_t* layout, int dtype, const void* q,
                     layout->T ? v_text : nullptr, o_soft, false, lse, stream);
 }
 
-int vdn_vda_scan_fwd(const vdn_layout_t* layout, int dtype, const void* q, const void* k,
-                     const void* v, const void* k_text, const void* v_text, const float* beta,
-                     const float* beta_text, void* o_lin, float* chunk_states, void* workspace,
-                     size_t workspace_bytes, cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+
+int vda_scan_impl(const vdn_layout_t* layout, int dtype, const void* q, const void* k,
+                  const void* v, const void* k_text, const void* v_text, const float* beta,
+                  const float* beta_text, const float* alpha, void* o_lin, float* chunk_states,
+                  void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   if (!layout_ok(layout)) return VDN_ERR_INVALID;
   if (!dtype_d_ok(dtype, layout->d)) return VDN_ERR_UNSUPPORTED;
   if (!q || !k || !v || !beta || !o_lin) return VDN_ERR_INVALID;
   if (layout->T > 0 && (!k_text || !v_text || !beta_text)) return VDN_ERR_INVALID;
-  const void* ptrs[] = {q, k, v, beta, o_lin, chunk_states, workspace};
+  const void* ptrs[] = {q, k, v, beta, alpha, o_lin, chunk_states, workspace};
   for (const void* p : ptrs) if (p && !aligned16(p)) return VDN_ERR_UNSUPPORTED;
   if (layout->T > 0 && (!aligned16(k_text) || !aligned16(v_text) || !aligned16(beta_text)))
     return VDN_ERR_UNSUPPORTED;
@@ -121,7 +125,8 @@ int vdn_vda_scan_fwd(const vdn_layout_t* layout, int dtype, const void* q, const
   const void* kt = layout->T ? k_text : nullptr;
   const void* vt = layout->T ? v_text : nullptr;
   const float* bt = layout->T ? beta_text : nullptr;
-  int s = cuda_status(vdn::launch_vda_states(l, dtype, k, v, kt, vt, beta, bt, w.am, w.bw, states, stream));
+  int s = cuda_status(vdn::launch_vda_states(l, dtype, k, v, kt, vt, beta, bt, alpha, w.am, w.bw,
+                                             states, stream));
   if (s != VDN_OK) return s;
   if (vdn::readout_tc_supported(l, dtype))
     return cuda_status(vdn::launch_readout_tc(l, q, states, o_lin, stream));
@@ -129,18 +134,17 @@ int vdn_vda_scan_fwd(const vdn_layout_t* layout, int dtype, const void* q, const
                                          0.f, o_lin, nullptr, nullptr, stream));
 }
 
-int vdn_hybrid_attn_fwd(const vdn_layout_t* layout, int dtype, const void* q, const void* k,
-                        const void* v, const void* k_text, const void* v_text, const float* beta,
-                        const float* beta_text, const void* g_soft, const void* g_lin,
-                        const float* rms_weight, float rms_eps, void* out, void* out_soft,
-                        void* out_lin, void* workspace, size_t workspace_bytes,
-                        cudaStream_t stream) {
+int hybrid_impl(const vdn_layout_t* layout, int dtype, const void* q, const void* k,
+                const void* v, const void* k_text, const void* v_text, const float* beta,
+                const float* beta_text, const float* alpha, const void* g_soft, const void* g_lin,
+                const float* rms_weight, float rms_eps, void* out, void* out_soft, void* out_lin,
+                void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   if (!layout_ok(layout)) return VDN_ERR_INVALID;
   if (!dtype_d_ok(dtype, layout->d)) return VDN_ERR_UNSUPPORTED;
   if (!q || !k || !v || !beta || !g_soft || !g_lin || !out) return VDN_ERR_INVALID;
   if (layout->T > 0 && (!k_text || !v_text || !beta_text)) return VDN_ERR_INVALID;
   if (!(rms_eps >= 0.f)) return VDN_ERR_INVALID;
-  const void* ptrs[] = {q, k, v, beta, g_soft, g_lin, rms_weight, out, out_soft, out_lin, workspace};
+  const void* ptrs[] = {q, k, v, beta, alpha, g_soft, g_lin, rms_weight, out, out_soft, out_lin, workspace};
   for (const void* p : ptrs) if (p && !aligned16(p)) return VDN_ERR_UNSUPPORTED;
   if (layout->T > 0 && (!aligned16(k_text) || !aligned16(v_text) || !aligned16(beta_text)))
     return VDN_ERR_UNSUPPORTED;
@@ -154,7 +158,8 @@ int vdn_hybrid_attn_fwd(const vdn_layout_t* layout, int dtype, const void* q, co
   const void* kt = layout->T ? k_text : nullptr;
   const void* vt = layout->T ? v_text : nullptr;
   const float* bt = layout->T ? beta_text : nullptr;
-  int s = cuda_status(vdn::launch_vda_states(l, dtype, k, v, kt, vt, beta, bt, w.am, w.bw, w.states, stream));
+  int s = cuda_status(vdn::launch_vda_states(l, dtype, k, v, kt, vt, beta, bt, alpha, w.am, w.bw,
+                                             w.states, stream));
   if (s != VDN_OK) return s;
   if (fused)
     return cuda_status(vdn::launch_hybrid_tc(l, q, k, v, kt, vt, w.states, g_soft, g_lin, rms_weight,
@@ -163,6 +168,49 @@ int vdn_hybrid_attn_fwd(const vdn_layout_t* layout, int dtype, const void* q, co
   if (s != VDN_OK) return s;
   return cuda_status(vdn::launch_readout(l, dtype, 1, q, w.states, w.o_soft, g_soft, g_lin,
                                          rms_weight, rms_eps, out, out_soft, out_lin, stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+int vdn_vda_scan_fwd(const vdn_layout_t* layout, int dtype, const void* q, const void* k,
+                     const void* v, const void* k_text, const void* v_text, const float* beta,
+                     const float* beta_text, void* o_lin, float* chunk_states, void* workspace,
+                     size_t workspace_bytes, cudaStream_t stream) {
+  return vda_scan_impl(layout, dtype, q, k, v, k_text, v_text, beta, beta_text, nullptr, o_lin,
+                       chunk_states, workspace, workspace_bytes, stream);
+}
+
+int vdn_vda_scan_fwd_decay(const vdn_layout_t* layout, int dtype, const void* q, const void* k,
+                           const void* v, const void* k_text, const void* v_text, const float* beta,
+                           const float* beta_text, const float* alpha, void* o_lin,
+                           float* chunk_states, void* workspace, size_t workspace_bytes,
+                           cudaStream_t stream) {
+  if (!alpha) return VDN_ERR_INVALID;
+  return vda_scan_impl(layout, dtype, q, k, v, k_text, v_text, beta, beta_text, alpha, o_lin,
+                       chunk_states, workspace, workspace_bytes, stream);
+}
+
+int vdn_hybrid_attn_fwd(const vdn_layout_t* layout, int dtype, const void* q, const void* k,
+                        const void* v, const void* k_text, const void* v_text, const float* beta,
+                        const float* beta_text, const void* g_soft, const void* g_lin,
+                        const float* rms_weight, float rms_eps, void* out, void* out_soft,
+                        void* out_lin, void* workspace, size_t workspace_bytes,
+                        cudaStream_t stream) {
+  return hybrid_impl(layout, dtype, q, k, v, k_text, v_text, beta, beta_text, nullptr, g_soft, g_lin,
+                     rms_weight, rms_eps, out, out_soft, out_lin, workspace, workspace_bytes, stream);
+}
+
+int vdn_hybrid_attn_fwd_decay(const vdn_layout_t* layout, int dtype, const void* q, const void* k,
+                              const void* v, const void* k_text, const void* v_text,
+                              const float* beta, const float* beta_text, const float* alpha,
+                              const void* g_soft, const void* g_lin, const float* rms_weight,
+                              float rms_eps, void* out, void* out_soft, void* out_lin,
+                              void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!alpha) return VDN_ERR_INVALID;
+  return hybrid_impl(layout, dtype, q, k, v, k_text, v_text, beta, beta_text, alpha, g_soft, g_lin,
+                     rms_weight, rms_eps, out, out_soft, out_lin, workspace, workspace_bytes, stream);
 }
 
 int vdn_device_status(void) {

@@ -209,11 +209,12 @@ cudaError_t launch_readout_tc(const Layout& l, const void* q, const float* state
 cudaError_t read_and_clear_readout_status(int* status);
 
 // VDA: Gram into (am, bw) slots [B, H, F, d, d] (slot 0 = text), inverse in place
-// of am, scans into states [B, H, 2, J, d, d].
+// of am, scans into states [B, H, 2, J, d, d]. alpha (nullable) [B, F, H, d]: KDA
+// channel decay applied to the state before each frame is written.
 cudaError_t launch_vda_states(const Layout& l, int dtype, const void* k, const void* v,
                               const void* kt, const void* vt, const float* beta,
-                              const float* beta_text, float* am, float* bw, float* states,
-                              cudaStream_t st);
+                              const float* beta_text, const float* alpha, float* am, float* bw,
+                              float* states, cudaStream_t st);
 
 // Readout / norm / gates. mode 0: o_lin only (ungated, pre-norm) into out.
 // mode 1: out = sig(gs) o_soft + sig(gl) rms(o_lin); optional out_soft/out_lin.

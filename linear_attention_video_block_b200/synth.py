@@ -13,6 +13,11 @@ beta = sigmoid(logit), and q/k/v/text/gates are cast to the storage dtype
 (beta stays fp32). ``repeated_keys`` sets, for each (frame, head), every key row
 of the frame to that frame's first key row (the repeated-evidence ablation).
 
+``make_decay`` draws the optional per-frame, per-key-channel decay alpha
+[B, F, H, d] (fp32) from a second generator seeded with ``seed``:
+alpha = 1 - 0.2 u with u ~ U[0, 1), i.e. in (0.8, 1], the slow-forgetting range
+of a channel-wise decay gate; it leaves ``make_inputs``' draws unchanged.
+
 The workloads mirror the token grids of the video model the pages describe
 (48 x 84 latent grid at 768p, 30 x 52 at 480p-like, chunks of 5 latent frames,
 text prompt tokens); no dataset or trained weights are involved.
@@ -95,6 +100,15 @@ def make_inputs(layout: Layout, dtype: str, seed: int, repeated_keys: bool = Fal
     out["g_s"] = _normal((B, L, H, d), gen, device).to(st)
     out["g_l"] = _normal((B, L, H, d), gen, device).to(st)
     return out
+
+
+def make_decay(layout: Layout, seed: int, device: str = "cpu"):
+    """Per-frame channel decay alpha [B, F, H, d] float32 in (0.8, 1]."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    u = torch.rand((layout.B, layout.F, layout.H, layout.d), generator=gen,
+                   dtype=torch.float32, device=device)
+    return 1.0 - 0.2 * u
 
 
 def as_float64_numpy(inputs):

@@ -6,7 +6,9 @@ CPU fallback: the functions raise if the library or a CUDA device is missing.
 
 Public calls (same names as the C ABI, without the ``vdn_`` prefix):
   window_softmax_fwd, vda_scan_fwd, hybrid_attn_fwd, workspace_bytes,
-  device_status.
+  device_status, vda_scan_fwd_noalloc. vda_scan_fwd and hybrid_attn_fwd take an
+  optional ``alpha`` [B, F, H, d] float32 (KDA channel decay); when given they
+  call the ``_decay`` entry points.
 Tensors follow the C ABI's layout: q/k/v/gates/outputs [B, L, H, d],
 text k/v [B, T, H, d], beta [B, L, H] and beta_text [B, T, H] in float32.
 """
@@ -27,7 +29,8 @@ VDN_F32, VDN_BF16 = 0, 1
 STATUS = {0: "VDN_OK", 1: "VDN_ERR_INVALID", 2: "VDN_ERR_UNSUPPORTED",
           3: "VDN_ERR_WORKSPACE", 4: "VDN_ERR_CUDA", 5: "VDN_ERR_TIMEOUT"}
 EXPORTS = ("vdn_workspace_bytes", "vdn_window_softmax_fwd", "vdn_vda_scan_fwd",
-           "vdn_hybrid_attn_fwd", "vdn_device_status", "vdn_status_string")
+           "vdn_vda_scan_fwd_decay", "vdn_hybrid_attn_fwd", "vdn_hybrid_attn_fwd_decay",
+           "vdn_vda_scan_fwd_noalloc", "vdn_device_status", "vdn_status_string")
 
 
 class VdnError(RuntimeError):
@@ -59,6 +62,13 @@ def lib():
         L.vdn_vda_scan_fwd.restype = I
         L.vdn_hybrid_attn_fwd.argtypes = [LP, I] + [P] * 9 + [P, ctypes.c_float] + [P] * 3 + [P, S, P]
         L.vdn_hybrid_attn_fwd.restype = I
+        L.vdn_vda_scan_fwd_decay.argtypes = [LP, I] + [P] * 10 + [P, S, P]
+        L.vdn_vda_scan_fwd_decay.restype = I
+        L.vdn_hybrid_attn_fwd_decay.argtypes = ([LP, I] + [P] * 10 + [P, ctypes.c_float]
+                                                + [P] * 3 + [P, S, P])
+        L.vdn_hybrid_attn_fwd_decay.restype = I
+        L.vdn_vda_scan_fwd_noalloc.argtypes = [LP, I] + [P] * 10
+        L.vdn_vda_scan_fwd_noalloc.restype = I
         L.vdn_device_status.argtypes = []
         L.vdn_device_status.restype = I
         L.vdn_status_string.argtypes = [I]
@@ -124,9 +134,10 @@ def window_softmax_fwd(layout: Layout, q, k, v, k_text, v_text, o_soft=None, lse
 
 
 def vda_scan_fwd(layout: Layout, q, k, v, k_text, v_text, beta, beta_text, o_lin=None,
-                 chunk_states=None, want_states=False, workspace=None):
+                 chunk_states=None, want_states=False, workspace=None, alpha=None):
     """Linear branch: returns o_lin (ungated, pre-norm) and, if want_states, the
-    chunk table [B, H, 2, J, d, d] float32."""
+    chunk table [B, H, 2, J, d, d] float32. alpha (optional, [B, F, H, d]
+    float32) decays the state per key channel before each frame's write."""
     _require_cuda()
     if o_lin is None:
         o_lin = torch.empty_like(q)
@@ -136,18 +147,23 @@ def vda_scan_fwd(layout: Layout, q, k, v, k_text, v_text, beta, beta_text, o_lin
                                    dtype=torch.float32, device=q.device)
     if workspace is None:
         workspace = torch.empty(workspace_bytes(layout, q.dtype), dtype=torch.uint8, device=q.device)
-    code = lib().vdn_vda_scan_fwd(
-        ctypes.byref(_clayout(layout)), _dtype_code(q), _ptr(q), _ptr(k), _ptr(v),
-        _ptr(k_text), _ptr(v_text), _ptr(beta), _ptr(beta_text), _ptr(o_lin),
-        _ptr(chunk_states), _ptr(workspace), workspace.numel(), _stream(q.device))
-    _check(code, "vdn_vda_scan_fwd")
+    head = [ctypes.byref(_clayout(layout)), _dtype_code(q), _ptr(q), _ptr(k), _ptr(v),
+            _ptr(k_text), _ptr(v_text), _ptr(beta), _ptr(beta_text)]
+    tail = [_ptr(o_lin), _ptr(chunk_states), _ptr(workspace), workspace.numel(), _stream(q.device)]
+    if alpha is None:
+        code, name = lib().vdn_vda_scan_fwd(*head, *tail), "vdn_vda_scan_fwd"
+    else:
+        code = lib().vdn_vda_scan_fwd_decay(*head, _ptr(alpha), *tail)
+        name = "vdn_vda_scan_fwd_decay"
+    _check(code, name)
     return (o_lin, chunk_states) if want_states else o_lin
 
 
 def hybrid_attn_fwd(layout: Layout, q, k, v, k_text, v_text, beta, beta_text, g_soft, g_lin,
                     rms_weight=None, rms_eps=1e-6, out=None, out_soft=None, out_lin=None,
-                    workspace=None, device=None):
+                    workspace=None, device=None, alpha=None):
     """The hybrid forward: out = sigmoid(g_soft) o_soft + sigmoid(g_lin) RMSNorm(o_lin).
+    alpha (optional, [B, F, H, d] float32): KDA decay of the linear branch.
 
     Device tensors: launched asynchronously on the current stream; returns out.
     Host tensors: copied to ``device`` (default cuda:0), computed, and the
@@ -161,19 +177,23 @@ def hybrid_attn_fwd(layout: Layout, q, k, v, k_text, v_text, beta, beta_text, g_
         out_host, out = out, None
         if out_soft is not None or out_lin is not None:
             raise ValueError("out_soft/out_lin need device tensors")
-        args = [q, k, v, k_text, v_text, beta, beta_text, g_soft, g_lin, rms_weight]
-        q, k, v, k_text, v_text, beta, beta_text, g_soft, g_lin, rms_weight = [
+        args = [q, k, v, k_text, v_text, beta, beta_text, g_soft, g_lin, rms_weight, alpha]
+        q, k, v, k_text, v_text, beta, beta_text, g_soft, g_lin, rms_weight, alpha = [
             None if a is None else a.to(dev, non_blocking=True) for a in args]
     if out is None:
         out = torch.empty_like(q)
     if workspace is None:
         workspace = torch.empty(workspace_bytes(layout, q.dtype), dtype=torch.uint8, device=q.device)
-    code = lib().vdn_hybrid_attn_fwd(
-        ctypes.byref(_clayout(layout)), _dtype_code(q), _ptr(q), _ptr(k), _ptr(v),
-        _ptr(k_text), _ptr(v_text), _ptr(beta), _ptr(beta_text), _ptr(g_soft), _ptr(g_lin),
-        _ptr(rms_weight), ctypes.c_float(rms_eps), _ptr(out), _ptr(out_soft), _ptr(out_lin),
-        _ptr(workspace), workspace.numel(), _stream(q.device))
-    _check(code, "vdn_hybrid_attn_fwd")
+    head = [ctypes.byref(_clayout(layout)), _dtype_code(q), _ptr(q), _ptr(k), _ptr(v),
+            _ptr(k_text), _ptr(v_text), _ptr(beta), _ptr(beta_text)]
+    tail = [_ptr(g_soft), _ptr(g_lin), _ptr(rms_weight), ctypes.c_float(rms_eps), _ptr(out),
+            _ptr(out_soft), _ptr(out_lin), _ptr(workspace), workspace.numel(), _stream(q.device)]
+    if alpha is None:
+        code, name = lib().vdn_hybrid_attn_fwd(*head, *tail), "vdn_hybrid_attn_fwd"
+    else:
+        code = lib().vdn_hybrid_attn_fwd_decay(*head, _ptr(alpha), *tail)
+        name = "vdn_hybrid_attn_fwd_decay"
+    _check(code, name)
     if host:
         if out_host is None:
             out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
@@ -194,11 +214,7 @@ def vda_scan_fwd_noalloc(layout: Layout, q, k, v, k_text, v_text, beta, beta_tex
     overlapping calls race). o_lin (and chunk_states, if wanted) are
     caller-provided device tensors."""
     _require_cuda()
-    f = lib().vdn_vda_scan_fwd_noalloc
-    if f.argtypes is None:
-        f.argtypes = [ctypes.POINTER(_CLayout), ctypes.c_int] + [ctypes.c_void_p] * 10
-        f.restype = ctypes.c_int
-    code = f(ctypes.byref(_clayout(layout)), _dtype_code(q), _ptr(q), _ptr(k), _ptr(v),
+    code = lib().vdn_vda_scan_fwd_noalloc(ctypes.byref(_clayout(layout)), _dtype_code(q), _ptr(q), _ptr(k), _ptr(v),
              _ptr(k_text), _ptr(v_text), _ptr(beta), _ptr(beta_text), _ptr(o_lin),
              _ptr(chunk_states), _stream(q.device))
     _check(code, "vdn_vda_scan_fwd_noalloc")

@@ -26,7 +26,7 @@ import pytest
 import torch
 
 from linear_attention_video_block_b200 import vdn
-from linear_attention_video_block_b200.synth import Layout, WORKLOADS, make_inputs
+from linear_attention_video_block_b200.synth import Layout, WORKLOADS, make_decay, make_inputs
 from oracle import vdn_oracle as O
 
 from conftest import bf16_storage_ratio, rel_err
@@ -72,18 +72,21 @@ def name_of(layout):
     return "B{B}F{F}N{N}T{T}c{c}H{H}d{d}".format(**layout.as_dict())
 
 
-def _check_all(layout, dtype, inp, heads=None, rows=None):
-    """Runs the three entry points and compares with the oracle on (heads, rows)."""
+def _check_all(layout, dtype, inp, heads=None, rows=None, alpha=None):
+    """Runs the three entry points (the _decay forms when alpha is given) and
+    compares with the oracle on (heads, rows)."""
     tol = TOL[dtype]
     d = _dev(inp)
+    alpha_d = None if alpha is None else alpha.to("cuda")
     o_soft, lse = vdn.window_softmax_fwd(layout, d["q"], d["k"], d["v"], d["k_text"], d["v_text"],
                                          want_lse=True)
     o_lin, states = vdn.vda_scan_fwd(layout, d["q"], d["k"], d["v"], d["k_text"], d["v_text"],
-                                     d["beta"], d["beta_text"], want_states=True)
+                                     d["beta"], d["beta_text"], want_states=True, alpha=alpha_d)
     out_soft = torch.empty_like(d["q"])
     out_lin = torch.empty_like(d["q"])
     out = vdn.hybrid_attn_fwd(layout, d["q"], d["k"], d["v"], d["k_text"], d["v_text"], d["beta"],
-                              d["beta_text"], d["g_s"], d["g_l"], out_soft=out_soft, out_lin=out_lin)
+                              d["beta_text"], d["g_s"], d["g_l"], out_soft=out_soft, out_lin=out_lin,
+                              alpha=alpha_d)
     torch.cuda.synchronize()
     assert vdn.device_status() == 0
     hsel = list(range(layout.H)) if heads is None else heads
@@ -91,8 +94,9 @@ def _check_all(layout, dtype, inp, heads=None, rows=None):
     F, N, c = layout.F, layout.N, layout.c
     ref_soft, ref_lse = O.softmax_branch(a["q"], a["k"], a["v"], a["k_text"], a["v_text"], F, N, c,
                                          rows=rows, return_lse=True)
+    a_np = None if alpha is None else _np(alpha, hsel)
     ref_lin, st = O.linear_branch(a["q"], a["k"], a["v"], a["k_text"], a["v_text"], a["beta"],
-                                  a["beta_text"], F, N, c, return_states=True)
+                                  a["beta_text"], F, N, c, return_states=True, alpha=a_np)
     ref_out, ref_gs, ref_gl = O.combine(ref_soft, ref_lin, a["g_s"], a["g_l"])
     res = {}
     comp = {"out": (out, ref_out), "o_soft": (o_soft, ref_soft), "o_lin": (o_lin, ref_lin),
@@ -129,7 +133,8 @@ def _check_all(layout, dtype, inp, heads=None, rows=None):
         else:
             assert res[key + "_storage_ratio"] <= 1.0, (key, res)
     assert res["lse"] <= (1e-4 if dtype == "f32" else 1e-3), res
-    print(name_of(layout), dtype, {k: round(v, 6) for k, v in res.items()})
+    print(name_of(layout), dtype, "decay" if alpha is not None else "",
+          {k: round(v, 6) for k, v in res.items()})
     return res
 
 
@@ -213,3 +218,46 @@ def test_repeated_calls_are_deterministic():
     a = vdn.hybrid_attn_fwd(*args).clone()
     b = vdn.hybrid_attn_fwd(*args)
     assert torch.equal(a, b)
+
+
+# KDA channel decay (the _decay entry points): alpha in (0.8, 1] per frame and
+# key channel, same bounds as without decay.
+DECAY = [
+    ("tiny-f32", None), ("small-bf16", None),
+    ("no-text", Layout(B=1, F=9, N=70, T=0, c=2, H=2, d=128)),
+    ("one-token-frames", Layout(B=1, F=12, N=1, T=2, c=2, H=3, d=64)),
+    ("f32-d16-no-text", Layout(B=1, F=13, N=8, T=0, c=4, H=2, d=16)),
+]
+
+
+@pytest.mark.parametrize("name,layout", DECAY, ids=[e[0] for e in DECAY])
+def test_decay_small_full(name, layout):
+    if layout is None:
+        layout, dtype, seed = WORKLOADS[name]
+    else:
+        dtype, seed = ("f32" if name.startswith("f32") else "bf16"), 200 + len(name)
+    inp = make_inputs(layout, dtype, seed)
+    _check_all(layout, dtype, inp, alpha=make_decay(layout, seed + 1))
+
+
+@pytest.mark.parametrize("name", ["480p-bf16", "768p-bf16"])
+def test_decay_full_size_sampled(name):
+    layout, dtype, seed = WORKLOADS[name]
+    inp = make_inputs(layout, dtype, seed)
+    _check_all(layout, dtype, inp, heads=[0, layout.H - 1], rows=_sample_rows(layout, 16),
+               alpha=make_decay(layout, seed + 1))
+
+
+def test_unit_decay_is_bit_identical_to_no_decay():
+    """alpha = 1 everywhere: S * 1 + B is exact, so the _decay entries reproduce
+    the plain entries bit for bit."""
+    layout, dtype, seed = WORKLOADS["small-bf16"]
+    d = _dev(make_inputs(layout, dtype, seed))
+    ones = torch.ones((layout.B, layout.F, layout.H, layout.d), dtype=torch.float32, device="cuda")
+    args = (layout, d["q"], d["k"], d["v"], d["k_text"], d["v_text"], d["beta"], d["beta_text"])
+    a, sa = vdn.vda_scan_fwd(*args, want_states=True)
+    b, sb = vdn.vda_scan_fwd(*args, want_states=True, alpha=ones)
+    assert torch.equal(a, b) and torch.equal(sa, sb)
+    ha = vdn.hybrid_attn_fwd(*args, d["g_s"], d["g_l"])
+    hb = vdn.hybrid_attn_fwd(*args, d["g_s"], d["g_l"], alpha=ones)
+    assert torch.equal(ha, hb)

@@ -78,6 +78,24 @@ def test_validation_rejects_before_any_launch(lib):
     assert h(ctypes.byref(ok), 0, *hargs[:9], None, ctypes.c_float(-1.0), FAKE, None, None, FAKE, need, None) == 1
 
 
+def test_decay_entries_validate_alpha(lib):
+    """The _decay entry points require alpha and its alignment; everything else is
+    validated as in the plain entries (no GPU is touched by any of these)."""
+    ok = _layout()
+    need = lib.vdn_workspace_bytes(ctypes.byref(ok), 0)
+    v = lib.vdn_vda_scan_fwd_decay
+    pre = [FAKE] * 7                                    # q k v kt vt beta beta_text
+    assert v(ctypes.byref(ok), 0, *pre, None, FAKE, None, FAKE, need, None) == 1
+    assert v(ctypes.byref(ok), 0, *pre, MISALIGNED, FAKE, None, FAKE, need, None) == 2
+    assert v(ctypes.byref(ok), 0, *pre, FAKE, FAKE, None, FAKE, 256, None) == 3
+    assert v(ctypes.byref(_layout(F=0)), 0, *pre, FAKE, FAKE, None, FAKE, need, None) == 1
+    h = lib.vdn_hybrid_attn_fwd_decay
+    post = [FAKE, FAKE, None, ctypes.c_float(1e-6), FAKE, None, None, FAKE]
+    assert h(ctypes.byref(ok), 0, *pre, None, *post, need, None) == 1
+    assert h(ctypes.byref(ok), 0, *pre, MISALIGNED, *post, need, None) == 2
+    assert h(ctypes.byref(ok), 0, *pre, FAKE, *post, need - 1, None) == 3
+
+
 @pytest.fixture(scope="module")
 def schedule_dump():
     out = os.path.join(tempfile.mkdtemp(), "schedule_dump")
