@@ -18,6 +18,13 @@ of the frame to that frame's first key row (the repeated-evidence ablation).
 alpha = 1 - 0.2 u with u ~ U[0, 1), i.e. in (0.8, 1], the slow-forgetting range
 of a channel-wise decay gate; it leaves ``make_inputs``' draws unchanged.
 
+``make_context`` draws the other tokens of a joint text-video-audio layer from a
+third generator seeded with ``seed``: q_text [B, T, H, d], then q_audio,
+k_audio, v_audio [B, A, H, d], all ~ N(0, 1), audio keys L2-normalised like the
+others. ``audio_tokens(F)`` is the audio length that goes with F latent frames
+in the H3 data layout: 575 audio latents (40 per second) beside 102 latent
+frames, so A = round(575 F / 102) (203 at F = 36).
+
 The workloads mirror the token grids of the video model the pages describe
 (48 x 84 latent grid at 768p, 30 x 52 at 480p-like, chunks of 5 latent frames,
 text prompt tokens); no dataset or trained weights are involved.
@@ -109,6 +116,25 @@ def make_decay(layout: Layout, seed: int, device: str = "cpu"):
     u = torch.rand((layout.B, layout.F, layout.H, layout.d), generator=gen,
                    dtype=torch.float32, device=device)
     return 1.0 - 0.2 * u
+
+
+def audio_tokens(F: int) -> int:
+    """Audio tokens beside F latent frames (575 audio latents per 102 frames)."""
+    return int(round(575 * F / 102))
+
+
+def make_context(layout: Layout, A: int, dtype: str, seed: int, device: str = "cpu"):
+    """Text query rows and the audio tokens of a joint layer (see module doc)."""
+    B, T, H, d = layout.B, layout.T, layout.H, layout.d
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    st = TORCH_DTYPES[dtype]
+    out = {}
+    out["q_text"] = _normal((B, T, H, d), gen, device).to(st)
+    out["q_audio"] = _normal((B, A, H, d), gen, device).to(st)
+    out["k_audio"] = _l2_normalise_(_normal((B, A, H, d), gen, device)).to(st)
+    out["v_audio"] = _normal((B, A, H, d), gen, device).to(st)
+    return out
 
 
 def as_float64_numpy(inputs):

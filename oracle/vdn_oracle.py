@@ -47,6 +47,14 @@ Readings of points the pages leave open (the CUDA path uses the same ones):
   R9  RMSNorm over d per head, eps = 1e-6, weight 1 unless given.
   R10 Gates are element-wise logits of shape [B, L, H, d] for both branches:
       out = sigmoid(g_s) * o_soft + sigmoid(g_l) * RMSNorm(o_lin).
+  R14 Audio and the context query rows (joint attention layer): the video
+      queries' softmax also sees every audio token (after the text keys, one
+      normaliser); audio is never written into the VDA states (only the text
+      prompt is). Text and audio query rows keep the original dense softmax
+      over every key of the layer (all video, text and audio tokens), scale
+      1/sqrt(d), no gates (the output projections are outside this op)
+      [VDN "Local Softmax ...", attention-map paragraph; glonce "Video DeltaNet
+      speeds MiniMax H3 video generation 14.5x", key facts].
   Parity unpinned beyond the invariants tested: R5 (beyond "text counted exactly
   once"), R9 constants, R10 granularity.
 
@@ -54,6 +62,8 @@ Tensor layout (numpy float64 arrays):
   q, k, v, g_s, g_l : [B, L, H, d], L = F * N, token index = f * N + n
   k_text, v_text    : [B, T, H, d]
   beta              : [B, L, H];  beta_text : [B, T, H]
+  q_text            : [B, T, H, d]  (context query rows, R14)
+  q_audio, k_audio, v_audio : [B, A, H, d]
 """
 
 from __future__ import annotations
@@ -162,9 +172,9 @@ def token_mask(F: int, N: int, T: int, c: int) -> np.ndarray:
 # ----------------------------------------------------------------------------
 
 def softmax_branch(q, k, v, k_text, v_text, F, N, c, rows=None, heads=None,
-                   return_lse=False):
+                   return_lse=False, k_audio=None, v_audio=None):
     """o_soft = softmax(q K^T / sqrt(d) over the allowed keys) V, one normaliser
-    over window + anchors + text (R4).
+    over window + anchors + text (R4), and the audio keys when given (R14).
 
     A dense masked softmax: for each query frame the boolean mask row is built
     explicitly and disallowed scores are set to -inf before max-subtraction.
@@ -175,7 +185,10 @@ def softmax_branch(q, k, v, k_text, v_text, F, N, c, rows=None, heads=None,
     Returns o_soft [B, L, H, d] (and lse [B, L, H], natural log, if asked).
     """
     Bn, L, H, d = q.shape
-    T = k_text.shape[1]
+    if k_audio is None:
+        k_audio = np.zeros((Bn, 0, H, d))
+        v_audio = np.zeros((Bn, 0, H, d))
+    T = k_text.shape[1] + k_audio.shape[1]     # every globally visible key
     assert L == F * N
     out = np.full(q.shape, np.nan)
     lse = np.full((Bn, L, H), np.nan)
@@ -186,8 +199,8 @@ def softmax_branch(q, k, v, k_text, v_text, F, N, c, rows=None, heads=None,
     row_frames = rows // N
     for b in range(Bn):
         for h in heads:
-            keys = np.concatenate([k[b, :, h, :], k_text[b, :, h, :]], axis=0)
-            vals = np.concatenate([v[b, :, h, :], v_text[b, :, h, :]], axis=0)
+            keys = np.concatenate([k[b, :, h, :], k_text[b, :, h, :], k_audio[b, :, h, :]], axis=0)
+            vals = np.concatenate([v[b, :, h, :], v_text[b, :, h, :], v_audio[b, :, h, :]], axis=0)
             for f in np.unique(row_frames):
                 sel = rows[row_frames == f]
                 allowed = np.zeros(L + T, dtype=bool)
@@ -202,6 +215,36 @@ def softmax_branch(q, k, v, k_text, v_text, F, N, c, rows=None, heads=None,
                 z = p.sum(axis=1, keepdims=True)
                 out[b, sel, h, :] = (p @ vals) / z
                 lse[b, sel, h] = (m + np.log(z))[:, 0]
+    return (out, lse) if return_lse else out
+
+
+def context_rows(q_ctx, k, v, k_text, v_text, k_audio=None, v_audio=None, heads=None,
+                 return_lse=False):
+    """Text or audio query rows (R14): the dense softmax of the original layer,
+    softmax(q K^T / sqrt(d)) V over every video, text and audio key.
+
+    q_ctx: [B, R, H, d] query rows (text or audio). Returns [B, R, H, d] (and
+    the natural-log normaliser [B, R, H] if asked); heads outside ``heads``
+    are NaN.
+    """
+    Bn, R, H, d = q_ctx.shape
+    if k_audio is None:
+        k_audio = np.zeros((Bn, 0, H, d))
+        v_audio = np.zeros((Bn, 0, H, d))
+    out = np.full(q_ctx.shape, np.nan)
+    lse = np.full((Bn, R, H), np.nan)
+    heads = range(H) if heads is None else heads
+    scale = 1.0 / np.sqrt(d)
+    for b in range(Bn):
+        for h in heads:
+            keys = np.concatenate([k[b, :, h, :], k_text[b, :, h, :], k_audio[b, :, h, :]], axis=0)
+            vals = np.concatenate([v[b, :, h, :], v_text[b, :, h, :], v_audio[b, :, h, :]], axis=0)
+            s = (q_ctx[b, :, h, :] @ keys.T) * scale
+            m = s.max(axis=1, keepdims=True)
+            p = np.exp(s - m)
+            z = p.sum(axis=1, keepdims=True)
+            out[b, :, h, :] = (p @ vals) / z
+            lse[b, :, h] = (m + np.log(z))[:, 0]
     return (out, lse) if return_lse else out
 
 
@@ -348,6 +391,30 @@ def hybrid(q, k, v, k_text, v_text, beta, beta_text, g_s, g_l, F, N, c,
                           alpha=alpha)
     out, gs, gl = combine(o_soft, o_lin, g_s, g_l, eps, weight)
     return {"out": out, "out_soft": gs, "out_lin": gl, "o_soft": o_soft, "o_lin": o_lin}
+
+
+def joint_attention(q, k, v, k_text, v_text, beta, beta_text, g_s, g_l, F, N, c,
+                    q_text=None, q_audio=None, k_audio=None, v_audio=None,
+                    rows=None, heads=None, eps=RMS_EPS, weight=None, alpha=None):
+    """The attention of one joint text-video-audio layer (R14): video rows take
+    the hybrid (softmax branch with text and audio keys, VDA with the text
+    init), text and audio query rows the dense softmax.
+
+    Returns the dict of ``hybrid`` plus o_text and o_audio (None when the
+    corresponding query rows are not given).
+    """
+    o_soft = softmax_branch(q, k, v, k_text, v_text, F, N, c, rows=rows, heads=heads,
+                            k_audio=k_audio, v_audio=v_audio)
+    o_lin = linear_branch(q, k, v, k_text, v_text, beta, beta_text, F, N, c, heads=heads,
+                          alpha=alpha)
+    out, gs, gl = combine(o_soft, o_lin, g_s, g_l, eps, weight)
+    res = {"out": out, "out_soft": gs, "out_lin": gl, "o_soft": o_soft, "o_lin": o_lin,
+           "o_text": None, "o_audio": None}
+    if q_text is not None:
+        res["o_text"] = context_rows(q_text, k, v, k_text, v_text, k_audio, v_audio, heads=heads)
+    if q_audio is not None:
+        res["o_audio"] = context_rows(q_audio, k, v, k_text, v_text, k_audio, v_audio, heads=heads)
+    return res
 
 
 # ----------------------------------------------------------------------------

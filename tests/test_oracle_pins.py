@@ -545,3 +545,84 @@ def test_unit_decay_is_no_decay():
     a = O.hybrid(q, k, v, kt, vt, beta, bt, gs, gl, F, N, c)["out"]
     b = O.hybrid(q, k, v, kt, vt, beta, bt, gs, gl, F, N, c, alpha=np.ones((B, F, H, d)))["out"]
     np.testing.assert_array_equal(a, b)
+
+
+# ---------------------------------------------- joint layer: audio, context rows ---
+
+def _rand_context(rng, B, T, A, H, d):
+    qt = rng.standard_normal((B, T, H, d))
+    qa = rng.standard_normal((B, A, H, d))
+    ka = rng.standard_normal((B, A, H, d))
+    if A:
+        ka /= np.linalg.norm(ka, axis=-1, keepdims=True)
+    va = rng.standard_normal((B, A, H, d))
+    return qt, qa, ka, va
+
+
+def _sdpa_rows(qrows, keys, vals):
+    """torch float64 scaled_dot_product_attention of [B, R, H, d] query rows over
+    [B, S, H, d] keys/values, back in [B, R, H, d]."""
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x)).permute(0, 2, 1, 3)
+    return torch.nn.functional.scaled_dot_product_attention(
+        t(qrows), t(keys), t(vals)).permute(0, 2, 1, 3).numpy()
+
+
+def test_joint_layer_is_dense_attention_when_windows_cover_the_clip():
+    """Project page, attention-map paragraph, and the H3 key facts (text and audio
+    interactions stay dense softmax): with F <= 2c every video window covers the
+    clip, so the softmax part of the joint layer is the original dense attention
+    of the whole sequence [text; video; audio] for every query row. Compared with
+    torch's SDPA over the concatenated sequence."""
+    rng = np.random.default_rng(40)
+    B, F, N, T, A, H, d, c = 2, 5, 4, 3, 2, 2, 8, 3
+    q, k, v, kt, vt, beta, bt, gs, gl = _rand_inputs(rng, B, F, N, T, H, d)
+    qt, qa, ka, va = _rand_context(rng, B, T, A, H, d)
+    res = O.joint_attention(q, k, v, kt, vt, beta, bt, gs, gl, F, N, c,
+                            q_text=qt, q_audio=qa, k_audio=ka, v_audio=va)
+    seq_q = np.concatenate([qt, q, qa], 1)
+    seq_k = np.concatenate([kt, k, ka], 1)
+    seq_v = np.concatenate([vt, v, va], 1)
+    dense = _sdpa_rows(seq_q, seq_k, seq_v)
+    L = F * N
+    np.testing.assert_allclose(res["o_text"], dense[:, :T], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(res["o_soft"], dense[:, T:T + L], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(res["o_audio"], dense[:, T + L:], rtol=1e-12, atol=1e-12)
+
+
+def test_context_rows_are_dense_for_any_window():
+    """Text and audio query rows see every key however small the video window:
+    at F = 13, c = 2 they still equal dense SDPA over all video, text and audio
+    keys, and their normaliser is the full logsumexp."""
+    rng = np.random.default_rng(41)
+    B, F, N, T, A, H, d, c = 1, 13, 3, 4, 3, 2, 8, 2
+    q, k, v, kt, vt, *_ = _rand_inputs(rng, B, F, N, T, H, d)
+    qt, qa, ka, va = _rand_context(rng, B, T, A, H, d)
+    keys = np.concatenate([k, kt, ka], 1)
+    vals = np.concatenate([v, vt, va], 1)
+    for qr in (qt, qa):
+        got, lse = O.context_rows(qr, k, v, kt, vt, ka, va, return_lse=True)
+        np.testing.assert_allclose(got, _sdpa_rows(qr, keys, vals), rtol=1e-12, atol=1e-12)
+        tq = torch.from_numpy(qr).permute(0, 2, 1, 3)
+        tk = torch.from_numpy(keys).permute(0, 2, 1, 3)
+        ref_lse = torch.logsumexp(tq @ tk.transpose(-1, -2) / np.sqrt(d), -1).permute(0, 2, 1)
+        np.testing.assert_allclose(lse, ref_lse.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_audio_keys_reach_every_video_query_and_no_state():
+    """An audio key aligned with every query and of large norm takes the whole
+    softmax mass of every video row, boundary or not (audio is globally visible);
+    the linear branch ignores audio entirely (only the text prompt is written
+    into the VDA states)."""
+    rng = np.random.default_rng(42)
+    B, F, N, T, A, H, d, c = 1, 14, 2, 2, 2, 1, 4, 2
+    q, k, v, kt, vt, beta, bt, gs, gl = _rand_inputs(rng, B, F, N, T, H, d)
+    q[...] = np.abs(q) + 0.5            # every query in the positive orthant
+    _, _, ka, va = _rand_context(rng, B, T, A, H, d)
+    ka[0, 0, 0] = 200.0 * np.ones(d)     # dominates every video query's scores
+    va[0, 0, 0] = np.arange(1.0, d + 1)
+    res = O.joint_attention(q, k, v, kt, vt, beta, bt, gs, gl, F, N, c, k_audio=ka, v_audio=va)
+    np.testing.assert_allclose(res["o_soft"][0, :, 0], np.tile(va[0, 0, 0], (F * N, 1)), atol=1e-12)
+    no_audio = O.joint_attention(q, k, v, kt, vt, beta, bt, gs, gl, F, N, c)
+    np.testing.assert_array_equal(res["o_lin"], no_audio["o_lin"])
+    # without audio the video rows reduce to the plain hybrid
+    np.testing.assert_array_equal(no_audio["out"], O.hybrid(q, k, v, kt, vt, beta, bt, gs, gl, F, N, c)["out"])
