@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload 768p-bf16]
-                    [--entry hybrid|window|vda|vda-decay|hybrid-decay]
+                    [--entry hybrid|window|vda|vda-decay|hybrid-decay|joint|joint-window]
 
 A step is one vdn_hybrid_attn_fwd call (window softmax + VDA scans + readout,
 norm, gates) over one 768p-like layer input (B=1, H=40, d=128, F=36 frames of
@@ -18,7 +18,10 @@ reported time is the maximum over ranks.
 forward (default, the headline), or the softmax branch or the linear branch
 alone (vdn_window_softmax_fwd / vdn_vda_scan_fwd), for per-branch numbers and
 for profiling one kernel family at a time, or the KDA-decayed forms
-(vdn_vda_scan_fwd_decay / vdn_hybrid_attn_fwd_decay, alpha in (0.8, 1]).
+(vdn_vda_scan_fwd_decay / vdn_hybrid_attn_fwd_decay, alpha in (0.8, 1]), or
+the joint text-video-audio layer (vdn_joint_attn_fwd / vdn_joint_softmax_fwd:
+audio keys for every video query, dense text and audio query rows; the audio
+length that goes with the clip, 203 tokens at 768p).
 
 Printed on rank 0: one JSON line with the throughput (video tokens/s over all
 ranks), the roofline of the dominant kernel (window softmax, tensor-core bound),
@@ -68,6 +71,14 @@ def window_pairs(lay) -> int:
 def window_flops(lay) -> float:
     """4 d flops per allowed pair (q.k and p.v), all heads and batches."""
     return 4.0 * lay.d * window_pairs(lay) * lay.H * lay.B
+
+
+def joint_flops(lay, A) -> float:
+    """Window flops of a joint layer: every video query also sees the A audio
+    keys, and the T text + A audio query rows see every video, text and audio
+    key (4 d flops per pair)."""
+    extra = lay.L * A + (lay.T + A) * (lay.L + lay.T + A)
+    return window_flops(lay) + 4.0 * lay.d * extra * lay.H * lay.B
 
 
 def launches_per_step(lay, dtype) -> int:
@@ -432,7 +443,8 @@ def run_entry(args, rank, world, local_rank):
     or the _decay forms of the linear branch and the hybrid forward."""
     import torch
     from linear_attention_video_block_b200 import vdn
-    from linear_attention_video_block_b200.synth import WORKLOADS, make_decay, make_inputs
+    from linear_attention_video_block_b200.synth import (WORKLOADS, audio_tokens, make_context,
+                                                         make_decay, make_inputs)
 
     lay, dtype, seed = WORKLOADS[args.workload]
     dev = torch.device("cuda", local_rank)
@@ -441,10 +453,29 @@ def run_entry(args, rank, world, local_rank):
     alpha = make_decay(lay, rank_seed(seed, rank) + 1, device=str(dev))
     out = torch.empty_like(inp["q"])
     ws = torch.empty(vdn.workspace_bytes(lay, inp["q"].dtype), dtype=torch.uint8, device=dev)
+    A = audio_tokens(lay.F)
+    cx = make_context(lay, A, dtype, rank_seed(seed, rank) + 7, device=str(dev)) \
+        if args.entry.startswith("joint") else None
     if args.entry == "window":
         def step():
             vdn.window_softmax_fwd(lay, inp["q"], inp["k"], inp["v"], inp["k_text"], inp["v_text"],
                                    o_soft=out)
+    elif args.entry == "joint":
+        o_text, o_audio = torch.empty_like(cx["q_text"]), torch.empty_like(cx["q_audio"])
+
+        def step():
+            vdn.joint_attn_fwd(lay, inp["q"], inp["k"], inp["v"], inp["k_text"], inp["v_text"],
+                               inp["beta"], inp["beta_text"], inp["g_s"], inp["g_l"],
+                               k_audio=cx["k_audio"], v_audio=cx["v_audio"], q_text=cx["q_text"],
+                               q_audio=cx["q_audio"], out=out, o_text=o_text, o_audio=o_audio,
+                               workspace=ws)
+    elif args.entry == "joint-window":
+        o_text, o_audio = torch.empty_like(cx["q_text"]), torch.empty_like(cx["q_audio"])
+
+        def step():
+            vdn.joint_softmax_fwd(lay, inp["q"], inp["k"], inp["v"], inp["k_text"], inp["v_text"],
+                                  k_audio=cx["k_audio"], v_audio=cx["v_audio"], q_text=cx["q_text"],
+                                  q_audio=cx["q_audio"], o_soft=out, o_text=o_text, o_audio=o_audio)
     elif args.entry == "hybrid-decay":
         def step():
             vdn.hybrid_attn_fwd(lay, inp["q"], inp["k"], inp["v"], inp["k_text"], inp["v_text"],
@@ -475,7 +506,10 @@ def run_entry(args, rank, world, local_rank):
     if args.entry == "window":
         work, unit, peak = window_flops(lay) / 1e12, "TFLOP/s", float(peaks["bf16_tflops"])
         bound = "tensor"
-    elif args.entry == "hybrid-decay":
+    elif args.entry == "joint-window":
+        work, unit, peak = joint_flops(lay, A) / 1e12, "TFLOP/s", float(peaks["bf16_tflops"])
+        bound = "tensor"
+    elif args.entry in ("hybrid-decay", "joint"):
         work, unit, peak, bound = None, None, None, None
     else:
         extra = decay_bytes(lay) if args.entry == "vda-decay" else 0.0
@@ -490,7 +524,10 @@ def run_entry(args, rank, world, local_rank):
         "impl": "ours", "entry": args.entry, "metric": f"{args.entry} fwd video tokens/s",
         "value": lay.L * lay.B / (ms * 1e-3), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "dtype": dtype,
-        "config": config_of(args.workload, lay), "roofline": roof,
+        "config": dict(config_of(args.workload, lay),
+                       **({"audio_tokens": A, "context_query_rows": lay.T + A}
+                          if args.entry.startswith("joint") else {})),
+        "roofline": roof,
     }), flush=True)
 
 
@@ -501,8 +538,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="768p-bf16")
-    ap.add_argument("--entry", choices=["hybrid", "window", "vda", "vda-decay", "hybrid-decay"],
-                    default="hybrid")
+    ap.add_argument("--entry", choices=["hybrid", "window", "vda", "vda-decay", "hybrid-decay",
+                                        "joint", "joint-window"], default="hybrid")
     ap.add_argument("--ref-rows", type=int, default=96,
                     help="query rows per frame in the oracle's bounded sample")
     args = ap.parse_args()

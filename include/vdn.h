@@ -157,6 +157,60 @@ int vdn_hybrid_attn_fwd_decay(const vdn_layout_t* layout, int dtype,
                               void* out, void* out_soft, void* out_lin,
                               void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* The other tokens of a joint text-video-audio attention layer (project page
+ * "Video DeltaNet", attention-map paragraph of "Local Softmax and Long-Range
+ * Linear Memory"; "Video DeltaNet speeds MiniMax H3 video generation 14.5x",
+ * key facts: the hybrid replaces only video-to-video attention, interactions
+ * involving text or audio keep the original softmax).
+ *   Audio keys: every video query's softmax also runs over all A audio tokens
+ *     (after the text keys, one normaliser). Audio is never written into the
+ *     VDA states; only the text prompt initialises them.
+ *   Context query rows: the text query rows (q_text, T rows) and the audio
+ *     query rows (q_audio, A rows) get the dense softmax over every key of the
+ *     layer (all L video, T text and A audio tokens), scale 1/sqrt(d), no gates
+ *     and no linear branch, written to o_text / o_audio in the io dtype, with
+ *     the natural-log normaliser in lse_text / lse_audio when given.
+ * Tensors are dense and row-major like the video ones: [B, T, H, d] for
+ * q_text/o_text, [B, A, H, d] for q_audio/k_audio/v_audio/o_audio, [B, T, H]
+ * and [B, A, H] float32 for the lse outputs; 16-byte aligned; caller-owned
+ * device memory. A NULL q_text (or T = 0) skips the text rows and a NULL
+ * q_audio (or A = 0) the audio rows; o_text / o_audio are then not touched.
+ * k_audio and v_audio are required when A > 0. */
+typedef struct {
+  int A;                  /* audio tokens, 0 <= A <= 2^30 */
+  const void* k_audio;    /* [B, A, H, d] */
+  const void* v_audio;    /* [B, A, H, d] */
+  const void* q_text;     /* nullable [B, T, H, d] */
+  const void* q_audio;    /* nullable [B, A, H, d] */
+  void* o_text;           /* [B, T, H, d], required with q_text when T > 0 */
+  void* o_audio;          /* [B, A, H, d], required with q_audio when A > 0 */
+  float* lse_text;        /* nullable [B, T, H] */
+  float* lse_audio;       /* nullable [B, A, H] */
+} vdn_context_t;
+
+/* Softmax part of a joint layer: vdn_window_softmax_fwd with the audio keys
+ * added to every video query's key set, plus the dense context query rows
+ * (vdn_context_t). ctx is required (VDN_ERR_INVALID if NULL). One launch: the
+ * context rows are extra query groups of the same grid. */
+int vdn_joint_softmax_fwd(const vdn_layout_t* layout, int dtype, const vdn_context_t* ctx,
+                          const void* q, const void* k, const void* v,
+                          const void* k_text, const void* v_text,
+                          void* o_soft, float* lse, cudaStream_t stream);
+
+/* The attention of a joint text-video-audio layer: video rows get the hybrid
+ * forward of vdn_hybrid_attn_fwd (their softmax branch also sees the audio
+ * keys), with the KDA decay of vdn_vda_scan_fwd_decay when alpha is not NULL;
+ * text and audio query rows get the dense softmax (vdn_context_t). ctx is
+ * required; workspace as for vdn_hybrid_attn_fwd (vdn_workspace_bytes). */
+int vdn_joint_attn_fwd(const vdn_layout_t* layout, int dtype, const vdn_context_t* ctx,
+                       const void* q, const void* k, const void* v,
+                       const void* k_text, const void* v_text,
+                       const float* beta, const float* beta_text, const float* alpha,
+                       const void* g_soft, const void* g_lin,
+                       const float* rms_weight, float rms_eps,
+                       void* out, void* out_soft, void* out_lin,
+                       void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* Size of the device scratch array behind vdn_vda_scan_fwd_noalloc: 64 MiB. */
 #define VDN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 

@@ -69,10 +69,59 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? VDN_OK : VDN_ERR_CUDA
 
 int run_window(const Layout& l, int dtype, const void* q, const void* k, const void* v,
                const void* kt, const void* vt, void* o, bool out_f32, float* lse,
-               cudaStream_t st) {
+               const vdn::JointArgs& ja, cudaStream_t st) {
   if (vdn::window_tc_supported(l, dtype))
-    return cuda_status(vdn::launch_window_tc(l, q, k, v, kt, vt, o, out_f32, lse, st));
-  return cuda_status(vdn::launch_window_simt(l, dtype, q, k, v, kt, vt, o, out_f32, lse, st));
+    return cuda_status(vdn::launch_window_tc(l, q, k, v, kt, vt, o, out_f32, lse, ja, st));
+  return cuda_status(vdn::launch_window_simt(l, dtype, q, k, v, kt, vt, o, out_f32, lse, ja, st));
+}
+
+// Validates the joint-layer context and returns the softmax launches' layout
+// (audio count and context query bits set) and tensors. ctx == nullptr: a
+// video-only call.
+int joint_setup(const vdn_layout_t* layout, const vdn_context_t* ctx, Layout& ls,
+                vdn::JointArgs& ja) {
+  ls = to_layout(layout);
+  ja = vdn::JointArgs{};
+  if (!ctx) return VDN_OK;
+  const int A = ctx->A;
+  if (A < 0 || A > (1 << 30)) return VDN_ERR_INVALID;
+  if ((long long)layout->B * A * layout->H * layout->d > (1LL << 46)) return VDN_ERR_INVALID;
+  if (A > 0 && (!ctx->k_audio || !ctx->v_audio)) return VDN_ERR_INVALID;
+  const bool text_rows = ctx->q_text != nullptr && layout->T > 0;
+  const bool audio_rows = ctx->q_audio != nullptr && A > 0;
+  if (text_rows && !ctx->o_text) return VDN_ERR_INVALID;
+  if (audio_rows && !ctx->o_audio) return VDN_ERR_INVALID;
+  const void* ptrs[] = {A > 0 ? ctx->k_audio : nullptr, A > 0 ? ctx->v_audio : nullptr,
+                        text_rows ? ctx->q_text : nullptr, text_rows ? ctx->o_text : nullptr,
+                        text_rows ? ctx->lse_text : nullptr, audio_rows ? ctx->q_audio : nullptr,
+                        audio_rows ? ctx->o_audio : nullptr, audio_rows ? ctx->lse_audio : nullptr};
+  for (const void* p : ptrs) if (p && !aligned16(p)) return VDN_ERR_UNSUPPORTED;
+  ls.A = A;
+  ls.ctx = (text_rows ? vdn::kCtxText : 0) | (audio_rows ? vdn::kCtxAudio : 0);
+  if (A > 0) { ja.k_audio = ctx->k_audio; ja.v_audio = ctx->v_audio; }
+  if (text_rows) { ja.q_text = ctx->q_text; ja.o_text = ctx->o_text; ja.lse_text = ctx->lse_text; }
+  if (audio_rows) {
+    ja.q_audio = ctx->q_audio; ja.o_audio = ctx->o_audio; ja.lse_audio = ctx->lse_audio;
+  }
+  return VDN_OK;
+}
+
+int window_impl(const vdn_layout_t* layout, int dtype, const vdn_context_t* ctx, const void* q,
+                const void* k, const void* v, const void* k_text, const void* v_text,
+                void* o_soft, float* lse, cudaStream_t stream) {
+  if (!layout_ok(layout)) return VDN_ERR_INVALID;
+  if (!dtype_d_ok(dtype, layout->d)) return VDN_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !o_soft) return VDN_ERR_INVALID;
+  if (layout->T > 0 && (!k_text || !v_text)) return VDN_ERR_INVALID;
+  const void* ptrs[] = {q, k, v, o_soft, lse};
+  for (const void* p : ptrs) if (p && !aligned16(p)) return VDN_ERR_UNSUPPORTED;
+  if (layout->T > 0 && (!aligned16(k_text) || !aligned16(v_text))) return VDN_ERR_UNSUPPORTED;
+  Layout ls;
+  vdn::JointArgs ja;
+  const int s = joint_setup(layout, ctx, ls, ja);
+  if (s != VDN_OK) return s;
+  return run_window(ls, dtype, q, k, v, layout->T ? k_text : nullptr,
+                    layout->T ? v_text : nullptr, o_soft, false, lse, ja, stream);
 }
 
 }  // namespace
@@ -88,16 +137,14 @@ size_t vdn_workspace_bytes(const vdn_layout_t* layout, int dtype) {
 int vdn_window_softmax_fwd(const vdn_layout_t* layout, int dtype, const void* q, const void* k,
                            const void* v, const void* k_text, const void* v_text, void* o_soft,
                            float* lse, cudaStream_t stream) {
-  if (!layout_ok(layout)) return VDN_ERR_INVALID;
-  if (!dtype_d_ok(dtype, layout->d)) return VDN_ERR_UNSUPPORTED;
-  if (!q || !k || !v || !o_soft) return VDN_ERR_INVALID;
-  if (layout->T > 0 && (!k_text || !v_text)) return VDN_ERR_INVALID;
-  const void* ptrs[] = {q, k, v, o_soft, lse};
-  for (const void* p : ptrs) if (p && !aligned16(p)) return VDN_ERR_UNSUPPORTED;
-  if (layout->T > 0 && (!aligned16(k_text) || !aligned16(v_text))) return VDN_ERR_UNSUPPORTED;
-  const Layout l = to_layout(layout);
-  return run_window(l, dtype, q, k, v, layout->T ? k_text : nullptr,
-                    layout->T ? v_text : nullptr, o_soft, false, lse, stream);
+  return window_impl(layout, dtype, nullptr, q, k, v, k_text, v_text, o_soft, lse, stream);
+}
+
+int vdn_joint_softmax_fwd(const vdn_layout_t* layout, int dtype, const vdn_context_t* ctx,
+                          const void* q, const void* k, const void* v, const void* k_text,
+                          const void* v_text, void* o_soft, float* lse, cudaStream_t stream) {
+  if (!ctx) return VDN_ERR_INVALID;
+  return window_impl(layout, dtype, ctx, q, k, v, k_text, v_text, o_soft, lse, stream);
 }
 
 }  // extern "C"
@@ -134,11 +181,12 @@ int vda_scan_impl(const vdn_layout_t* layout, int dtype, const void* q, const vo
                                          0.f, o_lin, nullptr, nullptr, stream));
 }
 
-int hybrid_impl(const vdn_layout_t* layout, int dtype, const void* q, const void* k,
-                const void* v, const void* k_text, const void* v_text, const float* beta,
-                const float* beta_text, const float* alpha, const void* g_soft, const void* g_lin,
-                const float* rms_weight, float rms_eps, void* out, void* out_soft, void* out_lin,
-                void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+int hybrid_impl(const vdn_layout_t* layout, int dtype, const vdn_context_t* ctx, const void* q,
+                const void* k, const void* v, const void* k_text, const void* v_text,
+                const float* beta, const float* beta_text, const float* alpha, const void* g_soft,
+                const void* g_lin, const float* rms_weight, float rms_eps, void* out,
+                void* out_soft, void* out_lin, void* workspace, size_t workspace_bytes,
+                cudaStream_t stream) {
   if (!layout_ok(layout)) return VDN_ERR_INVALID;
   if (!dtype_d_ok(dtype, layout->d)) return VDN_ERR_UNSUPPORTED;
   if (!q || !k || !v || !beta || !g_soft || !g_lin || !out) return VDN_ERR_INVALID;
@@ -149,6 +197,10 @@ int hybrid_impl(const vdn_layout_t* layout, int dtype, const void* q, const void
   if (layout->T > 0 && (!aligned16(k_text) || !aligned16(v_text) || !aligned16(beta_text)))
     return VDN_ERR_UNSUPPORTED;
   const Layout l = to_layout(layout);
+  Layout ls;  // the softmax launches' layout: with the audio keys and context rows
+  vdn::JointArgs ja;
+  const int js = joint_setup(layout, ctx, ls, ja);
+  if (js != VDN_OK) return js;
   // The tcgen05 path fuses readout, norm and gates into the window kernel and
   // needs no o_soft intermediate; the CUDA-core path keeps it in fp32.
   const bool fused = vdn::window_tc_supported(l, dtype);
@@ -162,9 +214,9 @@ int hybrid_impl(const vdn_layout_t* layout, int dtype, const void* q, const void
                                              w.states, stream));
   if (s != VDN_OK) return s;
   if (fused)
-    return cuda_status(vdn::launch_hybrid_tc(l, q, k, v, kt, vt, w.states, g_soft, g_lin, rms_weight,
-                                             rms_eps, out, out_soft, out_lin, stream));
-  s = run_window(l, dtype, q, k, v, kt, vt, w.o_soft, true, nullptr, stream);
+    return cuda_status(vdn::launch_hybrid_tc(ls, q, k, v, kt, vt, w.states, g_soft, g_lin, rms_weight,
+                                             rms_eps, out, out_soft, out_lin, ja, stream));
+  s = run_window(ls, dtype, q, k, v, kt, vt, w.o_soft, true, nullptr, ja, stream);
   if (s != VDN_OK) return s;
   return cuda_status(vdn::launch_readout(l, dtype, 1, q, w.states, w.o_soft, g_soft, g_lin,
                                          rms_weight, rms_eps, out, out_soft, out_lin, stream));
@@ -198,8 +250,9 @@ int vdn_hybrid_attn_fwd(const vdn_layout_t* layout, int dtype, const void* q, co
                         const float* rms_weight, float rms_eps, void* out, void* out_soft,
                         void* out_lin, void* workspace, size_t workspace_bytes,
                         cudaStream_t stream) {
-  return hybrid_impl(layout, dtype, q, k, v, k_text, v_text, beta, beta_text, nullptr, g_soft, g_lin,
-                     rms_weight, rms_eps, out, out_soft, out_lin, workspace, workspace_bytes, stream);
+  return hybrid_impl(layout, dtype, nullptr, q, k, v, k_text, v_text, beta, beta_text, nullptr, g_soft,
+                     g_lin, rms_weight, rms_eps, out, out_soft, out_lin, workspace, workspace_bytes,
+                     stream);
 }
 
 int vdn_hybrid_attn_fwd_decay(const vdn_layout_t* layout, int dtype, const void* q, const void* k,
@@ -209,8 +262,22 @@ int vdn_hybrid_attn_fwd_decay(const vdn_layout_t* layout, int dtype, const void*
                               float rms_eps, void* out, void* out_soft, void* out_lin,
                               void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   if (!alpha) return VDN_ERR_INVALID;
-  return hybrid_impl(layout, dtype, q, k, v, k_text, v_text, beta, beta_text, alpha, g_soft, g_lin,
-                     rms_weight, rms_eps, out, out_soft, out_lin, workspace, workspace_bytes, stream);
+  return hybrid_impl(layout, dtype, nullptr, q, k, v, k_text, v_text, beta, beta_text, alpha, g_soft,
+                     g_lin, rms_weight, rms_eps, out, out_soft, out_lin, workspace, workspace_bytes,
+                     stream);
+}
+
+int vdn_joint_attn_fwd(const vdn_layout_t* layout, int dtype, const vdn_context_t* ctx,
+                       const void* q, const void* k, const void* v, const void* k_text,
+                       const void* v_text, const float* beta, const float* beta_text,
+                       const float* alpha, const void* g_soft, const void* g_lin,
+                       const float* rms_weight, float rms_eps, void* out, void* out_soft,
+                       void* out_lin, void* workspace, size_t workspace_bytes,
+                       cudaStream_t stream) {
+  if (!ctx) return VDN_ERR_INVALID;
+  return hybrid_impl(layout, dtype, ctx, q, k, v, k_text, v_text, beta, beta_text, alpha, g_soft,
+                     g_lin, rms_weight, rms_eps, out, out_soft, out_lin, workspace, workspace_bytes,
+                     stream);
 }
 
 int vdn_device_status(void) {

@@ -5,12 +5,18 @@
 //   group 0          boundary frame 0          (sees every frame)
 //   group 1          boundary frame F-1        (sees every frame; absent if F < 2)
 //   group 2 + j      non-boundary frames of chunk j, j = 0 .. J-1 (may be empty)
-// The heavy boundary groups come first so that they are scheduled early.
+//   group J + 2      text query rows  (joint layer only; dense over every key)
+//   group J + 3      audio query rows (joint layer only; dense over every key)
+// Tiles are enumerated in schedule order: the context groups (the heaviest:
+// every key) first, then the boundary groups, then the chunks, so that the
+// long tiles start early.
 // Key set of a chunk group (project page "Local Softmax and Long-Range Linear
 // Memory": each chunk attends to itself and both neighbour chunks, plus the
 // 4-way boundary anchors and the text tokens): frames [lo, hi] with
 // lo = max(0, c(j-1)), hi = min(F-1, c(j+2)-1), plus frames 0 and F-1, merged
-// into at most 3 disjoint token intervals; text keys are a separate segment.
+// into at most 3 disjoint token intervals; the text keys and then the audio
+// keys are separate segments seen by every group. Only the softmax launches of
+// the joint layer set A or the context bits; the VDA kernels never see audio.
 #pragma once
 
 #include <cstdint>
@@ -23,13 +29,22 @@ namespace vdn {
 
 struct Layout {
   int B, F, N, T, c, H, d;
+  int A = 0;       // audio tokens: softmax keys of every query, never written to VDA
+  int ctx = 0;     // context query rows to compute: kCtxText | kCtxAudio
   __host__ __device__ long long L() const { return (long long)F * N; }
   __host__ __device__ int J() const { return (F + c - 1) / c; }
-  __host__ __device__ int groups() const { return J() + 2; }
+  __host__ __device__ int groups() const { return J() + 4; }
 };
 
+constexpr int kCtxText = 1;
+constexpr int kCtxAudio = 2;
+
+// Query source of a group: video tokens, text query rows or audio query rows.
+enum QuerySource { kQVideo = 0, kQText = 1, kQAudio = 2 };
+
 struct Group {
-  int q0;          // first video token of the group
+  int qsrc;        // QuerySource
+  int q0;          // first query token of the group (in its source tensor)
   int nq;          // number of query tokens (0 = empty group)
   int nseg;        // video key segments
   int seg0[3];     // segment start token
@@ -48,12 +63,24 @@ __host__ __device__ inline void chunk_window(const Layout& l, int j, int& lo, in
 
 __host__ __device__ inline Group make_group(const Layout& l, int g) {
   Group G;
+  G.qsrc = kQVideo;
   G.nseg = 0;
   G.chunk = -1;
   G.fwd_idx = 0;
   G.rev_idx = l.F - 1;
   for (int s = 0; s < 3; ++s) { G.seg0[s] = 0; G.segn[s] = 0; }
   const int N = l.N, F = l.F;
+  if (g >= l.J() + 2) {
+    // context query rows: every video token is a key
+    const bool text = g == l.J() + 2;
+    G.qsrc = text ? kQText : kQAudio;
+    G.q0 = 0;
+    G.nq = text ? ((l.ctx & kCtxText) ? l.T : 0) : ((l.ctx & kCtxAudio) ? l.A : 0);
+    G.nseg = 1;
+    G.seg0[0] = 0;
+    G.segn[0] = F * N;
+    return G;
+  }
   if (g == 0 || g == 1) {
     int f = (g == 0) ? 0 : F - 1;
     if (g == 1 && F < 2) { G.q0 = 0; G.nq = 0; return G; }
@@ -86,18 +113,25 @@ __host__ __device__ inline Group make_group(const Layout& l, int g) {
   return G;
 }
 
-// Per-(b, h) tile enumeration over groups: tile t of `rows`-row tiles.
+// Group at position i of the schedule order (context groups first).
+__host__ __device__ inline int sched_group(const Layout& l, int i) {
+  return i < 2 ? l.J() + 2 + i : i - 2;
+}
+
+// Per-(b, h) tile enumeration over groups in schedule order: tile t of
+// `rows`-row tiles.
 __host__ __device__ inline int tiles_per_head(const Layout& l, int rows) {
   int n = 0;
-  for (int g = 0; g < l.groups(); ++g) {
-    Group G = make_group(l, g);
+  for (int i = 0; i < l.groups(); ++i) {
+    Group G = make_group(l, sched_group(l, i));
     n += (G.nq + rows - 1) / rows;
   }
   return n;
 }
 
 __host__ __device__ inline void tile_to_group(const Layout& l, int rows, int t, int& g, int& r0) {
-  for (g = 0; g < l.groups(); ++g) {
+  for (int i = 0; i < l.groups(); ++i) {
+    g = sched_group(l, i);
     Group G = make_group(l, g);
     int n = (G.nq + rows - 1) / rows;
     if (t < n) { r0 = G.q0 + t * rows; return; }
@@ -108,32 +142,33 @@ __host__ __device__ inline void tile_to_group(const Layout& l, int rows, int t, 
 }
 
 // Key tile t of a query group (tiles of `keys` keys): video segments first,
-// then the text keys.
+// then the text keys, then the audio keys.
+enum KeySource { kKVideo = 0, kKText = 1, kKAudio = 2 };
 struct KeyTile {
-  int text;   // 1: rows index the text tensor
+  int src;    // KeySource: which tensor the rows index
   int row;    // first key row of the tile
   int valid;  // keys of the tile that belong to the segment (<= keys)
 };
 
 // (The loops below run over the at most 3 video segments with compile-time
 // indices, so a Group stays in registers on the device.)
-__host__ __device__ inline int key_tile_count(const Group& G, int T, int keys) {
+__host__ __device__ inline int key_tile_count(const Group& G, int T, int A, int keys) {
   int n = 0;
 #pragma unroll
   for (int s = 0; s < 3; ++s)
     if (s < G.nseg) n += (G.segn[s] + keys - 1) / keys;
-  return n + (T + keys - 1) / keys;
+  return n + (T + keys - 1) / keys + (A + keys - 1) / keys;
 }
 
-__host__ __device__ inline KeyTile key_tile(const Group& G, int T, int t, int keys) {
-  KeyTile k{1, 0, 0};
+__host__ __device__ inline KeyTile key_tile(const Group& G, int T, int A, int t, int keys) {
+  KeyTile k{kKText, 0, 0};
   bool found = false;
   int first = 0;  // first tile index of segment s
 #pragma unroll
   for (int s = 0; s < 3; ++s) {
     const int n = (s < G.nseg) ? (G.segn[s] + keys - 1) / keys : 0;
     if (!found && t < first + n) {
-      k.text = 0;
+      k.src = kKVideo;
       k.row = G.seg0[s] + (t - first) * keys;
       k.valid = G.segn[s] - (t - first) * keys;
       found = true;
@@ -141,8 +176,15 @@ __host__ __device__ inline KeyTile key_tile(const Group& G, int T, int t, int ke
     first += n;
   }
   if (!found) {
-    k.row = (t - first) * keys;
-    k.valid = T - (t - first) * keys;
+    const int nt = (T + keys - 1) / keys;
+    if (t < first + nt) {
+      k.row = (t - first) * keys;
+      k.valid = T - (t - first) * keys;
+    } else {
+      k.src = kKAudio;
+      k.row = (t - first - nt) * keys;
+      k.valid = A - (t - first - nt) * keys;
+    }
   }
   if (k.valid > keys) k.valid = keys;
   return k;
@@ -171,24 +213,38 @@ template <> __device__ inline __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { r
 // ---------------------------------------------------------------- launchers
 // Each returns cudaGetLastError() after its launch(es).
 
+// Audio keys and the context query rows of a joint layer (all null / unused
+// when l.A == 0 and l.ctx == 0). Tensors [B, A, H, d] / [B, T, H, d] in the io
+// dtype; the context outputs are written in the io dtype.
+struct JointArgs {
+  const void* k_audio = nullptr;
+  const void* v_audio = nullptr;
+  const void* q_text = nullptr;
+  const void* q_audio = nullptr;
+  void* o_text = nullptr;
+  void* o_audio = nullptr;
+  float* lse_text = nullptr;   // [B, T, H], nullable
+  float* lse_audio = nullptr;  // [B, A, H], nullable
+};
+
 // SIMT window softmax (any supported dtype/d); o_soft in the io dtype, or in
 // float32 when out_f32 (the hybrid path's intermediate).
 cudaError_t launch_window_simt(const Layout& l, int dtype, const void* q, const void* k,
                                const void* v, const void* kt, const void* vt, void* o,
-                               bool out_f32, float* lse, cudaStream_t st);
+                               bool out_f32, float* lse, const JointArgs& ja, cudaStream_t st);
 // tcgen05 window softmax (bf16, d in {64, 128}).
 bool window_tc_supported(const Layout& l, int dtype);
 cudaError_t launch_window_tc(const Layout& l, const void* q, const void* k, const void* v,
                              const void* kt, const void* vt, void* o, bool out_f32, float* lse,
-                             cudaStream_t st);
+                             const JointArgs& ja, cudaStream_t st);
 
 // tcgen05 window softmax with the hybrid epilogue fused (bf16, d in {64, 128}):
 // needs the chunk read states first; writes out (and optionally the two gated
-// branches) directly.
+// branches) directly; context query rows (if any) get the plain epilogue.
 cudaError_t launch_hybrid_tc(const Layout& l, const void* q, const void* k, const void* v,
                              const void* kt, const void* vt, const float* states, const void* gs,
                              const void* gl, const float* rms_w, float eps, void* out,
-                             void* out_soft, void* out_lin, cudaStream_t st);
+                             void* out_soft, void* out_lin, const JointArgs& ja, cudaStream_t st);
 
 // Reads and clears the device status word of the tcgen05 kernels' translation
 // unit (bounded waits record VDN_ERR_TIMEOUT there).

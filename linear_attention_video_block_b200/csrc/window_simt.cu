@@ -3,8 +3,10 @@
 // Used for float32 tensors (the tcgen05 kernel in window_tc.cu takes bf16).
 // One CTA = 64 query rows of one query group of one (b, h); it walks the
 // group's key segments (merged window + anchor frame intervals, then the text
-// keys) in 64-key tiles with an online softmax (project page "Local Softmax and
-// Long-Range Linear Memory": one normaliser over window, anchors and text).
+// keys, then the audio keys of a joint layer) in 64-key tiles with an online
+// softmax (project page "Local Softmax and Long-Range Linear Memory": one
+// normaliser over window, anchors and text). The context query rows of a joint
+// layer (text, audio) are groups whose key set is every token.
 #include <type_traits>
 
 #include "vdn_internal.cuh"
@@ -24,11 +26,25 @@ struct SimtSmem {
   float p[BQ][BK + 1];
 };
 
+// Joint-layer tensors in the io dtype (null when absent).
+template <typename T>
+struct SimtJoint {
+  const T* ka;
+  const T* va;
+  const T* qt;
+  const T* qa;
+  T* ot;
+  T* oa;
+  float* lse_t;
+  float* lse_a;
+};
+
 template <typename T, typename TO, int D>
 __global__ void __launch_bounds__(NT)
 window_simt_kernel(Layout l, const T* __restrict__ q, const T* __restrict__ k,
                    const T* __restrict__ v, const T* __restrict__ kt,
-                   const T* __restrict__ vt, TO* __restrict__ o, float* __restrict__ lse) {
+                   const T* __restrict__ vt, TO* __restrict__ o, float* __restrict__ lse,
+                   const SimtJoint<T> jn) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SimtSmem<D>& sm = *reinterpret_cast<SimtSmem<D>*>(smem_raw);
   const int tid = threadIdx.x;
@@ -40,11 +56,16 @@ window_simt_kernel(Layout l, const T* __restrict__ q, const T* __restrict__ k,
   const int rows_valid = min(BQ, G.q0 + G.nq - r0);
   const long long L = l.L();
   const long long HD = (long long)l.H * D;
-  const T* qb = q + ((long long)b * L) * HD + (long long)h * D;
+  // rows of the query's own tensor: video L, text T, audio A
+  const long long qrows = G.qsrc == kQVideo ? L : (G.qsrc == kQText ? l.T : l.A);
+  const T* qsrc = G.qsrc == kQVideo ? q : (G.qsrc == kQText ? jn.qt : jn.qa);
+  const T* qb = qsrc + ((long long)b * qrows) * HD + (long long)h * D;
   const T* kb = k + ((long long)b * L) * HD + (long long)h * D;
   const T* vb = v + ((long long)b * L) * HD + (long long)h * D;
   const T* ktb = kt ? kt + ((long long)b * l.T) * HD + (long long)h * D : nullptr;
   const T* vtb = vt ? vt + ((long long)b * l.T) * HD + (long long)h * D : nullptr;
+  const T* kab = jn.ka ? jn.ka + ((long long)b * l.A) * HD + (long long)h * D : nullptr;
+  const T* vab = jn.va ? jn.va + ((long long)b * l.A) * HD + (long long)h * D : nullptr;
 
   for (int i = tid; i < BQ * D; i += NT) {
     int r = i / D, cidx = i % D;
@@ -61,13 +82,14 @@ window_simt_kernel(Layout l, const T* __restrict__ q, const T* __restrict__ k,
   float m_run = -INFINITY, l_run = 0.f;
   const float scale = rsqrtf((float)D);
 
-  const int nseg = G.nseg + (l.T > 0 ? 1 : 0);
-  for (int s = 0; s < nseg; ++s) {
-    const bool text = (s == G.nseg);
-    const int seg_start = text ? 0 : G.seg0[s];
-    const int seg_len = text ? l.T : G.segn[s];
-    const T* ks = text ? ktb : kb;
-    const T* vs = text ? vtb : vb;
+  // segments: the group's video segments, then the text, then the audio
+  for (int s = 0; s < G.nseg + 2; ++s) {
+    const bool text = (s == G.nseg), audio = (s == G.nseg + 1);
+    const int seg_start = (text || audio) ? 0 : G.seg0[s];
+    const int seg_len = text ? l.T : (audio ? l.A : G.segn[s]);
+    if (seg_len == 0) continue;
+    const T* ks = text ? ktb : (audio ? kab : kb);
+    const T* vs = text ? vtb : (audio ? vab : vb);
     for (int k0 = 0; k0 < seg_len; k0 += BK) {
       const int kv = min(BK, seg_len - k0);
       __syncthreads();
@@ -142,18 +164,30 @@ window_simt_kernel(Layout l, const T* __restrict__ q, const T* __restrict__ k,
   }
   if (orow < rows_valid) {
     const float inv = 1.f / l_run;
-    TO* orow_ptr = o + ((long long)b * L + r0 + orow) * HD + (long long)h * D + ocg * OC;
+    const long long rix = (long long)b * qrows + r0 + orow;
+    if (G.qsrc == kQVideo) {
+      TO* orow_ptr = o + rix * HD + (long long)h * D + ocg * OC;
 #pragma unroll
-    for (int i = 0; i < OC; ++i) orow_ptr[i] = from_f32<TO>(acc[i] * inv);
-    if (lse && ocg == 0) lse[((long long)b * L + r0 + orow) * l.H + h] = m_run + logf(l_run);
+      for (int i = 0; i < OC; ++i) orow_ptr[i] = from_f32<TO>(acc[i] * inv);
+      if (lse && ocg == 0) lse[rix * l.H + h] = m_run + logf(l_run);
+    } else {
+      T* orow_ptr = (G.qsrc == kQText ? jn.ot : jn.oa) + rix * HD + (long long)h * D + ocg * OC;
+#pragma unroll
+      for (int i = 0; i < OC; ++i) orow_ptr[i] = from_f32<T>(acc[i] * inv);
+      float* lp = G.qsrc == kQText ? jn.lse_t : jn.lse_a;
+      if (lp && ocg == 0) lp[rix * l.H + h] = m_run + logf(l_run);
+    }
   }
 }
 
 template <typename T, int D>
 cudaError_t launch_simt_t(const Layout& l, const void* q, const void* k, const void* v,
                           const void* kt, const void* vt, void* o, bool out_f32, float* lse,
-                          cudaStream_t st) {
+                          const JointArgs& ja, cudaStream_t st) {
   if (!out_f32 && std::is_same<T, float>::value) out_f32 = true;
+  const SimtJoint<T> jn{(const T*)ja.k_audio, (const T*)ja.v_audio, (const T*)ja.q_text,
+                        (const T*)ja.q_audio, (T*)ja.o_text, (T*)ja.o_audio, ja.lse_text,
+                        ja.lse_audio};
   const int smem = (int)sizeof(SimtSmem<D>);
   dim3 grid(tiles_per_head(l, BQ), l.H, l.B);
   if (grid.x == 0) return cudaSuccess;
@@ -162,14 +196,14 @@ cudaError_t launch_simt_t(const Layout& l, const void* q, const void* k, const v
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, NT, smem, st>>>(l, (const T*)q, (const T*)k, (const T*)v, (const T*)kt,
-                                 (const T*)vt, (float*)o, lse);
+                                 (const T*)vt, (float*)o, lse, jn);
     return cudaGetLastError();
   }
   auto kern = window_simt_kernel<T, T, D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, NT, smem, st>>>(l, (const T*)q, (const T*)k, (const T*)v, (const T*)kt,
-                               (const T*)vt, (T*)o, lse);
+                               (const T*)vt, (T*)o, lse, jn);
   return cudaGetLastError();
 }
 
@@ -177,18 +211,18 @@ cudaError_t launch_simt_t(const Layout& l, const void* q, const void* k, const v
 
 cudaError_t launch_window_simt(const Layout& l, int dtype, const void* q, const void* k,
                                const void* v, const void* kt, const void* vt, void* o,
-                               bool out_f32, float* lse, cudaStream_t st) {
+                               bool out_f32, float* lse, const JointArgs& ja, cudaStream_t st) {
   if (dtype == VDN_F32) {
     switch (l.d) {
-      case 16: return launch_simt_t<float, 16>(l, q, k, v, kt, vt, o, out_f32, lse, st);
-      case 32: return launch_simt_t<float, 32>(l, q, k, v, kt, vt, o, out_f32, lse, st);
-      case 64: return launch_simt_t<float, 64>(l, q, k, v, kt, vt, o, out_f32, lse, st);
-      case 128: return launch_simt_t<float, 128>(l, q, k, v, kt, vt, o, out_f32, lse, st);
+      case 16: return launch_simt_t<float, 16>(l, q, k, v, kt, vt, o, out_f32, lse, ja, st);
+      case 32: return launch_simt_t<float, 32>(l, q, k, v, kt, vt, o, out_f32, lse, ja, st);
+      case 64: return launch_simt_t<float, 64>(l, q, k, v, kt, vt, o, out_f32, lse, ja, st);
+      case 128: return launch_simt_t<float, 128>(l, q, k, v, kt, vt, o, out_f32, lse, ja, st);
     }
   } else {
     switch (l.d) {
-      case 64: return launch_simt_t<__nv_bfloat16, 64>(l, q, k, v, kt, vt, o, out_f32, lse, st);
-      case 128: return launch_simt_t<__nv_bfloat16, 128>(l, q, k, v, kt, vt, o, out_f32, lse, st);
+      case 64: return launch_simt_t<__nv_bfloat16, 64>(l, q, k, v, kt, vt, o, out_f32, lse, ja, st);
+      case 128: return launch_simt_t<__nv_bfloat16, 128>(l, q, k, v, kt, vt, o, out_f32, lse, ja, st);
     }
   }
   return cudaErrorInvalidValue;

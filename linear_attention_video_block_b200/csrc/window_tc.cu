@@ -4,10 +4,14 @@
 //
 // What it computes (project page "Local Softmax and Long-Range Linear Memory"):
 // for every video query, softmax(q K^T / sqrt(d)) V over the keys of its
-// chunk window, the boundary anchor frames and all text tokens, one
-// normaliser. Keys are visited per query group as merged token segments
-// (window/anchor intervals, then text) in 128-key tiles; only the last tile of
-// each segment is partially masked.
+// chunk window, the boundary anchor frames and all text tokens (and, in a
+// joint text-video-audio layer, all audio tokens), one normaliser. Keys are
+// visited per query group as merged token segments (window/anchor intervals,
+// then text, then audio) in 128-key tiles; only the last tile of each segment
+// is partially masked. In a joint layer the text and audio query rows are
+// extra groups of the same grid whose key set is every token (the dense
+// softmax the pages keep for interactions involving text or audio); they are
+// scheduled first, being the longest, and always take the plain epilogue.
 //
 // CTA = 256 query rows (two 128-row Q tiles) of one query group of one
 // (b, h); 320 threads (at most 200 registers each):
@@ -91,6 +95,14 @@ __device__ __forceinline__ bool mbar_wait(unsigned long long* bar, uint32_t pari
 
 // ------------------------------------------------------------------ kernel
 
+// Outputs of the context query rows (joint layer), io dtype [B, T|A, H, D].
+struct CtxOut {
+  __nv_bfloat16* o_text;
+  __nv_bfloat16* o_audio;
+  float* lse_text;
+  float* lse_audio;
+};
+
 // Extra arguments of the fused hybrid epilogue.
 struct HybridArgs {
   const float* states;             // [B, H, 2, J, D, D] fp32 chunk read states
@@ -138,8 +150,10 @@ template <int D, bool kFuse>
 __global__ void __launch_bounds__(kThreads, 1)
 window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kt,
-                 const __grid_constant__ CUtensorMap tm_vt, const Layout l, void* out, int out_f32,
-                 float* lse, const HybridArgs hy) {
+                 const __grid_constant__ CUtensorMap tm_vt, const __grid_constant__ CUtensorMap tm_ka,
+                 const __grid_constant__ CUtensorMap tm_va, const __grid_constant__ CUtensorMap tm_qt,
+                 const __grid_constant__ CUtensorMap tm_qa, const Layout l, void* out, int out_f32,
+                 float* lse, const HybridArgs hy, const CtxOut cx) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -155,8 +169,9 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   int g, r0;
   tile_to_group(l, 2 * kRows, blockIdx.x, g, r0);
   const Group G = make_group(l, g < 0 ? 0 : g);
-  const int n_tiles = key_tile_count(G, l.T, kRows);
+  const int n_tiles = key_tile_count(G, l.T, l.A, kRows);
   const bool has_lin = kFuse && G.chunk >= 0;
+  const bool ctx_rows = G.qsrc != kQVideo;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -220,15 +235,16 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     if (lane == 0 && !*abort) {
       // ------------------------------------------------------- TMA producer
+      const CUtensorMap* mq = G.qsrc == kQVideo ? &tm_q : (G.qsrc == kQText ? &tm_qt : &tm_qa);
       mbar_expect_tx(&bars->q_full, 2 * C::kTileBytes);
       for (int qt = 0; qt < 2; ++qt)
         for (int hf = 0; hf < C::kHalves; ++hf)
-          tma_load_4d(sQ + qt * C::kTileBytes + hf * C::kHalfBytes, &tm_q, &bars->q_full, hf * 64,
+          tma_load_4d(sQ + qt * C::kTileBytes + hf * C::kHalfBytes, mq, &bars->q_full, hf * 64,
                       h, r0 + qt * kRows, b);
       int fill = 0;
       bool ok = true;
       for (int t = 0; t < n_tiles && ok; ++t) {
-        const KeyTile kt = key_tile(G, l.T, t, kRows);
+        const KeyTile kt = key_tile(G, l.T, l.A, t, kRows);
         for (int kv = 0; kv < 2; ++kv, ++fill) {
           const int slot = fill % C::kSlots;
           const int use = fill / C::kSlots;
@@ -236,7 +252,9 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             ok = false;
             break;
           }
-          const CUtensorMap* map = kt.text ? (kv ? &tm_vt : &tm_kt) : (kv ? &tm_v : &tm_k);
+          const CUtensorMap* map = kt.src == kKVideo ? (kv ? &tm_v : &tm_k)
+                                   : kt.src == kKText ? (kv ? &tm_vt : &tm_kt)
+                                                      : (kv ? &tm_va : &tm_ka);
           mbar_expect_tx(&bars->kv_full[slot], C::kTileBytes);
           for (int hf = 0; hf < C::kHalves; ++hf)
             tma_load_4d(sKV + slot * C::kTileBytes + hf * C::kHalfBytes, map, &bars->kv_full[slot],
@@ -364,14 +382,15 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     float m = -INFINITY, lsum = 0.f;
     bool ok = !*abort;
     // The only partially valid key tiles are the last tile of each segment
-    // (3 video segments at most, then the text): (tile index << 8) | valid
-    // count for each (valid <= 128 fits in 8 bits; -1 when a segment is empty).
-    int edge[4];
+    // (3 video segments at most, then the text, then the audio): (tile index
+    // << 8) | valid count for each (valid <= 128 fits in 8 bits; -1 when a
+    // segment is empty).
+    int edge[5];
     {
       int first = 0;
 #pragma unroll
-      for (int sgi = 0; sgi < 4; ++sgi) {
-        const int len = (sgi < 3) ? ((sgi < G.nseg) ? G.segn[sgi] : 0) : l.T;
+      for (int sgi = 0; sgi < 5; ++sgi) {
+        const int len = (sgi < 3) ? ((sgi < G.nseg) ? G.segn[sgi] : 0) : (sgi == 3 ? l.T : l.A);
         const int n = (len + kRows - 1) / kRows;
         edge[sgi] = (n > 0) ? (((first + n - 1) << 8) | (len - (n - 1) * kRows)) : -1;
         first += n;
@@ -390,7 +409,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       float* s = reinterpret_cast<float*>(sr);
       int valid = kRows;
 #pragma unroll
-      for (int sgi = 0; sgi < 4; ++sgi)
+      for (int sgi = 0; sgi < 5; ++sgi)
         if (edge[sgi] >= 0 && (edge[sgi] >> 8) == t) valid = edge[sgi] & 255;
       if (valid < kRows) {
 #pragma unroll
@@ -465,21 +484,32 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const int grow = r0 + kRows * w + row;
       const bool store = grow < q_end;
       const float inv = 1.f / lsum;
-      const long long base = (((long long)b * l.L() + grow) * l.H + h) * D;
-      if constexpr (!kFuse) {
+      // rows of the query's own tensor: video [B, L, H, D], text [B, T, H, D],
+      // audio [B, A, H, D]
+      const long long qrows = G.qsrc == kQVideo ? l.L() : (G.qsrc == kQText ? l.T : l.A);
+      const long long base = (((long long)b * qrows + grow) * l.H + h) * D;
+      if (!kFuse || ctx_rows) {
+        void* dst_o = out;
+        float* dst_lse = lse;
+        bool f32 = out_f32 != 0;
+        if (ctx_rows) {
+          dst_o = G.qsrc == kQText ? cx.o_text : cx.o_audio;
+          dst_lse = G.qsrc == kQText ? cx.lse_text : cx.lse_audio;
+          f32 = false;
+        }
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t o[32];
           tmem_ld_x32(tO + c0, o);
           if (store) {
-            if (out_f32) {
-              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + base + c0);
+            if (f32) {
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(dst_o) + base + c0);
 #pragma unroll
               for (int i = 0; i < 8; ++i)
                 dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
                                      __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
             } else {
-              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + base + c0);
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dst_o) + base + c0);
 #pragma unroll
               for (int i = 0; i < 4; ++i)
                 dst[i] = make_uint4(pack_bf16(__uint_as_float(o[8 * i]) * inv, __uint_as_float(o[8 * i + 1]) * inv),
@@ -489,7 +519,8 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
           }
         }
-        if (store && lse) lse[((long long)b * l.L() + grow) * l.H + h] = (m + log2f(lsum)) * 0.6931471805599453f;
+        if (store && dst_lse)
+          dst_lse[((long long)b * qrows + grow) * l.H + h] = (m + log2f(lsum)) * 0.6931471805599453f;
       } else {
         // RMSNorm statistic of o_lin (whole row in this thread)
         float rstd = 0.f;
@@ -569,26 +600,33 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 template <int D, bool kFuse>
 cudaError_t launch_tc_t(const Layout& l, const void* q, const void* k, const void* v,
                         const void* kt, const void* vt, void* o, bool out_f32, float* lse,
-                        const HybridArgs& hy, cudaStream_t st) {
-  CUtensorMap mq, mk, mv, mkt, mvt;
+                        const HybridArgs& hy, const JointArgs& ja, cudaStream_t st) {
+  CUtensorMap mq, mk, mv, mkt, mvt, mka, mva, mqt, mqa;
   const long long L = l.L();
   if (!make_map(&mq, q, D, l.H, L, l.B) || !make_map(&mk, k, D, l.H, L, l.B) ||
       !make_map(&mv, v, D, l.H, L, l.B))
     return cudaErrorInvalidValue;
-  if (l.T > 0) {
-    if (!make_map(&mkt, kt, D, l.H, l.T, l.B) || !make_map(&mvt, vt, D, l.H, l.T, l.B))
-      return cudaErrorInvalidValue;
-  } else {
-    mkt = mk;  // never read: no text tiles
-    mvt = mv;
-  }
+  // maps of absent tensors are copies that are never read (no tiles use them)
+  mkt = mk; mvt = mv; mka = mk; mva = mv; mqt = mq; mqa = mq;
+  if (l.T > 0 && (!make_map(&mkt, kt, D, l.H, l.T, l.B) || !make_map(&mvt, vt, D, l.H, l.T, l.B)))
+    return cudaErrorInvalidValue;
+  if (l.A > 0 && (!make_map(&mka, ja.k_audio, D, l.H, l.A, l.B) ||
+                  !make_map(&mva, ja.v_audio, D, l.H, l.A, l.B)))
+    return cudaErrorInvalidValue;
+  if ((l.ctx & kCtxText) && l.T > 0 && !make_map(&mqt, ja.q_text, D, l.H, l.T, l.B))
+    return cudaErrorInvalidValue;
+  if ((l.ctx & kCtxAudio) && l.A > 0 && !make_map(&mqa, ja.q_audio, D, l.H, l.A, l.B))
+    return cudaErrorInvalidValue;
+  const CtxOut cx{static_cast<__nv_bfloat16*>(ja.o_text), static_cast<__nv_bfloat16*>(ja.o_audio),
+                  ja.lse_text, ja.lse_audio};
   auto kern = window_tc_kernel<D, kFuse>;
   const int smem = Cfg<D>::kSmemBytes - (kFuse ? 0 : Cfg<D>::kSsumBytes);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(tiles_per_head(l, 2 * kRows), l.H, l.B);
   if (grid.x == 0) return cudaSuccess;
-  kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, mkt, mvt, l, o, out_f32 ? 1 : 0, lse, hy);
+  kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, mkt, mvt, mka, mva, mqt, mqa, l, o, out_f32 ? 1 : 0,
+                                     lse, hy, cx);
   return cudaGetLastError();
 }
 
@@ -600,17 +638,17 @@ bool window_tc_supported(const Layout& l, int dtype) {
 
 cudaError_t launch_window_tc(const Layout& l, const void* q, const void* k, const void* v,
                              const void* kt, const void* vt, void* o, bool out_f32, float* lse,
-                             cudaStream_t st) {
+                             const JointArgs& ja, cudaStream_t st) {
   HybridArgs hy{};
-  if (l.d == 128) return launch_tc_t<128, false>(l, q, k, v, kt, vt, o, out_f32, lse, hy, st);
-  if (l.d == 64) return launch_tc_t<64, false>(l, q, k, v, kt, vt, o, out_f32, lse, hy, st);
+  if (l.d == 128) return launch_tc_t<128, false>(l, q, k, v, kt, vt, o, out_f32, lse, hy, ja, st);
+  if (l.d == 64) return launch_tc_t<64, false>(l, q, k, v, kt, vt, o, out_f32, lse, hy, ja, st);
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_hybrid_tc(const Layout& l, const void* q, const void* k, const void* v,
                              const void* kt, const void* vt, const float* states, const void* gs,
                              const void* gl, const float* rms_w, float eps, void* out,
-                             void* out_soft, void* out_lin, cudaStream_t st) {
+                             void* out_soft, void* out_lin, const JointArgs& ja, cudaStream_t st) {
   HybridArgs hy;
   hy.states = states;
   hy.g_soft = static_cast<const __nv_bfloat16*>(gs);
@@ -620,8 +658,8 @@ cudaError_t launch_hybrid_tc(const Layout& l, const void* q, const void* k, cons
   hy.out = static_cast<__nv_bfloat16*>(out);
   hy.out_soft = static_cast<__nv_bfloat16*>(out_soft);
   hy.out_lin = static_cast<__nv_bfloat16*>(out_lin);
-  if (l.d == 128) return launch_tc_t<128, true>(l, q, k, v, kt, vt, nullptr, false, nullptr, hy, st);
-  if (l.d == 64) return launch_tc_t<64, true>(l, q, k, v, kt, vt, nullptr, false, nullptr, hy, st);
+  if (l.d == 128) return launch_tc_t<128, true>(l, q, k, v, kt, vt, nullptr, false, nullptr, hy, ja, st);
+  if (l.d == 64) return launch_tc_t<64, true>(l, q, k, v, kt, vt, nullptr, false, nullptr, hy, ja, st);
   return cudaErrorInvalidValue;
 }
 

@@ -6,9 +6,11 @@ CPU fallback: the functions raise if the library or a CUDA device is missing.
 
 Public calls (same names as the C ABI, without the ``vdn_`` prefix):
   window_softmax_fwd, vda_scan_fwd, hybrid_attn_fwd, workspace_bytes,
-  device_status, vda_scan_fwd_noalloc. vda_scan_fwd and hybrid_attn_fwd take an
-  optional ``alpha`` [B, F, H, d] float32 (KDA channel decay); when given they
-  call the ``_decay`` entry points.
+  device_status, vda_scan_fwd_noalloc, joint_softmax_fwd, joint_attn_fwd.
+vda_scan_fwd and hybrid_attn_fwd take an optional ``alpha`` [B, F, H, d]
+float32 (KDA channel decay); when given they call the ``_decay`` entry points.
+The joint_* calls add the audio keys and the dense text/audio query rows of a
+joint text-video-audio layer (the C ABI's vdn_context_t).
 Tensors follow the C ABI's layout: q/k/v/gates/outputs [B, L, H, d],
 text k/v [B, T, H, d], beta [B, L, H] and beta_text [B, T, H] in float32.
 """
@@ -30,7 +32,8 @@ STATUS = {0: "VDN_OK", 1: "VDN_ERR_INVALID", 2: "VDN_ERR_UNSUPPORTED",
           3: "VDN_ERR_WORKSPACE", 4: "VDN_ERR_CUDA", 5: "VDN_ERR_TIMEOUT"}
 EXPORTS = ("vdn_workspace_bytes", "vdn_window_softmax_fwd", "vdn_vda_scan_fwd",
            "vdn_vda_scan_fwd_decay", "vdn_hybrid_attn_fwd", "vdn_hybrid_attn_fwd_decay",
-           "vdn_vda_scan_fwd_noalloc", "vdn_device_status", "vdn_status_string")
+           "vdn_vda_scan_fwd_noalloc", "vdn_joint_softmax_fwd", "vdn_joint_attn_fwd",
+           "vdn_device_status", "vdn_status_string")
 
 
 class VdnError(RuntimeError):
@@ -42,6 +45,11 @@ class VdnError(RuntimeError):
 
 class _CLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in ("B", "F", "N", "T", "c", "H", "d")]
+
+
+class _CContext(ctypes.Structure):
+    _fields_ = [("A", ctypes.c_int)] + [(n, ctypes.c_void_p) for n in (
+        "k_audio", "v_audio", "q_text", "q_audio", "o_text", "o_audio", "lse_text", "lse_audio")]
 
 
 def lib():
@@ -67,6 +75,12 @@ def lib():
         L.vdn_hybrid_attn_fwd_decay.argtypes = ([LP, I] + [P] * 10 + [P, ctypes.c_float]
                                                 + [P] * 3 + [P, S, P])
         L.vdn_hybrid_attn_fwd_decay.restype = I
+        CP = ctypes.POINTER(_CContext)
+        L.vdn_joint_softmax_fwd.argtypes = [LP, I, CP] + [P] * 8
+        L.vdn_joint_softmax_fwd.restype = I
+        L.vdn_joint_attn_fwd.argtypes = ([LP, I, CP] + [P] * 10 + [P, ctypes.c_float]
+                                         + [P] * 3 + [P, S, P])
+        L.vdn_joint_attn_fwd.restype = I
         L.vdn_vda_scan_fwd_noalloc.argtypes = [LP, I] + [P] * 10
         L.vdn_vda_scan_fwd_noalloc.restype = I
         L.vdn_device_status.argtypes = []
@@ -224,3 +238,67 @@ def vda_scan_fwd_noalloc(layout: Layout, q, k, v, k_text, v_text, beta, beta_tex
 def device_status() -> int:
     """Reads and clears libvdn's device status word (synchronises the device)."""
     return int(lib().vdn_device_status())
+
+
+def _context(k_audio, v_audio, q_text, q_audio, o_text, o_audio, lse_text=None, lse_audio=None):
+    A = 0 if k_audio is None else int(k_audio.shape[1])
+    return _CContext(A, _ptr(k_audio), _ptr(v_audio), _ptr(q_text), _ptr(q_audio), _ptr(o_text),
+                     _ptr(o_audio), _ptr(lse_text), _ptr(lse_audio))
+
+
+def _context_outputs(q_text, q_audio, o_text, o_audio, want_lse):
+    if q_text is not None and o_text is None:
+        o_text = torch.empty_like(q_text)
+    if q_audio is not None and o_audio is None:
+        o_audio = torch.empty_like(q_audio)
+    lt = la = None
+    if want_lse:
+        if q_text is not None:
+            lt = torch.empty(q_text.shape[:3], dtype=torch.float32, device=q_text.device)
+        if q_audio is not None:
+            la = torch.empty(q_audio.shape[:3], dtype=torch.float32, device=q_audio.device)
+    return o_text, o_audio, lt, la
+
+
+def joint_softmax_fwd(layout: Layout, q, k, v, k_text, v_text, k_audio=None, v_audio=None,
+                      q_text=None, q_audio=None, o_soft=None, o_text=None, o_audio=None,
+                      want_lse=False):
+    """Softmax part of a joint text-video-audio layer. Returns a dict with
+    o_soft (video rows; their key sets include the audio keys), o_text and
+    o_audio (dense context query rows, None when not asked for) and, with
+    want_lse, lse / lse_text / lse_audio."""
+    _require_cuda()
+    if o_soft is None:
+        o_soft = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if want_lse else None
+    o_text, o_audio, lt, la = _context_outputs(q_text, q_audio, o_text, o_audio, want_lse)
+    cx = _context(k_audio, v_audio, q_text, q_audio, o_text, o_audio, lt, la)
+    code = lib().vdn_joint_softmax_fwd(
+        ctypes.byref(_clayout(layout)), _dtype_code(q), ctypes.byref(cx), _ptr(q), _ptr(k), _ptr(v),
+        _ptr(k_text), _ptr(v_text), _ptr(o_soft), _ptr(lse), _stream(q.device))
+    _check(code, "vdn_joint_softmax_fwd")
+    return {"o_soft": o_soft, "o_text": o_text, "o_audio": o_audio, "lse": lse,
+            "lse_text": lt, "lse_audio": la}
+
+
+def joint_attn_fwd(layout: Layout, q, k, v, k_text, v_text, beta, beta_text, g_soft, g_lin,
+                   k_audio=None, v_audio=None, q_text=None, q_audio=None, alpha=None,
+                   rms_weight=None, rms_eps=1e-6, out=None, o_text=None, o_audio=None,
+                   out_soft=None, out_lin=None, workspace=None):
+    """The attention of a joint text-video-audio layer: video rows get the
+    hybrid (softmax branch with the audio keys; KDA decay when alpha is given),
+    text/audio query rows the dense softmax. Returns (out, o_text, o_audio)."""
+    _require_cuda()
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = torch.empty(workspace_bytes(layout, q.dtype), dtype=torch.uint8, device=q.device)
+    o_text, o_audio, _, _ = _context_outputs(q_text, q_audio, o_text, o_audio, False)
+    cx = _context(k_audio, v_audio, q_text, q_audio, o_text, o_audio)
+    code = lib().vdn_joint_attn_fwd(
+        ctypes.byref(_clayout(layout)), _dtype_code(q), ctypes.byref(cx), _ptr(q), _ptr(k), _ptr(v),
+        _ptr(k_text), _ptr(v_text), _ptr(beta), _ptr(beta_text), _ptr(alpha), _ptr(g_soft),
+        _ptr(g_lin), _ptr(rms_weight), ctypes.c_float(rms_eps), _ptr(out), _ptr(out_soft),
+        _ptr(out_lin), _ptr(workspace), workspace.numel(), _stream(q.device))
+    _check(code, "vdn_joint_attn_fwd")
+    return out, o_text, o_audio

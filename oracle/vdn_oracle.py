@@ -239,12 +239,14 @@ def context_rows(q_ctx, k, v, k_text, v_text, k_audio=None, v_audio=None, heads=
         for h in heads:
             keys = np.concatenate([k[b, :, h, :], k_text[b, :, h, :], k_audio[b, :, h, :]], axis=0)
             vals = np.concatenate([v[b, :, h, :], v_text[b, :, h, :], v_audio[b, :, h, :]], axis=0)
-            s = (q_ctx[b, :, h, :] @ keys.T) * scale
-            m = s.max(axis=1, keepdims=True)
-            p = np.exp(s - m)
-            z = p.sum(axis=1, keepdims=True)
-            out[b, :, h, :] = (p @ vals) / z
-            lse[b, :, h] = (m + np.log(z))[:, 0]
+            for r0 in range(0, R, 256):          # row blocks bound the score matrix
+                sl = slice(r0, min(R, r0 + 256))
+                s = (q_ctx[b, sl, h, :] @ keys.T) * scale
+                m = s.max(axis=1, keepdims=True)
+                p = np.exp(s - m)
+                z = p.sum(axis=1, keepdims=True)
+                out[b, sl, h, :] = (p @ vals) / z
+                lse[b, sl, h] = (m + np.log(z))[:, 0]
     return (out, lse) if return_lse else out
 
 

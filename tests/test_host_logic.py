@@ -113,6 +113,9 @@ def _parse(text, extras=None):
         if extras is not None and t[0] == "keytiles":
             extras.setdefault(t[0], {})[int(t[1])] = t[2:]
             continue
+        if t[0] == "qsrc":
+            groups[int(t[1])]["qsrc"] = int(t[2])
+            continue
         if t[0] == "extent":
             extent = (int(t[1]), int(t[2]), int(t[4]))
         elif t[0] == "group":
@@ -136,6 +139,7 @@ def test_cuda_schedule_matches_oracle_key_sets(schedule_dump, F, c):
     for G in groups:
         if G["nq"] == 0:
             continue
+        assert G["qsrc"] == 0          # no context rows without the joint bits
         frames = sorted({t // N for t in range(G["q0"], G["q0"] + G["nq"])})
         covered += list(range(G["q0"], G["q0"] + G["nq"]))
         key_tokens = set()
@@ -180,8 +184,8 @@ def test_key_tiles_cover_segments_exactly(schedule_dump, F, c, N, T):
         if G["nq"] == 0:
             continue
         tiles = [tuple(map(int, x.split(":"))) for x in extras["keytiles"][G["g"]]]
-        video = [(row, valid) for text, row, valid in tiles if text == 0]
-        text_tiles = [(row, valid) for text, row, valid in tiles if text == 1]
+        video = [(row, valid) for src, row, valid in tiles if src == 0]
+        text_tiles = [(row, valid) for src, row, valid in tiles if src == 1]
         keys = []
         for row, valid in video:
             assert 1 <= valid <= 128
@@ -190,3 +194,91 @@ def test_key_tiles_cover_segments_exactly(schedule_dump, F, c, N, T):
         assert len(keys) == len(set(keys))
         assert [v for _, v in text_tiles] == [1]  # the dump program uses one text token
 
+
+
+
+@pytest.mark.parametrize("F,c,N,T,A,ctx", [(7, 2, 70, 130, 203, 3), (36, 5, 100, 64, 1, 1),
+                                           (3, 1, 50, 0, 129, 2), (1, 3, 200, 7, 0, 3),
+                                           (12, 2, 1, 2, 5, 3)])
+def test_joint_schedule_context_groups_and_audio_tiles(schedule_dump, F, c, N, T, A, ctx):
+    """Joint layer: the text/audio query rows are groups scheduled before every
+    video group, each row in exactly one tile, with every video token as keys;
+    every group's key tiles are its video segments, then the text, then the
+    audio, each key once."""
+    rows = 4
+    r = subprocess.run([schedule_dump, str(F), str(N), str(c), str(rows), str(T), str(A), str(ctx)],
+                       check=True, capture_output=True, text=True)
+    extras = {}
+    (_, _, ntiles), groups, tiles = _parse(r.stdout, extras)
+    want_rows = {1: T if ctx & 1 else 0, 2: A if ctx & 2 else 0}
+    for src in (1, 2):
+        gs = [G for G in groups if G["qsrc"] == src]
+        assert len(gs) == 1 and gs[0]["nq"] == want_rows[src] and gs[0]["q0"] == 0
+        assert gs[0]["segs"] == [(0, F * N)] and gs[0]["chunk"] == -1
+    # schedule order: all context tiles come first, every row once
+    first_video = next(i for i, (g, _) in enumerate(tiles) if groups[g]["qsrc"] == 0)
+    assert all(groups[g]["qsrc"] != 0 for g, _ in tiles[:first_video])
+    assert all(groups[g]["qsrc"] == 0 for g, _ in tiles[first_video:])
+    for src in (1, 2):
+        seen = []
+        for g, r0 in tiles:
+            if groups[g]["qsrc"] == src:
+                seen += list(range(r0, min(r0 + rows, want_rows[src])))
+        assert sorted(seen) == list(range(want_rows[src]))
+    video_rows = []
+    for g, r0 in tiles:
+        G = groups[g]
+        if G["qsrc"] == 0:
+            video_rows += list(range(r0, min(r0 + rows, G["q0"] + G["nq"])))
+    assert sorted(video_rows) == list(range(F * N)) and len(tiles) == ntiles
+    for G in groups:
+        if G["nq"] == 0:
+            continue
+        kt = [tuple(map(int, x.split(":"))) for x in extras["keytiles"][G["g"]]]
+        srcs = [s for s, _, _ in kt]
+        assert srcs == sorted(srcs)     # video, then text, then audio
+        for src, n, segs in ((0, None, G["segs"]), (1, T, [(0, T)]), (2, A, [(0, A)])):
+            keys = []
+            for s, row, valid in kt:
+                if s == src:
+                    assert 1 <= valid <= 128
+                    keys += list(range(row, row + valid))
+            assert keys == [k for s0, sn in segs for k in range(s0, s0 + sn)]
+
+
+def _ctx(lib, **kw):
+    from linear_attention_video_block_b200 import vdn
+    base = dict(A=0, k_audio=None, v_audio=None, q_text=None, q_audio=None, o_text=None,
+                o_audio=None, lse_text=None, lse_audio=None)
+    base.update(kw)
+    return vdn._CContext(base["A"], *[base[k] for k in ("k_audio", "v_audio", "q_text", "q_audio",
+                                                         "o_text", "o_audio", "lse_text", "lse_audio")])
+
+
+def test_joint_entries_validate_context(lib):
+    """vdn_joint_softmax_fwd / vdn_joint_attn_fwd: the context struct is required;
+    audio tensors are required when A > 0, outputs with their query rows, every
+    given pointer 16-byte aligned (no GPU is touched by any of these)."""
+    ok = _layout()
+    js = lib.vdn_joint_softmax_fwd
+    args = [FAKE] * 6 + [None, None]
+    assert js(ctypes.byref(ok), 0, None, *args) == 1
+    assert js(ctypes.byref(ok), 0, ctypes.byref(_ctx(lib, A=-1)), *args) == 1
+    assert js(ctypes.byref(ok), 0, ctypes.byref(_ctx(lib, A=3)), *args) == 1            # no audio k/v
+    assert js(ctypes.byref(ok), 0, ctypes.byref(_ctx(lib, A=3, k_audio=FAKE, v_audio=MISALIGNED)),
+              *args) == 2
+    assert js(ctypes.byref(ok), 0, ctypes.byref(_ctx(lib, q_text=FAKE)), *args) == 1     # no o_text
+    assert js(ctypes.byref(ok), 0, ctypes.byref(_ctx(lib, q_text=FAKE, o_text=MISALIGNED)),
+              *args) == 2
+    assert js(ctypes.byref(ok), 0, ctypes.byref(_ctx(lib, A=2, k_audio=FAKE, v_audio=FAKE,
+                                                     q_audio=FAKE)), *args) == 1         # no o_audio
+    assert js(ctypes.byref(_layout(B=0)), 0, ctypes.byref(_ctx(lib)), *args) == 1
+    ja = lib.vdn_joint_attn_fwd
+    need = lib.vdn_workspace_bytes(ctypes.byref(ok), 0)
+    pre = [FAKE] * 7
+    post = [None, FAKE, FAKE, None, ctypes.c_float(1e-6), FAKE, None, None, FAKE]
+    assert ja(ctypes.byref(ok), 0, None, *pre, *post, need, None) == 1
+    assert ja(ctypes.byref(ok), 0, ctypes.byref(_ctx(lib, A=1)), *pre, *post, need, None) == 1
+    assert ja(ctypes.byref(ok), 0, ctypes.byref(_ctx(lib)), *pre, *post, need - 1, None) == 3
+    assert ja(ctypes.byref(ok), 0, ctypes.byref(_ctx(lib)), *pre, MISALIGNED, *post[1:], need,
+              None) == 2                                                                  # alpha
