@@ -245,6 +245,11 @@ int vdn_device_status(void);
 /* Static string for a status code. */
 const char* vdn_status_string(int status);
 
+/* The CUDA runtime's description of the error behind the last VDN_ERR_CUDA
+ * returned on the calling host thread (by any entry point except
+ * vdn_vda_scan_fwd_noalloc), or "no CUDA error". Static string. */
+const char* vdn_last_cuda_error(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -65,7 +65,14 @@ Workspace carve(const Layout& l, int dtype, void* base, bool need_states, bool n
   return w;
 }
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? VDN_OK : VDN_ERR_CUDA; }
+// The CUDA error behind the last VDN_ERR_CUDA returned on this host thread.
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return VDN_OK;
+  t_last_cuda_error = e;
+  return VDN_ERR_CUDA;
+}
 
 int run_window(const Layout& l, int dtype, const void* q, const void* k, const void* v,
                const void* kt, const void* vt, void* o, bool out_f32, float* lse,
@@ -281,14 +288,18 @@ int vdn_joint_attn_fwd(const vdn_layout_t* layout, int dtype, const vdn_context_
 }
 
 int vdn_device_status(void) {
-  if (cudaDeviceSynchronize() != cudaSuccess) return VDN_ERR_CUDA;
+  if (cuda_status(cudaDeviceSynchronize()) != VDN_OK) return VDN_ERR_CUDA;
   int s[3] = {0, 0, 0};
-  if (vdn::read_and_clear_tc_status(&s[0]) != cudaSuccess) return VDN_ERR_CUDA;
-  if (vdn::read_and_clear_gram_status(&s[1]) != cudaSuccess) return VDN_ERR_CUDA;
-  if (vdn::read_and_clear_readout_status(&s[2]) != cudaSuccess) return VDN_ERR_CUDA;
+  if (cuda_status(vdn::read_and_clear_tc_status(&s[0])) != VDN_OK) return VDN_ERR_CUDA;
+  if (cuda_status(vdn::read_and_clear_gram_status(&s[1])) != VDN_OK) return VDN_ERR_CUDA;
+  if (cuda_status(vdn::read_and_clear_readout_status(&s[2])) != VDN_OK) return VDN_ERR_CUDA;
   for (int i = 0; i < 3; ++i)
     if (s[i] != 0) return s[i];
   return VDN_OK;
+}
+
+const char* vdn_last_cuda_error(void) {
+  return t_last_cuda_error == cudaSuccess ? "no CUDA error" : cudaGetErrorString(t_last_cuda_error);
 }
 
 const char* vdn_status_string(int status) {

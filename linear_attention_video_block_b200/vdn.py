@@ -33,12 +33,14 @@ STATUS = {0: "VDN_OK", 1: "VDN_ERR_INVALID", 2: "VDN_ERR_UNSUPPORTED",
 EXPORTS = ("vdn_workspace_bytes", "vdn_window_softmax_fwd", "vdn_vda_scan_fwd",
            "vdn_vda_scan_fwd_decay", "vdn_hybrid_attn_fwd", "vdn_hybrid_attn_fwd_decay",
            "vdn_vda_scan_fwd_noalloc", "vdn_joint_softmax_fwd", "vdn_joint_attn_fwd",
-           "vdn_device_status", "vdn_status_string")
+           "vdn_device_status", "vdn_status_string", "vdn_last_cuda_error")
 
 
 class VdnError(RuntimeError):
     def __init__(self, code, where):
         msg = lib().vdn_status_string(code).decode() if _lib is not None else ""
+        if code == 4 and _lib is not None:
+            msg += ": " + lib().vdn_last_cuda_error().decode()
         super().__init__(f"{where}: {STATUS.get(code, code)} ({msg})")
         self.code = code
 
@@ -87,6 +89,8 @@ def lib():
         L.vdn_device_status.restype = I
         L.vdn_status_string.argtypes = [I]
         L.vdn_status_string.restype = ctypes.c_char_p
+        L.vdn_last_cuda_error.argtypes = []
+        L.vdn_last_cuda_error.restype = ctypes.c_char_p
         _lib = L
     return _lib
 

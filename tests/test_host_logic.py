@@ -39,6 +39,7 @@ def test_status_strings(lib):
     for code in range(6):
         assert lib.vdn_status_string(code)
     assert lib.vdn_status_string(99) == b"unknown status"
+    assert lib.vdn_last_cuda_error() == b"no CUDA error"
 
 
 def _layout(**kw):
