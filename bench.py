@@ -83,10 +83,9 @@ def joint_flops(lay, A) -> float:
 
 def launches_per_step(lay, dtype) -> int:
     """Kernels of one vdn_hybrid_attn_fwd call: gram, inverse, scan, zero-fill of
-    unused chunk entries, and the window softmax with the readout, norm and
-    gates fused (bf16, d in {64, 128}); the CUDA-core path adds a separate
-    readout/combine kernel."""
-    return 5 if (dtype == "bf16" and lay.d in (64, 128)) else 6
+    unused chunk entries, the window softmax (float32 o_soft) and the readout
+    finishing the output (o_lin, RMSNorm, gates)."""
+    return 6
 
 
 # ----------------------------------------------------------------- clocks

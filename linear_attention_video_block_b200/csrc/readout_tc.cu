@@ -12,6 +12,13 @@
 //              (S_hi = bf16(S_sum), S_lo = bf16(S_sum - S_hi)), then drain each
 //              accumulator to global memory as bf16 (one row per thread)
 // Boundary-frame groups write zeros. HBM-bound: q is read once, o_lin written once.
+//
+// Combine variant (project page, "Gating the Softmax and Linear Branch
+// Outputs"): instead of o_lin, each drain thread finishes its row of the hybrid
+// output, out = sigmoid(g_s) o_soft + sigmoid(g_l) RMSNorm(o_lin), from the
+// float32 softmax-branch output of the window kernel and the two gates
+// (boundary frames: out = sigmoid(g_s) o_soft); optionally the two gated
+// branches separately.
 #include "tc_common.cuh"
 
 namespace vdn {
@@ -51,16 +58,61 @@ struct RBars {
   int abort;
 };
 
+// Inputs and outputs of the combine variant.
+struct CombineArgs {
+  const float* o_soft;             // [B, L, H, D] fp32 softmax branch
+  const __nv_bfloat16* g_soft;     // [B, L, H, D]
+  const __nv_bfloat16* g_lin;      // [B, L, H, D]
+  const float* rms_w;              // [D] or null
+  float eps;
+  __nv_bfloat16* out;              // [B, L, H, D]
+  __nv_bfloat16* out_soft;         // nullable
+  __nv_bfloat16* out_lin;          // nullable
+};
+
+__device__ __forceinline__ float sigmoid_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.f + ex2(-1.4426950408889634f * x)));
+  return r;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Combines 8 consecutive elements of one row: o (softmax branch, fp32), lin
+// (RMS-normalised linear branch, already weighted; 0 for boundary rows) and
+// the two gate words; writes out (and the gated branches when asked).
+__device__ __forceinline__ void combine8(const CombineArgs& cx, long long off, const float* o,
+                                         const float* lin, uint4 gs4, uint4 gl4, bool has_lin) {
+  const uint32_t gsw[4] = {gs4.x, gs4.y, gs4.z, gs4.w};
+  const uint32_t glw[4] = {gl4.x, gl4.y, gl4.z, gl4.w};
+  uint32_t ow[4], osw[4], olw[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float a0 = sigmoid_approx(bf16_lo(gsw[e])) * o[2 * e];
+    const float a1 = sigmoid_approx(bf16_hi(gsw[e])) * o[2 * e + 1];
+    const float b0 = has_lin ? sigmoid_approx(bf16_lo(glw[e])) * lin[2 * e] : 0.f;
+    const float b1 = has_lin ? sigmoid_approx(bf16_hi(glw[e])) * lin[2 * e + 1] : 0.f;
+    ow[e] = pack_bf16(a0 + b0, a1 + b1);
+    osw[e] = pack_bf16(a0, a1);
+    olw[e] = pack_bf16(b0, b1);
+  }
+  *reinterpret_cast<uint4*>(cx.out + off) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+  if (cx.out_soft) *reinterpret_cast<uint4*>(cx.out_soft + off) = make_uint4(osw[0], osw[1], osw[2], osw[3]);
+  if (cx.out_lin) *reinterpret_cast<uint4*>(cx.out_lin + off) = make_uint4(olw[0], olw[1], olw[2], olw[3]);
+}
+
 __device__ __forceinline__ bool rwait(unsigned long long* bar, uint32_t parity, volatile int* abort,
                                       bool watch_abort = true) {
   if (mbar_try_wait(smem_u32(bar), parity)) return true;
   return mbar_wait_impl(bar, parity, abort, &g_readout_status, watch_abort);
 }
 
-template <int D>
+template <int D, bool kCombine>
 __global__ void __launch_bounds__(kThreads, 1)
 readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Layout l,
-                  const float* __restrict__ states, __nv_bfloat16* __restrict__ o_lin) {
+                  const float* __restrict__ states, __nv_bfloat16* __restrict__ o_lin,
+                  const CombineArgs cx) {
   using C = RCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -82,8 +134,17 @@ readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Layout l,
     // boundary frame: no linear readout
     for (int i = threadIdx.x; i < rows * (D / 8); i += kThreads) {
       const int r = i / (D / 8), c = i % (D / 8);
-      reinterpret_cast<uint4*>(o_lin + ((long long)b * l.L() + r0 + r) * HD + (long long)h * D)[c] =
-          make_uint4(0u, 0u, 0u, 0u);
+      const long long off = ((long long)b * l.L() + r0 + r) * HD + (long long)h * D + c * 8;
+      if constexpr (kCombine) {
+        const float4 o0 = *reinterpret_cast<const float4*>(cx.o_soft + off);
+        const float4 o1 = *reinterpret_cast<const float4*>(cx.o_soft + off + 4);
+        const float o[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+        const float lin[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        combine8(cx, off, o, lin, *reinterpret_cast<const uint4*>(cx.g_soft + off),
+                 make_uint4(0u, 0u, 0u, 0u), false);
+      } else {
+        *reinterpret_cast<uint4*>(o_lin + off) = make_uint4(0u, 0u, 0u, 0u);
+      }
     }
     return;
   }
@@ -207,7 +268,44 @@ readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Layout l,
       tc_fence_after();
       const int grow = r0 + t * kRows + m;
       const bool store = grow < G.q0 + G.nq;
-      __nv_bfloat16* dst = o_lin + ((long long)b * l.L() + grow) * HD + (long long)h * D;
+      const long long rbase = ((long long)b * l.L() + grow) * HD + (long long)h * D;
+      __nv_bfloat16* dst = o_lin + rbase;
+      if constexpr (kCombine) {
+        // RMSNorm statistic of the row, then the gated sum in 32-column pieces
+        const uint32_t tacc = tmem + lane_base + s * D;
+        float ss4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld_x32(tacc + c0, r);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ss4[i & 3] = fmaf(__uint_as_float(r[i]), __uint_as_float(r[i]), ss4[i & 3]);
+        }
+        const float rstd = rsqrtf(((ss4[0] + ss4[1]) + (ss4[2] + ss4[3])) / (float)D + cx.eps);
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld_x32(tacc + c0, r);
+          if (store) {
+#pragma unroll
+            for (int g8 = 0; g8 < 4; ++g8) {
+              const long long off = rbase + c0 + 8 * g8;
+              const float4 o0 = *reinterpret_cast<const float4*>(cx.o_soft + off);
+              const float4 o1 = *reinterpret_cast<const float4*>(cx.o_soft + off + 4);
+              const float o[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+              float lin[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                lin[e] = __uint_as_float(r[8 * g8 + e]) * rstd * (cx.rms_w ? cx.rms_w[c0 + 8 * g8 + e] : 1.f);
+              combine8(cx, off, o, lin, *reinterpret_cast<const uint4*>(cx.g_soft + off),
+                       *reinterpret_cast<const uint4*>(cx.g_lin + off), true);
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&bars->d_empty[s]);
+        continue;
+      }
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t r[32];
@@ -236,18 +334,18 @@ readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Layout l,
   }
 }
 
-template <int D>
+template <int D, bool kCombine>
 cudaError_t launch_readout_t(const Layout& l, const void* q, const float* states, void* o_lin,
-                             cudaStream_t st) {
+                             const CombineArgs& cx, cudaStream_t st) {
   CUtensorMap mq;
   if (!make_map(&mq, q, D, l.H, l.L(), l.B)) return cudaErrorInvalidValue;
-  auto kern = readout_tc_kernel<D>;
+  auto kern = readout_tc_kernel<D, kCombine>;
   const int smem = RCfg<D>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(tiles_per_head(l, kRows * kTilesPerCta), l.H, l.B);
   if (grid.x == 0) return cudaSuccess;
-  kern<<<grid, kThreads, smem, st>>>(mq, l, states, static_cast<__nv_bfloat16*>(o_lin));
+  kern<<<grid, kThreads, smem, st>>>(mq, l, states, static_cast<__nv_bfloat16*>(o_lin), cx);
   return cudaGetLastError();
 }
 
@@ -259,8 +357,22 @@ bool readout_tc_supported(const Layout& l, int dtype) {
 
 cudaError_t launch_readout_tc(const Layout& l, const void* q, const float* states, void* o_lin,
                               cudaStream_t st) {
-  if (l.d == 128) return launch_readout_t<128>(l, q, states, o_lin, st);
-  if (l.d == 64) return launch_readout_t<64>(l, q, states, o_lin, st);
+  const CombineArgs cx{};
+  if (l.d == 128) return launch_readout_t<128, false>(l, q, states, o_lin, cx, st);
+  if (l.d == 64) return launch_readout_t<64, false>(l, q, states, o_lin, cx, st);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_combine_tc(const Layout& l, const void* q, const float* states,
+                              const float* o_soft, const void* gs, const void* gl,
+                              const float* rms_w, float eps, void* out, void* out_soft,
+                              void* out_lin, cudaStream_t st) {
+  const CombineArgs cx{o_soft, static_cast<const __nv_bfloat16*>(gs),
+                       static_cast<const __nv_bfloat16*>(gl), rms_w, eps,
+                       static_cast<__nv_bfloat16*>(out), static_cast<__nv_bfloat16*>(out_soft),
+                       static_cast<__nv_bfloat16*>(out_lin)};
+  if (l.d == 128) return launch_readout_t<128, true>(l, q, states, nullptr, cx, st);
+  if (l.d == 64) return launch_readout_t<64, true>(l, q, states, nullptr, cx, st);
   return cudaErrorInvalidValue;
 }
 

@@ -41,7 +41,7 @@ struct Workspace {
   float* am = nullptr;
   float* bw = nullptr;
   float* states = nullptr;
-  float* o_soft = nullptr;  // float32 intermediate of the hybrid path
+  float* o_soft = nullptr;  // float32 softmax-branch output of the hybrid path
   size_t bytes = 0;
 };
 
@@ -138,7 +138,7 @@ extern "C" {
 size_t vdn_workspace_bytes(const vdn_layout_t* layout, int dtype) {
   if (!layout_ok(layout) || !dtype_d_ok(dtype, layout->d)) return 0;
   const Layout l = to_layout(layout);
-  return carve(l, dtype, nullptr, true, !vdn::window_tc_supported(l, dtype)).bytes;
+  return carve(l, dtype, nullptr, true, true).bytes;
 }
 
 int vdn_window_softmax_fwd(const vdn_layout_t* layout, int dtype, const void* q, const void* k,
@@ -208,23 +208,23 @@ int hybrid_impl(const vdn_layout_t* layout, int dtype, const vdn_context_t* ctx,
   vdn::JointArgs ja;
   const int js = joint_setup(layout, ctx, ls, ja);
   if (js != VDN_OK) return js;
-  // The tcgen05 path fuses readout, norm and gates into the window kernel and
-  // needs no o_soft intermediate; the CUDA-core path keeps it in fp32.
-  const bool fused = vdn::window_tc_supported(l, dtype);
-  const Workspace need = carve(l, dtype, nullptr, true, !fused);
+  // Window softmax into a float32 o_soft, then the readout finishing the
+  // output (tensor cores for bf16 with d in {64, 128}, CUDA cores otherwise).
+  const bool tc = vdn::readout_tc_supported(l, dtype);
+  const Workspace need = carve(l, dtype, nullptr, true, true);
   if (!workspace || workspace_bytes < need.bytes) return VDN_ERR_WORKSPACE;
-  const Workspace w = carve(l, dtype, workspace, true, !fused);
+  const Workspace w = carve(l, dtype, workspace, true, true);
   const void* kt = layout->T ? k_text : nullptr;
   const void* vt = layout->T ? v_text : nullptr;
   const float* bt = layout->T ? beta_text : nullptr;
   int s = cuda_status(vdn::launch_vda_states(l, dtype, k, v, kt, vt, beta, bt, alpha, w.am, w.bw,
                                              w.states, stream));
   if (s != VDN_OK) return s;
-  if (fused)
-    return cuda_status(vdn::launch_hybrid_tc(ls, q, k, v, kt, vt, w.states, g_soft, g_lin, rms_weight,
-                                             rms_eps, out, out_soft, out_lin, ja, stream));
   s = run_window(ls, dtype, q, k, v, kt, vt, w.o_soft, true, nullptr, ja, stream);
   if (s != VDN_OK) return s;
+  if (tc)
+    return cuda_status(vdn::launch_combine_tc(l, q, w.states, w.o_soft, g_soft, g_lin, rms_weight,
+                                              rms_eps, out, out_soft, out_lin, stream));
   return cuda_status(vdn::launch_readout(l, dtype, 1, q, w.states, w.o_soft, g_soft, g_lin,
                                          rms_weight, rms_eps, out, out_soft, out_lin, stream));
 }

@@ -238,14 +238,6 @@ cudaError_t launch_window_tc(const Layout& l, const void* q, const void* k, cons
                              const void* kt, const void* vt, void* o, bool out_f32, float* lse,
                              const JointArgs& ja, cudaStream_t st);
 
-// tcgen05 window softmax with the hybrid epilogue fused (bf16, d in {64, 128}):
-// needs the chunk read states first; writes out (and optionally the two gated
-// branches) directly; context query rows (if any) get the plain epilogue.
-cudaError_t launch_hybrid_tc(const Layout& l, const void* q, const void* k, const void* v,
-                             const void* kt, const void* vt, const float* states, const void* gs,
-                             const void* gl, const float* rms_w, float eps, void* out,
-                             void* out_soft, void* out_lin, const JointArgs& ja, cudaStream_t st);
-
 // Reads and clears the device status word of the tcgen05 kernels' translation
 // unit (bounded waits record VDN_ERR_TIMEOUT there).
 cudaError_t read_and_clear_tc_status(int* status);
@@ -263,6 +255,15 @@ bool readout_tc_supported(const Layout& l, int dtype);
 cudaError_t launch_readout_tc(const Layout& l, const void* q, const float* states, void* o_lin,
                               cudaStream_t st);
 cudaError_t read_and_clear_readout_status(int* status);
+
+// The same readout finishing the hybrid output instead of writing o_lin:
+// out = sig(gs) o_soft + sig(gl) RMSNorm(o_lin) (o_soft: fp32 [B, L, H, d] from
+// the window kernel; boundary frames: out = sig(gs) o_soft); out_soft and
+// out_lin (nullable) receive the two gated branches.
+cudaError_t launch_combine_tc(const Layout& l, const void* q, const float* states,
+                              const float* o_soft, const void* gs, const void* gl,
+                              const float* rms_w, float eps, void* out, void* out_soft,
+                              void* out_lin, cudaStream_t st);
 
 // VDA: Gram into (am, bw) slots [B, H, F, d, d] (slot 0 = text), inverse in place
 // of am, scans into states [B, H, 2, J, d, d]. alpha (nullable) [B, F, H, d]: KDA

@@ -11,23 +11,19 @@
 // is partially masked. In a joint layer the text and audio query rows are
 // extra groups of the same grid whose key set is every token (the dense
 // softmax the pages keep for interactions involving text or audio); they are
-// scheduled first, being the longest, and always take the plain epilogue.
+// scheduled first, being the longest.
 //
 // CTA = 256 query rows (two 128-row Q tiles) of one query group of one
 // (b, h); 320 threads (at most 200 registers each):
 //   warps 0-3   softmax warpgroup of Q tile 0 (thread i owns row i = TMEM lane i)
 //   warps 4-7   softmax warpgroup of Q tile 1
 //   warp  8     lane 0: TMA producer (Q once, then K_t, V_t tiles into a ring
-//               of shared-memory slots); lanes 1-31 (fused variant only) stage
-//               the chunk's VDA read state S_sum = S_fwd + S_rev in shared
-//               memory as a bf16 K-major operand while the mainloop runs, in
-//               two parts S_hi = bf16(S_sum) and S_lo = bf16(S_sum - S_hi), so
-//               that the readout keeps about 16 significant bits of the state
+//               of shared-memory slots)
 //   warp  9     MMA issuer (one elected lane) and TMEM owner
-// Fused hybrid variant (project page, "Gating the Softmax and Linear Branch
-// Outputs"): after the last P.V the MMA issuer computes O_lin = Q S_hi^T +
-// Q S_lo^T into the freed S columns of TMEM, and each softmax thread, owning a whole row,
-// finishes out = sigmoid(g_s) o_soft + sigmoid(g_l) RMSNorm(o_lin) in registers.
+// The hybrid output is finished by the tensor-core readout (readout_tc.cu)
+// from this kernel's float32 o_soft: fusing the readout, RMSNorm and gates
+// into this epilogue was measured slower (the long per-CTA epilogue holds the
+// SM, one CTA per SM, while a separate pass runs at full occupancy).
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+d) O1 [256+d,256+2d).
 // P (bf16) overwrites the first 64 columns of S and is the A operand of P.V
 // straight from TMEM. MMA issue order per key tile t:
@@ -70,8 +66,7 @@ struct Cfg {
   static constexpr int kHalfBytes = kRows * 128;       // one 128-row x 64-column atom column
   static constexpr int kSlots = (D == 128) ? 4 : 8;
   static constexpr int kQBytes = 2 * kTileBytes;
-  static constexpr int kSsumBytes = kRows * D * 2;     // bf16 S_sum, 128 x D (fused only)
-  static constexpr int kSmemBytes = 1024 + kQBytes + kSlots * kTileBytes + kSsumBytes + 256;
+  static constexpr int kSmemBytes = 1024 + kQBytes + kSlots * kTileBytes + 256;
 };
 
 struct Bars {
@@ -81,8 +76,6 @@ struct Bars {
   unsigned long long s_full[2];
   unsigned long long p_full[2][2];   // [Q tile][key half]: P of keys 0..63 / 64..127
   unsigned long long o_full;
-  unsigned long long ssum_ready;
-  unsigned long long ssum_free;
   uint32_t tmem_base;
   int abort;
 };
@@ -101,18 +94,6 @@ struct CtxOut {
   __nv_bfloat16* o_audio;
   float* lse_text;
   float* lse_audio;
-};
-
-// Extra arguments of the fused hybrid epilogue.
-struct HybridArgs {
-  const float* states;             // [B, H, 2, J, D, D] fp32 chunk read states
-  const __nv_bfloat16* g_soft;     // [B, L, H, D]
-  const __nv_bfloat16* g_lin;      // [B, L, H, D]
-  const float* rms_w;              // [D] or null
-  float eps;
-  __nv_bfloat16* out;              // [B, L, H, D]
-  __nv_bfloat16* out_soft;         // nullable
-  __nv_bfloat16* out_lin;          // nullable
 };
 
 // Packed fp32 pairs (sm_100 f32x2 arithmetic) and the 3-input max: they halve
@@ -142,26 +123,21 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-__device__ __forceinline__ float sigmoid_fast(float x) {
-  return 1.f / (1.f + ex2(-1.4426950408889634f * x));
-}
-
-template <int D, bool kFuse>
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kt,
                  const __grid_constant__ CUtensorMap tm_vt, const __grid_constant__ CUtensorMap tm_ka,
                  const __grid_constant__ CUtensorMap tm_va, const __grid_constant__ CUtensorMap tm_qt,
                  const __grid_constant__ CUtensorMap tm_qa, const Layout l, void* out, int out_f32,
-                 float* lse, const HybridArgs hy, const CtxOut cx) {
+                 float* lse, const CtxOut cx) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = smem;
   uint8_t* sKV = smem + C::kQBytes;
-  uint8_t* sSsum = sKV + C::kSlots * C::kTileBytes;
-  Bars* bars = reinterpret_cast<Bars*>(sSsum + (kFuse ? C::kSsumBytes : 0));
+  Bars* bars = reinterpret_cast<Bars*>(sKV + C::kSlots * C::kTileBytes);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -170,7 +146,6 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   tile_to_group(l, 2 * kRows, blockIdx.x, g, r0);
   const Group G = make_group(l, g < 0 ? 0 : g);
   const int n_tiles = key_tile_count(G, l.T, l.A, kRows);
-  const bool has_lin = kFuse && G.chunk >= 0;
   const bool ctx_rows = G.qsrc != kQVideo;
 
   if (threadIdx.x == 0) {
@@ -185,8 +160,6 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       mbar_init(&bars->p_full[w][1], 128);
     }
     mbar_init(&bars->o_full, 1);
-    mbar_init(&bars->ssum_ready, 31);
-    mbar_init(&bars->ssum_free, 1);
     bars->abort = (g < 0) ? 1 : 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -203,36 +176,6 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   volatile int* abort = &bars->abort;
 
   if (warp == kProducerWarp) {
-    // ---------------------------------------------- S_sum staging (fused)
-    if (lane > 0 && has_lin && !*abort) {
-      const int t = lane - 1;  // 31 staging lanes
-      const int J = l.J();
-      const float* sf = hy.states + ((((long long)b * l.H + h) * 2 + 0) * J + G.chunk) * D * D;
-      const float* sr = hy.states + ((((long long)b * l.H + h) * 2 + 1) * J + G.chunk) * D * D;
-      constexpr int kChunks = D / 8;  // 16-byte chunks per row
-      for (int part = 0; part < 2; ++part) {
-        if (part == 1 && !mbar_wait(&bars->ssum_free, 0, abort)) break;
-        for (int ch = t; ch < kRows * kChunks; ch += 31) {
-          const int n = ch / kChunks, kc = ch % kChunks;
-          const float4 a0 = *reinterpret_cast<const float4*>(sf + n * D + kc * 8);
-          const float4 a1 = *reinterpret_cast<const float4*>(sf + n * D + kc * 8 + 4);
-          const float4 b0 = *reinterpret_cast<const float4*>(sr + n * D + kc * 8);
-          const float4 b1 = *reinterpret_cast<const float4*>(sr + n * D + kc * 8 + 4);
-          float x[8] = {a0.x + b0.x, a0.y + b0.y, a0.z + b0.z, a0.w + b0.w,
-                        a1.x + b1.x, a1.y + b1.y, a1.z + b1.z, a1.w + b1.w};
-          if (part == 1) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] -= __bfloat162float(__float2bfloat16_rn(x[e]));
-          }
-          const uint4 v = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]),
-                                     pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
-          const int half = kc / 8, c16 = kc % 8;
-          *reinterpret_cast<uint4*>(sSsum + half * C::kHalfBytes + n * 128 + ((c16 ^ (n & 7)) * 16)) = v;
-        }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_arrive(&bars->ssum_ready);
-      }
-    }
     if (lane == 0 && !*abort) {
       // ------------------------------------------------------- TMA producer
       const CUtensorMap* mq = G.qsrc == kQVideo ? &tm_q : (G.qsrc == kQText ? &tm_qt : &tm_qa);
@@ -276,7 +219,6 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       // ------------------------------------------------------- MMA issuer
       constexpr uint32_t idesc_s = make_idesc(kRows, false);
       constexpr uint32_t idesc_o = make_idesc(D, true);
-      constexpr uint32_t idesc_lin = make_idesc(D, false);
       const uint32_t q_addr = smem_u32(sQ);
       const uint32_t kv_addr = smem_u32(sKV);
       int use = 0;
@@ -344,27 +286,6 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           issue_s(1, ks_next);
           tc_commit(&bars->s_full[1]);
           tc_commit(&bars->kv_empty[ks_next]);
-        }
-      }
-      if (ok && has_lin) {
-        // O_lin_w = Q_w S_hi^T + Q_w S_lo^T into the S columns of TMEM (issued after
-        // the last P.V, which reads P from those columns; tcgen05.mma runs in
-        // issue order). The helpers restage S_lo into the same buffer once the
-        // S_hi products have completed.
-        const uint32_t s_addr = smem_u32(sSsum);
-        for (int part = 0; part < 2 && ok; ++part) {
-          ok = mbar_wait(&bars->ssum_ready, part, abort);
-          if (!ok) break;
-          tc_fence_after();
-          for (int w = 0; w < 2; ++w) {
-#pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-              const uint32_t off = (uint32_t)((ks / 4) * C::kHalfBytes + (ks % 4) * 32);
-              mma_ss(tmem + 128 * w, desc_k_sw128(q_addr + w * C::kTileBytes + off),
-                     desc_k_sw128(s_addr + off), idesc_lin, (part > 0 || ks > 0) ? 1u : 0u);
-            }
-          }
-          if (part == 0) tc_commit(&bars->ssum_free);
         }
       }
       tc_commit(&bars->o_full);
@@ -488,7 +409,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       // audio [B, A, H, D]
       const long long qrows = G.qsrc == kQVideo ? l.L() : (G.qsrc == kQText ? l.T : l.A);
       const long long base = (((long long)b * qrows + grow) * l.H + h) * D;
-      if (!kFuse || ctx_rows) {
+      {
         void* dst_o = out;
         float* dst_lse = lse;
         bool f32 = out_f32 != 0;
@@ -521,67 +442,6 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         if (store && dst_lse)
           dst_lse[((long long)b * qrows + grow) * l.H + h] = (m + log2f(lsum)) * 0.6931471805599453f;
-      } else {
-        // RMSNorm statistic of o_lin (whole row in this thread)
-        float rstd = 0.f;
-        if (has_lin) {
-          float ss4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld_x32(tS + c0, o);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float x = __uint_as_float(o[i]);
-              ss4[i & 3] = fmaf(x, x, ss4[i & 3]);
-            }
-          }
-          rstd = rsqrtf(((ss4[0] + ss4[1]) + (ss4[2] + ss4[3])) / (float)D + hy.eps);
-        }
-#pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t os[32], ol[32];
-          tmem_ld_x32(tO + c0, os);
-          if (has_lin) tmem_ld_x32(tS + c0, ol);
-          if (store) {
-            const uint4* gsp = reinterpret_cast<const uint4*>(hy.g_soft + base + c0);
-            const uint4* glp = reinterpret_cast<const uint4*>(hy.g_lin + base + c0);
-#pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4) {
-              const uint4 gs4 = gsp[v4];
-              const uint4 gl4 = glp[v4];
-              const uint32_t gsw[4] = {gs4.x, gs4.y, gs4.z, gs4.w};
-              const uint32_t glw[4] = {gl4.x, gl4.y, gl4.z, gl4.w};
-              uint32_t ow[4], osw[4], olw[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                float r2[2], a2[2], b2[2];
-#pragma unroll
-                for (int k2 = 0; k2 < 2; ++k2) {
-                  const int i = v4 * 8 + e * 2 + k2;
-                  const float gsv = __uint_as_float(k2 ? (gsw[e] & 0xFFFF0000u) : (gsw[e] << 16));
-                  const float glv = __uint_as_float(k2 ? (glw[e] & 0xFFFF0000u) : (glw[e] << 16));
-                  a2[k2] = sigmoid_fast(gsv) * (__uint_as_float(os[i]) * inv);
-                  float lin = 0.f;
-                  if (has_lin) {
-                    const float wv = hy.rms_w ? hy.rms_w[c0 + i] : 1.f;
-                    lin = sigmoid_fast(glv) * (__uint_as_float(ol[i]) * rstd * wv);
-                  }
-                  b2[k2] = lin;
-                  r2[k2] = a2[k2] + lin;
-                }
-                ow[e] = pack_bf16(r2[0], r2[1]);
-                osw[e] = pack_bf16(a2[0], a2[1]);
-                olw[e] = pack_bf16(b2[0], b2[1]);
-              }
-              reinterpret_cast<uint4*>(hy.out + base + c0)[v4] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-              if (hy.out_soft)
-                reinterpret_cast<uint4*>(hy.out_soft + base + c0)[v4] = make_uint4(osw[0], osw[1], osw[2], osw[3]);
-              if (hy.out_lin)
-                reinterpret_cast<uint4*>(hy.out_lin + base + c0)[v4] = make_uint4(olw[0], olw[1], olw[2], olw[3]);
-            }
-          }
-        }
       }
     }
   }
@@ -597,10 +457,10 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
 // ------------------------------------------------------------------- host
 
-template <int D, bool kFuse>
+template <int D>
 cudaError_t launch_tc_t(const Layout& l, const void* q, const void* k, const void* v,
                         const void* kt, const void* vt, void* o, bool out_f32, float* lse,
-                        const HybridArgs& hy, const JointArgs& ja, cudaStream_t st) {
+                        const JointArgs& ja, cudaStream_t st) {
   CUtensorMap mq, mk, mv, mkt, mvt, mka, mva, mqt, mqa;
   const long long L = l.L();
   if (!make_map(&mq, q, D, l.H, L, l.B) || !make_map(&mk, k, D, l.H, L, l.B) ||
@@ -619,14 +479,14 @@ cudaError_t launch_tc_t(const Layout& l, const void* q, const void* k, const voi
     return cudaErrorInvalidValue;
   const CtxOut cx{static_cast<__nv_bfloat16*>(ja.o_text), static_cast<__nv_bfloat16*>(ja.o_audio),
                   ja.lse_text, ja.lse_audio};
-  auto kern = window_tc_kernel<D, kFuse>;
-  const int smem = Cfg<D>::kSmemBytes - (kFuse ? 0 : Cfg<D>::kSsumBytes);
+  auto kern = window_tc_kernel<D>;
+  const int smem = Cfg<D>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(tiles_per_head(l, 2 * kRows), l.H, l.B);
   if (grid.x == 0) return cudaSuccess;
   kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, mkt, mvt, mka, mva, mqt, mqa, l, o, out_f32 ? 1 : 0,
-                                     lse, hy, cx);
+                                     lse, cx);
   return cudaGetLastError();
 }
 
@@ -639,27 +499,8 @@ bool window_tc_supported(const Layout& l, int dtype) {
 cudaError_t launch_window_tc(const Layout& l, const void* q, const void* k, const void* v,
                              const void* kt, const void* vt, void* o, bool out_f32, float* lse,
                              const JointArgs& ja, cudaStream_t st) {
-  HybridArgs hy{};
-  if (l.d == 128) return launch_tc_t<128, false>(l, q, k, v, kt, vt, o, out_f32, lse, hy, ja, st);
-  if (l.d == 64) return launch_tc_t<64, false>(l, q, k, v, kt, vt, o, out_f32, lse, hy, ja, st);
-  return cudaErrorInvalidValue;
-}
-
-cudaError_t launch_hybrid_tc(const Layout& l, const void* q, const void* k, const void* v,
-                             const void* kt, const void* vt, const float* states, const void* gs,
-                             const void* gl, const float* rms_w, float eps, void* out,
-                             void* out_soft, void* out_lin, const JointArgs& ja, cudaStream_t st) {
-  HybridArgs hy;
-  hy.states = states;
-  hy.g_soft = static_cast<const __nv_bfloat16*>(gs);
-  hy.g_lin = static_cast<const __nv_bfloat16*>(gl);
-  hy.rms_w = rms_w;
-  hy.eps = eps;
-  hy.out = static_cast<__nv_bfloat16*>(out);
-  hy.out_soft = static_cast<__nv_bfloat16*>(out_soft);
-  hy.out_lin = static_cast<__nv_bfloat16*>(out_lin);
-  if (l.d == 128) return launch_tc_t<128, true>(l, q, k, v, kt, vt, nullptr, false, nullptr, hy, ja, st);
-  if (l.d == 64) return launch_tc_t<64, true>(l, q, k, v, kt, vt, nullptr, false, nullptr, hy, ja, st);
+  if (l.d == 128) return launch_tc_t<128>(l, q, k, v, kt, vt, o, out_f32, lse, ja, st);
+  if (l.d == 64) return launch_tc_t<64>(l, q, k, v, kt, vt, o, out_f32, lse, ja, st);
   return cudaErrorInvalidValue;
 }
 
