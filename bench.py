@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload 768p-bf16]
-                    [--entry hybrid|window|vda|vda-decay|hybrid-decay|joint|joint-window]
+                    [--entry hybrid|window|window-fp8|vda|vda-decay|hybrid-decay|joint|joint-window]
 
 A step is one vdn_hybrid_attn_fwd call (window softmax + VDA scans + readout,
 norm, gates) over one 768p-like layer input (B=1, H=40, d=128, F=36 frames of
@@ -21,7 +21,8 @@ for profiling one kernel family at a time, or the KDA-decayed forms
 (vdn_vda_scan_fwd_decay / vdn_hybrid_attn_fwd_decay, alpha in (0.8, 1]), or
 the joint text-video-audio layer (vdn_joint_attn_fwd / vdn_joint_softmax_fwd:
 audio keys for every video query, dense text and audio query rows; the audio
-length that goes with the clip, 203 tokens at 768p).
+length that goes with the clip, 203 tokens at 768p), or the softmax branch with
+float8 e4m3 operands (vdn_window_softmax_fwd_fp8).
 
 Printed on rank 0: one JSON line with the throughput (video tokens/s over all
 ranks), the roofline of the dominant kernel (window softmax, tensor-core bound),
@@ -443,7 +444,7 @@ def run_entry(args, rank, world, local_rank):
     import torch
     from linear_attention_video_block_b200 import vdn
     from linear_attention_video_block_b200.synth import (WORKLOADS, audio_tokens, make_context,
-                                                         make_decay, make_inputs)
+                                                         make_decay, make_inputs, quantize_e4m3)
 
     lay, dtype, seed = WORKLOADS[args.workload]
     dev = torch.device("cuda", local_rank)
@@ -459,6 +460,13 @@ def run_entry(args, rank, world, local_rank):
         def step():
             vdn.window_softmax_fwd(lay, inp["q"], inp["k"], inp["v"], inp["k_text"], inp["v_text"],
                                    o_soft=out)
+    elif args.entry == "window-fp8":
+        (q8,), sq = quantize_e4m3(inp["q"])
+        (k8, kt8), sk = quantize_e4m3(inp["k"], inp["k_text"])
+        (v8, vt8), sv = quantize_e4m3(inp["v"], inp["v_text"])
+
+        def step():
+            vdn.window_softmax_fwd_fp8(lay, q8, k8, v8, kt8, vt8, sq, sk, sv, o_soft=out)
     elif args.entry == "joint":
         o_text, o_audio = torch.empty_like(cx["q_text"]), torch.empty_like(cx["q_audio"])
 
@@ -508,6 +516,11 @@ def run_entry(args, rank, world, local_rank):
     elif args.entry == "joint-window":
         work, unit, peak = joint_flops(lay, A) / 1e12, "TFLOP/s", float(peaks["bf16_tflops"])
         bound = "tensor"
+    elif args.entry == "window-fp8":
+        # e4m3 dense peak: the measured bf16 peak times the nominal fp8 / bf16 ratio (2)
+        work, unit, peak = window_flops(lay) / 1e12, "TFLOP/s", 2.0 * float(peaks["bf16_tflops"])
+        bound = "tensor"
+        kind = f"{kind} bf16 x 2 (nominal e4m3 / bf16 ratio)"
     elif args.entry in ("hybrid-decay", "joint"):
         work, unit, peak, bound = None, None, None, None
     else:
@@ -522,7 +535,7 @@ def run_entry(args, rank, world, local_rank):
     print(json.dumps({
         "impl": "ours", "entry": args.entry, "metric": f"{args.entry} fwd video tokens/s",
         "value": lay.L * lay.B / (ms * 1e-3), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "dtype": dtype,
+        "warmup": args.warmup, "ms_per_step": ms, "dtype": "e4m3" if args.entry == "window-fp8" else dtype,
         "config": dict(config_of(args.workload, lay),
                        **({"audio_tokens": A, "context_query_rows": lay.T + A}
                           if args.entry.startswith("joint") else {})),
@@ -537,8 +550,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="768p-bf16")
-    ap.add_argument("--entry", choices=["hybrid", "window", "vda", "vda-decay", "hybrid-decay",
-                                        "joint", "joint-window"], default="hybrid")
+    ap.add_argument("--entry", choices=["hybrid", "window", "window-fp8", "vda", "vda-decay",
+                                        "hybrid-decay", "joint", "joint-window"], default="hybrid")
     ap.add_argument("--ref-rows", type=int, default=96,
                     help="query rows per frame in the oracle's bounded sample")
     args = ap.parse_args()

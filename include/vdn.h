@@ -157,6 +157,22 @@ int vdn_hybrid_attn_fwd_decay(const vdn_layout_t* layout, int dtype,
                               void* out, void* out_soft, void* out_lin,
                               void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* Softmax branch with FP8 operands (the FP8 attention of the pages' serving
+ * stack, "Faster Than It Plays" and the H3 serving notes): q, k, v, k_text,
+ * v_text are float8 e4m3 tensors (1 byte per element, same [B, L, H, d] and
+ * [B, T, H, d] layouts) with one scale per tensor: value = e4m3 * scale; the
+ * text keys and values share k_scale and v_scale. Same key sets and one
+ * normaliser as vdn_window_softmax_fwd; scores and softmax statistics in
+ * float32, the softmax weights rounded to e4m3 for the P.V product (the row
+ * sum adds them before rounding). o_soft: bf16 [B, L, H, d]; lse (nullable)
+ * as in vdn_window_softmax_fwd. d must be 128 (VDN_ERR_UNSUPPORTED otherwise);
+ * scales must be finite and positive (VDN_ERR_INVALID). */
+int vdn_window_softmax_fwd_fp8(const vdn_layout_t* layout,
+                               const void* q, const void* k, const void* v,
+                               const void* k_text, const void* v_text,
+                               float q_scale, float k_scale, float v_scale,
+                               void* o_soft, float* lse, cudaStream_t stream);
+
 /* The other tokens of a joint text-video-audio attention layer (project page
  * "Video DeltaNet", attention-map paragraph of "Local Softmax and Long-Range
  * Linear Memory"; "Video DeltaNet speeds MiniMax H3 video generation 14.5x",

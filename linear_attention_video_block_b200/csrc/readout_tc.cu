@@ -4,13 +4,15 @@
 // read and their outputs added; boundary frames read nothing).
 //
 // CTA = up to 24 consecutive 128-row query tiles of one query group of one
-// (b, h); 192 threads:
+// (b, h); 320 threads:
 //   warp 0     TMA producer: Q tiles into two shared-memory stages
 //   warp 1     MMA issuer and TMEM owner: O = Q S_hi^T + Q S_lo^T into one of two
 //              TMEM accumulators
-//   warps 2-5  stage S_sum = S_fwd + S_rev once as two bf16 K-major operands
-//              (S_hi = bf16(S_sum), S_lo = bf16(S_sum - S_hi)), then drain each
-//              accumulator to global memory as bf16 (one row per thread)
+//   warps 2-9  stage S_sum = S_fwd + S_rev once as two bf16 K-major operands
+//              (S_hi = bf16(S_sum), S_lo = bf16(S_sum - S_hi)); then warpgroup
+//              2-5 drains the accumulator of the even tiles and warpgroup 6-9
+//              that of the odd tiles to global memory (one row per thread), so
+//              that two tiles' worth of loads and stores are in flight
 // Boundary-frame groups write zeros. HBM-bound: q is read once, o_lin written once.
 //
 // Combine variant (project page, "Gating the Softmax and Linear Branch
@@ -36,7 +38,8 @@ namespace {
 
 constexpr int kRows = 128;
 constexpr int kTilesPerCta = 24;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
+constexpr int kDrainThreads = 256;
 
 template <int D>
 struct RCfg {
@@ -157,7 +160,7 @@ readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Layout l,
       mbar_init(&bars->d_full[i], 1);
       mbar_init(&bars->d_empty[i], 128);
     }
-    mbar_init(&bars->ssum_ready, 128);
+    mbar_init(&bars->ssum_ready, kDrainThreads);
     mbar_init(&bars->done, 1);
     bars->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -227,14 +230,15 @@ readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Layout l,
       }
     }
   } else {
-    const int t128 = threadIdx.x - 64;
+    const int t256 = threadIdx.x - 64;
+    const int dg = t256 / 128;  // drain warpgroup: tiles with (t & 1) == dg
     // stage S_sum (hi, lo) once
     {
       const int J = l.J();
       const float* sf = states + ((((long long)b * l.H + h) * 2 + 0) * J + G.chunk) * D * D;
       const float* sr = states + ((((long long)b * l.H + h) * 2 + 1) * J + G.chunk) * D * D;
       constexpr int kChunks = D / 8;
-      for (int ch = t128; ch < kRows * kChunks; ch += 128) {
+      for (int ch = t256; ch < kRows * kChunks; ch += kDrainThreads) {
         const int n = ch / kChunks, kc = ch % kChunks;
         if (n >= D) continue;  // rows beyond d (d = 64) stay unused: the MMA reads N = d rows
         const float4 a0 = *reinterpret_cast<const float4*>(sf + n * D + kc * 8);
@@ -262,7 +266,7 @@ readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Layout l,
     // drain accumulators
     const int m = 32 * (warp & 3) + lane;
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-    for (int t = 0; t < n_tiles; ++t) {
+    for (int t = dg; t < n_tiles; t += 2) {
       const int s = t & 1, use = t >> 1;
       if (!__all_sync(0xffffffffu, rwait(&bars->d_full[s], use & 1, abort))) break;
       tc_fence_after();

@@ -147,6 +147,26 @@ int vdn_window_softmax_fwd(const vdn_layout_t* layout, int dtype, const void* q,
   return window_impl(layout, dtype, nullptr, q, k, v, k_text, v_text, o_soft, lse, stream);
 }
 
+int vdn_window_softmax_fwd_fp8(const vdn_layout_t* layout, const void* q, const void* k,
+                               const void* v, const void* k_text, const void* v_text, float q_scale,
+                               float k_scale, float v_scale, void* o_soft, float* lse,
+                               cudaStream_t stream) {
+  if (!layout_ok(layout)) return VDN_ERR_INVALID;
+  if (layout->d != 128) return VDN_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !o_soft) return VDN_ERR_INVALID;
+  if (layout->T > 0 && (!k_text || !v_text)) return VDN_ERR_INVALID;
+  const float sc[3] = {q_scale, k_scale, v_scale};
+  for (float x : sc)
+    if (!(x > 0.f) || !(x < INFINITY)) return VDN_ERR_INVALID;
+  const void* ptrs[] = {q, k, v, o_soft, lse};
+  for (const void* p : ptrs) if (p && !aligned16(p)) return VDN_ERR_UNSUPPORTED;
+  if (layout->T > 0 && (!aligned16(k_text) || !aligned16(v_text))) return VDN_ERR_UNSUPPORTED;
+  const Layout l = to_layout(layout);
+  return cuda_status(vdn::launch_window_fp8(l, q, k, v, layout->T ? k_text : nullptr,
+                                            layout->T ? v_text : nullptr, q_scale * k_scale, v_scale,
+                                            o_soft, lse, stream));
+}
+
 int vdn_joint_softmax_fwd(const vdn_layout_t* layout, int dtype, const vdn_context_t* ctx,
                           const void* q, const void* k, const void* v, const void* k_text,
                           const void* v_text, void* o_soft, float* lse, cudaStream_t stream) {
@@ -289,11 +309,12 @@ int vdn_joint_attn_fwd(const vdn_layout_t* layout, int dtype, const vdn_context_
 
 int vdn_device_status(void) {
   if (cuda_status(cudaDeviceSynchronize()) != VDN_OK) return VDN_ERR_CUDA;
-  int s[3] = {0, 0, 0};
+  int s[4] = {0, 0, 0, 0};
   if (cuda_status(vdn::read_and_clear_tc_status(&s[0])) != VDN_OK) return VDN_ERR_CUDA;
   if (cuda_status(vdn::read_and_clear_gram_status(&s[1])) != VDN_OK) return VDN_ERR_CUDA;
   if (cuda_status(vdn::read_and_clear_readout_status(&s[2])) != VDN_OK) return VDN_ERR_CUDA;
-  for (int i = 0; i < 3; ++i)
+  if (cuda_status(vdn::read_and_clear_fp8_status(&s[3])) != VDN_OK) return VDN_ERR_CUDA;
+  for (int i = 0; i < 4; ++i)
     if (s[i] != 0) return s[i];
   return VDN_OK;
 }

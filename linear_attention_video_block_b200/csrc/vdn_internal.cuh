@@ -238,6 +238,13 @@ cudaError_t launch_window_tc(const Layout& l, const void* q, const void* k, cons
                              const void* kt, const void* vt, void* o, bool out_f32, float* lse,
                              const JointArgs& ja, cudaStream_t st);
 
+// FP8 (e4m3) window softmax (d = 128; no audio keys or context rows): scores
+// scaled by qk_scale / sqrt(d), output (bf16) by v_scale.
+cudaError_t launch_window_fp8(const Layout& l, const void* q, const void* k, const void* v,
+                              const void* kt, const void* vt, float qk_scale, float v_scale,
+                              void* o, float* lse, cudaStream_t st);
+cudaError_t read_and_clear_fp8_status(int* status);
+
 // Reads and clears the device status word of the tcgen05 kernels' translation
 // unit (bounded waits record VDN_ERR_TIMEOUT there).
 cudaError_t read_and_clear_tc_status(int* status);

@@ -137,6 +137,17 @@ def make_context(layout: Layout, A: int, dtype: str, seed: int, device: str = "c
     return out
 
 
+E4M3_MAX = 448.0
+
+
+def quantize_e4m3(*tensors):
+    """Float8 e4m3 copies of tensors that share one scale (value = e4m3 *
+    scale, scale = max |x| / 448 over all of them). Returns ([t8, ...], scale)."""
+    amax = max(float(t.float().abs().max()) if t.numel() else 0.0 for t in tensors)
+    scale = (amax / E4M3_MAX) if amax > 0 else 1.0
+    return [(t.float() / scale).to(torch.float8_e4m3fn) for t in tensors], scale
+
+
 def as_float64_numpy(inputs):
     """The oracle's view of an input set: every tensor upcast to float64 (bf16
     rounding of the stored inputs is therefore not counted as error)."""

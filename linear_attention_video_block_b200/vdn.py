@@ -33,7 +33,8 @@ STATUS = {0: "VDN_OK", 1: "VDN_ERR_INVALID", 2: "VDN_ERR_UNSUPPORTED",
 EXPORTS = ("vdn_workspace_bytes", "vdn_window_softmax_fwd", "vdn_vda_scan_fwd",
            "vdn_vda_scan_fwd_decay", "vdn_hybrid_attn_fwd", "vdn_hybrid_attn_fwd_decay",
            "vdn_vda_scan_fwd_noalloc", "vdn_joint_softmax_fwd", "vdn_joint_attn_fwd",
-           "vdn_device_status", "vdn_status_string", "vdn_last_cuda_error")
+           "vdn_window_softmax_fwd_fp8", "vdn_device_status", "vdn_status_string",
+           "vdn_last_cuda_error")
 
 
 class VdnError(RuntimeError):
@@ -77,6 +78,9 @@ def lib():
         L.vdn_hybrid_attn_fwd_decay.argtypes = ([LP, I] + [P] * 10 + [P, ctypes.c_float]
                                                 + [P] * 3 + [P, S, P])
         L.vdn_hybrid_attn_fwd_decay.restype = I
+        F = ctypes.c_float
+        L.vdn_window_softmax_fwd_fp8.argtypes = [LP] + [P] * 5 + [F, F, F] + [P, P, P]
+        L.vdn_window_softmax_fwd_fp8.restype = I
         CP = ctypes.POINTER(_CContext)
         L.vdn_joint_softmax_fwd.argtypes = [LP, I, CP] + [P] * 8
         L.vdn_joint_softmax_fwd.restype = I
@@ -306,3 +310,23 @@ def joint_attn_fwd(layout: Layout, q, k, v, k_text, v_text, beta, beta_text, g_s
         _ptr(out_lin), _ptr(workspace), workspace.numel(), _stream(q.device))
     _check(code, "vdn_joint_attn_fwd")
     return out, o_text, o_audio
+
+
+def window_softmax_fwd_fp8(layout: Layout, q, k, v, k_text, v_text, q_scale, k_scale, v_scale,
+                           o_soft=None, want_lse=False):
+    """Softmax branch with float8 e4m3 operands (torch.float8_e4m3fn tensors,
+    one scale per tensor; text shares k / v scales). Returns o_soft (bf16) and,
+    with want_lse, the natural-log normaliser."""
+    _require_cuda()
+    for t in (q, k, v):
+        if t.dtype != torch.float8_e4m3fn:
+            raise TypeError("q, k, v must be torch.float8_e4m3fn")
+    if o_soft is None:
+        o_soft = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if want_lse else None
+    code = lib().vdn_window_softmax_fwd_fp8(
+        ctypes.byref(_clayout(layout)), _ptr(q), _ptr(k), _ptr(v), _ptr(k_text), _ptr(v_text),
+        ctypes.c_float(q_scale), ctypes.c_float(k_scale), ctypes.c_float(v_scale), _ptr(o_soft),
+        _ptr(lse), _stream(q.device))
+    _check(code, "vdn_window_softmax_fwd_fp8")
+    return (o_soft, lse) if want_lse else o_soft

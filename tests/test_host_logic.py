@@ -283,3 +283,19 @@ def test_joint_entries_validate_context(lib):
     assert ja(ctypes.byref(ok), 0, ctypes.byref(_ctx(lib)), *pre, *post, need - 1, None) == 3
     assert ja(ctypes.byref(ok), 0, ctypes.byref(_ctx(lib)), *pre, MISALIGNED, *post[1:], need,
               None) == 2                                                                  # alpha
+
+
+def test_fp8_entry_validates(lib):
+    """vdn_window_softmax_fwd_fp8: d = 128 only, positive finite scales, required
+    pointers, 16-byte alignment (no GPU is touched)."""
+    f = lib.vdn_window_softmax_fwd_fp8
+    F = ctypes.c_float
+    ok = _layout(d=128)
+    args = [FAKE] * 5
+    assert f(ctypes.byref(_layout(d=64)), *args, F(1), F(1), F(1), FAKE, None, None) == 2
+    assert f(ctypes.byref(ok), *args, F(0), F(1), F(1), FAKE, None, None) == 1
+    assert f(ctypes.byref(ok), *args, F(1), F(-1), F(1), FAKE, None, None) == 1
+    assert f(ctypes.byref(ok), *args, F(1), F(1), F(float("inf")), FAKE, None, None) == 1
+    assert f(ctypes.byref(ok), *args, F(1), F(1), F(1), None, None, None) == 1
+    assert f(ctypes.byref(ok), MISALIGNED, *args[1:], F(1), F(1), F(1), FAKE, None, None) == 2
+    assert f(ctypes.byref(_layout(d=128, B=0)), *args, F(1), F(1), F(1), FAKE, None, None) == 1
