@@ -358,10 +358,16 @@ def run_ours(args, rank, world, local_rank):
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = out_h.numel() * out_h.element_size()
 
+    # the input copies and the video tensors of the device leg are released
+    # first: the host call keeps its own two chunk buffers on the device
+    del inp, out, o_soft, ws
+    torch.cuda.empty_cache()
+    ws_h = torch.empty(vdn.host_workspace_bytes(lay, host["q"].dtype), dtype=torch.uint8, device=dev)
+
     def e2e_step():
-        vdn.hybrid_attn_fwd(lay, host["q"], host["k"], host["v"], host["k_text"], host["v_text"],
-                            host["beta"], host["beta_text"], host["g_s"], host["g_l"], out=out_h,
-                            workspace=ws, device=str(dev))
+        vdn.hybrid_attn_fwd_host(lay, host["q"], host["k"], host["v"], host["k_text"], host["v_text"],
+                                 host["beta"], host["beta_text"], host["g_s"], host["g_l"], out=out_h,
+                                 workspace=ws_h, device=str(dev))
 
     e2e_step()
     torch.cuda.synchronize(dev)

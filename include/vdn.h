@@ -128,6 +128,26 @@ int vdn_hybrid_attn_fwd(const vdn_layout_t* layout, int dtype,
                         void* out, void* out_soft, void* out_lin,
                         void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* The hybrid forward on tensors in HOST memory (same arguments and layouts as
+ * vdn_hybrid_attn_fwd, every tensor pointer a host pointer; rms_weight, if
+ * given, a host array of d floats). The call copies in, computes and copies
+ * the output back, in chunks of head_chunk heads (<= 0: about ten chunks)
+ * pipelined on three internal streams so that the copies of one chunk overlap
+ * the kernels of the next; the heads are independent, so the result equals
+ * vdn_hybrid_attn_fwd's bit for bit. Host memory should be pinned
+ * (cudaHostAlloc / cudaHostRegister) for the copies to overlap. workspace:
+ * device memory of vdn_hybrid_host_workspace_bytes bytes (two chunk buffers).
+ * Synchronous: returns when out holds the result. Errors as
+ * vdn_hybrid_attn_fwd (validation before any copy). */
+size_t vdn_hybrid_host_workspace_bytes(const vdn_layout_t* layout, int dtype, int head_chunk);
+int vdn_hybrid_attn_fwd_host(const vdn_layout_t* layout, int dtype, int head_chunk,
+                             const void* q, const void* k, const void* v,
+                             const void* k_text, const void* v_text,
+                             const float* beta, const float* beta_text,
+                             const void* g_soft, const void* g_lin,
+                             const float* rms_weight, float rms_eps,
+                             void* out, void* workspace, size_t workspace_bytes);
+
 /* Linear branch with KDA channel decay (project page "Video DeltaNet", section
  * "Video Delta Attention: A Frame-Wise Solution": the inherited state is decayed
  * per key channel before a frame is written, S_bar = S Diag(alpha)). Same as

@@ -1,0 +1,178 @@
+// vdn_hybrid_attn_fwd_host: the hybrid forward on tensors in host memory, with
+// the host-device copies overlapped with the computation.
+//
+// Every (b, h) pair is independent in both branches, so the heads are taken in
+// chunks of head_chunk: chunk i is copied in (one strided 2-D copy per tensor:
+// B * L rows of head_chunk * d elements out of rows of H * d), computed by the
+// same kernels as vdn_hybrid_attn_fwd on a [B, L, head_chunk, d] layout, and its
+// output copied back into the strided host tensor, on three streams (in,
+// compute, out) with two device buffers, so that chunk i + 1 is copied in and
+// chunk i - 1 copied out while chunk i computes. PCIe carries both directions
+// at once; with pinned host memory the copies then hide under the kernels.
+#include <cstdint>
+
+#include "vdn_internal.cuh"
+
+namespace {
+
+constexpr size_t kAlignH = 256;
+size_t align_h(size_t x) { return (x + kAlignH - 1) / kAlignH * kAlignH; }
+
+int elem_size(int dtype) { return dtype == VDN_BF16 ? 2 : 4; }
+
+// One device buffer of the pipeline for a chunk of hc heads.
+struct ChunkBuf {
+  char* q; char* k; char* v; char* gs; char* gl; char* out;  // [B, L, hc, d]
+  char* kt; char* vt;                                          // [B, T, hc, d]
+  float* beta; float* beta_t;                                  // [B, L, hc], [B, T, hc]
+  void* ws;                                                    // hybrid workspace
+  size_t bytes;
+};
+
+// Carves one chunk buffer at base (nullptr: sizes only).
+ChunkBuf carve_chunk(const vdn_layout_t& lc, int dtype, char* base) {
+  ChunkBuf c{};
+  size_t off = 0;
+  auto take = [&](size_t n) -> char* {
+    char* r = base ? base + off : nullptr;
+    off = align_h(off + n);
+    return r;
+  };
+  const size_t es = elem_size(dtype);
+  const size_t video = (size_t)lc.B * lc.F * lc.N * lc.H * lc.d * es;
+  const size_t text = (size_t)lc.B * lc.T * lc.H * lc.d * es;
+  c.q = take(video); c.k = take(video); c.v = take(video); c.gs = take(video); c.gl = take(video);
+  c.out = take(video);
+  c.kt = take(text); c.vt = take(text);
+  c.beta = reinterpret_cast<float*>(take((size_t)lc.B * lc.F * lc.N * lc.H * 4));
+  c.beta_t = reinterpret_cast<float*>(take((size_t)lc.B * lc.T * lc.H * 4));
+  c.ws = take(vdn_workspace_bytes(&lc, dtype));
+  c.bytes = off;
+  return c;
+}
+
+// Default: about ten chunks. The first chunk's copy-in and the last chunk's
+// copy-out are not hidden, so smaller chunks shorten them; each chunk also
+// pays the latency-bound VDA kernels (about 0.7 ms, nearly independent of the
+// heads in the chunk), so chunks should not get too small.
+int effective_chunk(const vdn_layout_t* l, int head_chunk) {
+  if (head_chunk <= 0) head_chunk = (l->H + 9) / 10;
+  return head_chunk > l->H ? l->H : head_chunk;
+}
+
+// rows x width bytes, host rows at pitch hpitch, device rows packed.
+cudaError_t copy_in(void* dst, const void* src, size_t width, size_t hpitch, size_t rows,
+                    cudaStream_t st) {
+  if (rows == 0 || width == 0) return cudaSuccess;
+  return cudaMemcpy2DAsync(dst, width, src, hpitch, width, rows, cudaMemcpyHostToDevice, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t vdn_hybrid_host_workspace_bytes(const vdn_layout_t* layout, int dtype, int head_chunk) {
+  if (vdn_workspace_bytes(layout, dtype) == 0) return 0;
+  vdn_layout_t lc = *layout;
+  lc.H = effective_chunk(layout, head_chunk);
+  // alignment slack, the RMSNorm weight, two chunk buffers
+  return kAlignH + align_h((size_t)layout->d * 4) + 2 * carve_chunk(lc, dtype, nullptr).bytes;
+}
+
+int vdn_hybrid_attn_fwd_host(const vdn_layout_t* layout, int dtype, int head_chunk,
+                             const void* q, const void* k, const void* v, const void* k_text,
+                             const void* v_text, const float* beta, const float* beta_text,
+                             const void* g_soft, const void* g_lin, const float* rms_weight,
+                             float rms_eps, void* out, void* workspace, size_t workspace_bytes) {
+  if (!layout || layout->B < 1 || layout->F < 1 || layout->N < 1 || layout->T < 0 || layout->c < 1 ||
+      layout->H < 1 || layout->d < 1)
+    return VDN_ERR_INVALID;
+  const size_t need = vdn_hybrid_host_workspace_bytes(layout, dtype, head_chunk);
+  if (need == 0) return VDN_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !beta || !g_soft || !g_lin || !out) return VDN_ERR_INVALID;
+  if (layout->T > 0 && (!k_text || !v_text || !beta_text)) return VDN_ERR_INVALID;
+  if (!(rms_eps >= 0.f)) return VDN_ERR_INVALID;
+  if (!workspace || workspace_bytes < need) return VDN_ERR_WORKSPACE;
+
+  const int H = layout->H, d = layout->d, B = layout->B, T = layout->T;
+  const long long L = (long long)layout->F * layout->N;
+  const size_t es = elem_size(dtype);
+  const int hc_max = effective_chunk(layout, head_chunk);
+  const int n_chunks = (H + hc_max - 1) / hc_max;
+
+  vdn_layout_t lmax = *layout;
+  lmax.H = hc_max;
+  char* base = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(workspace) + kAlignH - 1) &
+                                       ~static_cast<uintptr_t>(kAlignH - 1));
+  float* rms_w_dev = rms_weight ? reinterpret_cast<float*>(base) : nullptr;
+  base += align_h((size_t)d * 4);
+  const size_t buf_bytes = carve_chunk(lmax, dtype, nullptr).bytes;
+
+  cudaStream_t s_in = nullptr, s_comp = nullptr, s_out = nullptr;
+  cudaEvent_t ev_in[2] = {nullptr, nullptr}, ev_comp[2] = {nullptr, nullptr}, ev_out[2] = {nullptr, nullptr};
+  int status = VDN_OK;
+  auto fail = [&](cudaError_t e) { if (e != cudaSuccess && status == VDN_OK) status = VDN_ERR_CUDA; };
+  fail(cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking));
+  fail(cudaStreamCreateWithFlags(&s_comp, cudaStreamNonBlocking));
+  fail(cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking));
+  for (int i = 0; i < 2; ++i) {
+    fail(cudaEventCreateWithFlags(&ev_in[i], cudaEventDisableTiming));
+    fail(cudaEventCreateWithFlags(&ev_comp[i], cudaEventDisableTiming));
+    fail(cudaEventCreateWithFlags(&ev_out[i], cudaEventDisableTiming));
+  }
+
+  if (rms_weight)
+    fail(cudaMemcpyAsync(rms_w_dev, rms_weight, (size_t)d * 4, cudaMemcpyHostToDevice, s_in));
+  for (int c = 0; c < n_chunks && status == VDN_OK; ++c) {
+    const int h0 = c * hc_max;
+    const int hc = (h0 + hc_max <= H) ? hc_max : H - h0;
+    const int slot = c & 1;
+    vdn_layout_t lc = *layout;
+    lc.H = hc;
+    const ChunkBuf buf = carve_chunk(lc, dtype, base + slot * buf_bytes);
+    // copy in, once the buffer's previous chunk has been copied out
+    if (c >= 2) fail(cudaStreamWaitEvent(s_in, ev_out[slot], 0));
+    const size_t w_vid = (size_t)hc * d * es, p_vid = (size_t)H * d * es, o_vid = (size_t)h0 * d * es;
+    const size_t rows_v = (size_t)B * L, rows_t = (size_t)B * T;
+    const char* src[5] = {static_cast<const char*>(q), static_cast<const char*>(k),
+                          static_cast<const char*>(v), static_cast<const char*>(g_soft),
+                          static_cast<const char*>(g_lin)};
+    char* dst[5] = {buf.q, buf.k, buf.v, buf.gs, buf.gl};
+    for (int t = 0; t < 5; ++t) fail(copy_in(dst[t], src[t] + o_vid, w_vid, p_vid, rows_v, s_in));
+    if (T > 0) {
+      fail(copy_in(buf.kt, static_cast<const char*>(k_text) + o_vid, w_vid, p_vid, rows_t, s_in));
+      fail(copy_in(buf.vt, static_cast<const char*>(v_text) + o_vid, w_vid, p_vid, rows_t, s_in));
+      fail(copy_in(buf.beta_t, beta_text + h0, (size_t)hc * 4, (size_t)H * 4, rows_t, s_in));
+    }
+    fail(copy_in(buf.beta, beta + h0, (size_t)hc * 4, (size_t)H * 4, rows_v, s_in));
+    fail(cudaEventRecord(ev_in[slot], s_in));
+    if (status != VDN_OK) break;
+    // compute
+    fail(cudaStreamWaitEvent(s_comp, ev_in[slot], 0));
+    const vdn_layout_t* lcp = &lc;
+    const int s = vdn_hybrid_attn_fwd(lcp, dtype, buf.q, buf.k, buf.v, T ? buf.kt : nullptr,
+                                      T ? buf.vt : nullptr, buf.beta, T ? buf.beta_t : nullptr, buf.gs,
+                                      buf.gl, rms_w_dev, rms_eps, buf.out, nullptr, nullptr, buf.ws,
+                                      vdn_workspace_bytes(lcp, dtype), s_comp);
+    if (s != VDN_OK) { status = s; break; }
+    fail(cudaEventRecord(ev_comp[slot], s_comp));
+    // copy out into the strided host tensor
+    fail(cudaStreamWaitEvent(s_out, ev_comp[slot], 0));
+    fail(cudaMemcpy2DAsync(static_cast<char*>(out) + o_vid, p_vid, buf.out, w_vid, w_vid, rows_v,
+                           cudaMemcpyDeviceToHost, s_out));
+    fail(cudaEventRecord(ev_out[slot], s_out));
+  }
+  // the call returns with the output in host memory (and nothing in flight)
+  for (cudaStream_t st : {s_in, s_comp, s_out})
+    if (st) fail(cudaStreamSynchronize(st));
+  for (int i = 0; i < 2; ++i) {
+    if (ev_in[i]) cudaEventDestroy(ev_in[i]);
+    if (ev_comp[i]) cudaEventDestroy(ev_comp[i]);
+    if (ev_out[i]) cudaEventDestroy(ev_out[i]);
+  }
+  for (cudaStream_t st : {s_in, s_comp, s_out})
+    if (st) cudaStreamDestroy(st);
+  return status;
+}
+
+}  // extern "C"

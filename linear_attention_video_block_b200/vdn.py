@@ -33,7 +33,8 @@ STATUS = {0: "VDN_OK", 1: "VDN_ERR_INVALID", 2: "VDN_ERR_UNSUPPORTED",
 EXPORTS = ("vdn_workspace_bytes", "vdn_window_softmax_fwd", "vdn_vda_scan_fwd",
            "vdn_vda_scan_fwd_decay", "vdn_hybrid_attn_fwd", "vdn_hybrid_attn_fwd_decay",
            "vdn_vda_scan_fwd_noalloc", "vdn_joint_softmax_fwd", "vdn_joint_attn_fwd",
-           "vdn_window_softmax_fwd_fp8", "vdn_device_status", "vdn_status_string",
+           "vdn_window_softmax_fwd_fp8", "vdn_hybrid_attn_fwd_host",
+           "vdn_hybrid_host_workspace_bytes", "vdn_device_status", "vdn_status_string",
            "vdn_last_cuda_error")
 
 
@@ -79,6 +80,10 @@ def lib():
                                                 + [P] * 3 + [P, S, P])
         L.vdn_hybrid_attn_fwd_decay.restype = I
         F = ctypes.c_float
+        L.vdn_hybrid_host_workspace_bytes.argtypes = [LP, I, I]
+        L.vdn_hybrid_host_workspace_bytes.restype = S
+        L.vdn_hybrid_attn_fwd_host.argtypes = [LP, I, I] + [P] * 10 + [F, P, P, S]
+        L.vdn_hybrid_attn_fwd_host.restype = I
         L.vdn_window_softmax_fwd_fp8.argtypes = [LP] + [P] * 5 + [F, F, F] + [P, P, P]
         L.vdn_window_softmax_fwd_fp8.restype = I
         CP = ctypes.POINTER(_CContext)
@@ -188,20 +193,17 @@ def hybrid_attn_fwd(layout: Layout, q, k, v, k_text, v_text, beta, beta_text, g_
     alpha (optional, [B, F, H, d] float32): KDA decay of the linear branch.
 
     Device tensors: launched asynchronously on the current stream; returns out.
-    Host tensors: copied to ``device`` (default cuda:0), computed, and the
-    result copied back to host memory (pinned inputs make the copies async).
+    Host tensors: vdn_hybrid_attn_fwd_host on ``device`` (default cuda:0), which
+    copies in, computes and copies out in pipelined head chunks; returns the
+    host output (pinned inputs let the copies overlap the kernels).
     """
     _require_cuda()
-    host = not q.is_cuda
-    out_host = None
-    if host:
-        dev = torch.device(device or "cuda:0")
-        out_host, out = out, None
-        if out_soft is not None or out_lin is not None:
-            raise ValueError("out_soft/out_lin need device tensors")
-        args = [q, k, v, k_text, v_text, beta, beta_text, g_soft, g_lin, rms_weight, alpha]
-        q, k, v, k_text, v_text, beta, beta_text, g_soft, g_lin, rms_weight, alpha = [
-            None if a is None else a.to(dev, non_blocking=True) for a in args]
+    if not q.is_cuda:
+        if out_soft is not None or out_lin is not None or alpha is not None:
+            raise ValueError("out_soft, out_lin and alpha need device tensors")
+        return hybrid_attn_fwd_host(layout, q, k, v, k_text, v_text, beta, beta_text, g_soft, g_lin,
+                                    rms_weight=rms_weight, rms_eps=rms_eps, out=out,
+                                    workspace=workspace, device=device)
     if out is None:
         out = torch.empty_like(q)
     if workspace is None:
@@ -216,12 +218,45 @@ def hybrid_attn_fwd(layout: Layout, q, k, v, k_text, v_text, beta, beta_text, g_
         code = lib().vdn_hybrid_attn_fwd_decay(*head, _ptr(alpha), *tail)
         name = "vdn_hybrid_attn_fwd_decay"
     _check(code, name)
-    if host:
-        if out_host is None:
-            out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-        out_host.copy_(out, non_blocking=True)
-        torch.cuda.current_stream(out.device).synchronize()
-        return out_host
+    return out
+
+
+def host_workspace_bytes(layout: Layout, dtype: torch.dtype, head_chunk: int = 0) -> int:
+    code = VDN_BF16 if dtype == torch.bfloat16 else VDN_F32
+    return int(lib().vdn_hybrid_host_workspace_bytes(ctypes.byref(_clayout(layout)), code, head_chunk))
+
+
+def _host_ptr(t):
+    if t is None:
+        return None
+    if t.is_cuda:
+        raise ValueError("tensor must live in host memory")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def hybrid_attn_fwd_host(layout: Layout, q, k, v, k_text, v_text, beta, beta_text, g_soft, g_lin,
+                         rms_weight=None, rms_eps=1e-6, out=None, head_chunk=0, workspace=None,
+                         device=None):
+    """The hybrid forward on host tensors (vdn_hybrid_attn_fwd_host): copies in,
+    computes and copies out in pipelined chunks of head_chunk heads (0: about
+    ten chunks). workspace: device uint8 tensor of host_workspace_bytes (made
+    here if None). Returns out, a host tensor (pinned when made here)."""
+    _require_cuda()
+    dev = torch.device(device or "cuda:0")
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    with torch.cuda.device(dev):
+        if workspace is None:
+            workspace = torch.empty(host_workspace_bytes(layout, q.dtype, head_chunk), dtype=torch.uint8,
+                                    device=dev)
+        code = lib().vdn_hybrid_attn_fwd_host(
+            ctypes.byref(_clayout(layout)), _dtype_code(q), head_chunk, _host_ptr(q), _host_ptr(k),
+            _host_ptr(v), _host_ptr(k_text), _host_ptr(v_text), _host_ptr(beta), _host_ptr(beta_text),
+            _host_ptr(g_soft), _host_ptr(g_lin), _host_ptr(rms_weight), ctypes.c_float(rms_eps),
+            _host_ptr(out), _ptr(workspace), workspace.numel())
+    _check(code, "vdn_hybrid_attn_fwd_host")
     return out
 
 

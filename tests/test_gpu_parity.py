@@ -261,3 +261,21 @@ def test_unit_decay_is_bit_identical_to_no_decay():
     ha = vdn.hybrid_attn_fwd(*args, d["g_s"], d["g_l"])
     hb = vdn.hybrid_attn_fwd(*args, d["g_s"], d["g_l"], alpha=ones)
     assert torch.equal(ha, hb)
+
+
+@pytest.mark.parametrize("head_chunk", [1, 3, 0])
+def test_host_pipeline_chunks_match_device_path(head_chunk):
+    """vdn_hybrid_attn_fwd_host in head chunks (3 of 4 heads: a ragged last
+    chunk; 1: one head per chunk; 0: automatic) with an RMSNorm weight equals
+    the device entry bit for bit (the heads are independent)."""
+    layout, dtype, seed = WORKLOADS["small-bf16"]
+    inp = make_inputs(layout, dtype, seed)
+    host = {k: v.pin_memory() for k, v in inp.items()}
+    w = torch.linspace(0.5, 1.5, layout.d, dtype=torch.float32)
+    out_h = vdn.hybrid_attn_fwd_host(layout, host["q"], host["k"], host["v"], host["k_text"],
+                                     host["v_text"], host["beta"], host["beta_text"], host["g_s"],
+                                     host["g_l"], rms_weight=w, rms_eps=1e-5, head_chunk=head_chunk)
+    d = _dev(inp)
+    out_d = vdn.hybrid_attn_fwd(layout, d["q"], d["k"], d["v"], d["k_text"], d["v_text"], d["beta"],
+                                d["beta_text"], d["g_s"], d["g_l"], rms_weight=w.cuda(), rms_eps=1e-5)
+    assert torch.equal(out_h, out_d.cpu())

@@ -299,3 +299,18 @@ def test_fp8_entry_validates(lib):
     assert f(ctypes.byref(ok), *args, F(1), F(1), F(1), None, None, None) == 1
     assert f(ctypes.byref(ok), MISALIGNED, *args[1:], F(1), F(1), F(1), FAKE, None, None) == 2
     assert f(ctypes.byref(_layout(d=128, B=0)), *args, F(1), F(1), F(1), FAKE, None, None) == 1
+
+
+def test_host_pipeline_entry_validates(lib):
+    """vdn_hybrid_attn_fwd_host rejects before any copy or launch."""
+    f = lib.vdn_hybrid_attn_fwd_host
+    ok = _layout()
+    need = lib.vdn_hybrid_host_workspace_bytes(ctypes.byref(ok), 0, 0)
+    assert need > lib.vdn_workspace_bytes(ctypes.byref(ok), 0)
+    args = [FAKE] * 9 + [None, ctypes.c_float(1e-6), FAKE, FAKE]
+    assert f(ctypes.byref(_layout(B=0)), 0, 0, *args, need) == 1
+    assert f(ctypes.byref(_layout(d=48)), 0, 0, *args, need) == 2
+    assert f(ctypes.byref(ok), 5, 0, *args, need) == 2
+    assert f(ctypes.byref(ok), 0, 0, *args, need - 1) == 3
+    assert f(ctypes.byref(ok), 0, 0, None, *args[1:], need) == 1
+    assert f(ctypes.byref(ok), 0, 0, *args[:10], ctypes.c_float(-1.0), FAKE, FAKE, need) == 1
