@@ -51,13 +51,54 @@ ChunkBuf carve_chunk(const vdn_layout_t& lc, int dtype, char* base) {
   return c;
 }
 
-// Default: about ten chunks. The first chunk's copy-in and the last chunk's
-// copy-out are not hidden, so smaller chunks shorten them; each chunk also
-// pays the latency-bound VDA kernels (about 0.7 ms, nearly independent of the
-// heads in the chunk), so chunks should not get too small.
-int effective_chunk(const vdn_layout_t* l, int head_chunk) {
-  if (head_chunk <= 0) head_chunk = (l->H + 9) / 10;
-  return head_chunk > l->H ? l->H : head_chunk;
+// Chunk sizes. Given head_chunk > 0: uniform. Default: the first chunk's
+// copy-in and the last chunk's copy-out are the only copies not hidden, so the
+// chunks grow from one head (each copy-in must fit under the previous chunk's
+// kernels: a head's inputs take about 3/4 of its compute time over PCIe, so a
+// chunk may be about a third larger than the one before), stay at up to
+// about an eighth of the heads, and shrink back to one head at the end; each
+// chunk also pays the latency-bound VDA kernels, so they do not get smaller.
+constexpr int kMaxChunks = 64;
+int chunk_plan(const vdn_layout_t* l, int head_chunk, int* sizes) {
+  const int H = l->H;
+  if (head_chunk > 0) {
+    const int hc = head_chunk > H ? H : head_chunk;
+    int n = 0;
+    for (int h0 = 0; h0 < H && n < kMaxChunks; h0 += hc) sizes[n++] = (h0 + hc <= H) ? hc : H - h0;
+    if (n == kMaxChunks) return -1;
+    return n;
+  }
+  const int cap = (H + 7) / 8;
+  int head[kMaxChunks], tail[kMaxChunks], nh = 0, nt = 0, left = H;
+  // grow from both ends, one head at the ends, about a third more each step
+  int s = 1;
+  while (left > 0 && nh + nt < kMaxChunks - 1) {
+    const int a = s < left ? s : left;
+    head[nh++] = a;
+    left -= a;
+    if (left <= 0) break;
+    const int b = s < left ? s : left;
+    tail[nt++] = b;
+    left -= b;
+    if (s >= cap) break;
+    s = (s * 4 + 2) / 3 > s ? (s * 4 + 2) / 3 : s + 1;
+    if (s > cap) s = cap;
+  }
+  int n = 0;
+  for (int i = 0; i < nh; ++i) sizes[n++] = head[i];
+  while (left > 0 && n < kMaxChunks - nt) {
+    const int a = cap < left ? cap : left;
+    sizes[n++] = a;
+    left -= a;
+  }
+  for (int i = nt - 1; i >= 0; --i) sizes[n++] = tail[i];
+  return left == 0 ? n : -1;
+}
+
+int max_chunk(const int* sizes, int n) {
+  int m = 0;
+  for (int i = 0; i < n; ++i) m = sizes[i] > m ? sizes[i] : m;
+  return m;
 }
 
 // rows x width bytes, host rows at pitch hpitch, device rows packed.
@@ -73,8 +114,11 @@ extern "C" {
 
 size_t vdn_hybrid_host_workspace_bytes(const vdn_layout_t* layout, int dtype, int head_chunk) {
   if (vdn_workspace_bytes(layout, dtype) == 0) return 0;
+  int sizes[kMaxChunks];
+  const int n = chunk_plan(layout, head_chunk, sizes);
+  if (n <= 0) return 0;
   vdn_layout_t lc = *layout;
-  lc.H = effective_chunk(layout, head_chunk);
+  lc.H = max_chunk(sizes, n);
   // alignment slack, the RMSNorm weight, two chunk buffers
   return kAlignH + align_h((size_t)layout->d * 4) + 2 * carve_chunk(lc, dtype, nullptr).bytes;
 }
@@ -97,8 +141,9 @@ int vdn_hybrid_attn_fwd_host(const vdn_layout_t* layout, int dtype, int head_chu
   const int H = layout->H, d = layout->d, B = layout->B, T = layout->T;
   const long long L = (long long)layout->F * layout->N;
   const size_t es = elem_size(dtype);
-  const int hc_max = effective_chunk(layout, head_chunk);
-  const int n_chunks = (H + hc_max - 1) / hc_max;
+  int sizes[kMaxChunks];
+  const int n_chunks = chunk_plan(layout, head_chunk, sizes);
+  const int hc_max = max_chunk(sizes, n_chunks);
 
   vdn_layout_t lmax = *layout;
   lmax.H = hc_max;
@@ -123,9 +168,9 @@ int vdn_hybrid_attn_fwd_host(const vdn_layout_t* layout, int dtype, int head_chu
 
   if (rms_weight)
     fail(cudaMemcpyAsync(rms_w_dev, rms_weight, (size_t)d * 4, cudaMemcpyHostToDevice, s_in));
-  for (int c = 0; c < n_chunks && status == VDN_OK; ++c) {
-    const int h0 = c * hc_max;
-    const int hc = (h0 + hc_max <= H) ? hc_max : H - h0;
+  int h0 = 0;
+  for (int c = 0; c < n_chunks && status == VDN_OK; h0 += sizes[c], ++c) {
+    const int hc = sizes[c];
     const int slot = c & 1;
     vdn_layout_t lc = *layout;
     lc.H = hc;
