@@ -6,7 +6,9 @@
 // CTA = one (b, h, slot); 192 threads:
 //   warp 0     TMA producer: 32-token K and V tiles into a ring of stages
 //   warp 1     MMA issuer (one lane) and TMEM owner
-//   warps 2-5  scalers: write Kw = beta (.) K next to K as two bf16 parts,
+//   warps 2-5  scalers: write Kw = beta (.) K into a ring of two Kw slots
+//              (separate from the K/V ring, so that more K/V tiles are in
+//              flight in the same shared memory) as two bf16 parts,
 //              Kw_hi = bf16(beta k) and Kw_lo = bf16(beta k - Kw_hi), so that the
 //              products keep ~16 significant bits of beta k (a single bf16 copy
 //              put the chunk states 1e-2 off); four threads per token row, beta
@@ -43,16 +45,19 @@ template <int D>
 struct GCfg {
   static constexpr int kHalves = D / 64;
   static constexpr int kTileBytes = kTok * D * 2;
-  static constexpr int kStageBytes = 4 * kTileBytes;          // K, V, Kw_hi, Kw_lo
-  static constexpr int kStages = (D == 128) ? 3 : 6;
+  static constexpr int kStageBytes = 2 * kTileBytes;          // K, V
+  static constexpr int kStages = (D == 128) ? 4 : 8;
+  static constexpr int kKwBytes = 2 * kTileBytes;             // Kw_hi, Kw_lo
+  static constexpr int kKwSlots = 2;
   static constexpr int kTmemCols = (D == 128) ? 256 : 64;
-  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 256;
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kKwSlots * kKwBytes + 256;
 };
 
 struct GBars {
-  unsigned long long full[8];
-  unsigned long long scaled[8];
-  unsigned long long empty[8];
+  unsigned long long full[8];        // K/V stage loaded
+  unsigned long long empty[8];       // K/V stage consumed by the MMAs
+  unsigned long long kw_full[2];     // Kw slot written by the scalers
+  unsigned long long kw_empty[2];    // Kw slot consumed by the MMAs
   unsigned long long done;
   uint32_t tmem_base;
   int abort;
@@ -93,7 +98,8 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  GBars* bars = reinterpret_cast<GBars*>(smem + C::kStages * C::kStageBytes);
+  uint8_t* sKw = smem + C::kStages * C::kStageBytes;
+  GBars* bars = reinterpret_cast<GBars*>(sKw + C::kKwSlots * C::kKwBytes);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int h = blockIdx.y, b = blockIdx.z;
   const bool text = slots.has_text && blockIdx.x == 0;
@@ -105,8 +111,11 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&bars->full[s], 1);
-      mbar_init(&bars->scaled[s], 128);
       mbar_init(&bars->empty[s], 1);
+    }
+    for (int j = 0; j < C::kKwSlots; ++j) {
+      mbar_init(&bars->kw_full[j], 128);
+      mbar_init(&bars->kw_empty[j], 1);
     }
     mbar_init(&bars->done, 1);
     bars->abort = 0;
@@ -160,13 +169,16 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       constexpr uint32_t idesc = idesc_mn_mn(D);
       bool ok = true;
       for (int t = 0; t < n_tiles && ok; ++t) {
-        const int s = t % C::kStages, use = t / C::kStages;
-        if (!gwait(&bars->scaled[s], use & 1, abort)) {
+        const int s = t % C::kStages;
+        const int j = t % C::kKwSlots, juse = t / C::kKwSlots;
+        // the scalers wrote Kw of tile t after its K/V stage had landed
+        if (!gwait(&bars->kw_full[j], juse & 1, abort)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t st = smem_u32(smem + s * C::kStageBytes);
+        const uint32_t kw = smem_u32(sKw + j * C::kKwBytes);
         const uint32_t k_addr = st, v_addr = st + C::kTileBytes;
 #pragma unroll
         for (int ks = 0; ks < kTok / 16; ++ks) {
@@ -174,7 +186,7 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
 #pragma unroll
           for (int part = 0; part < 2; ++part) {
             const uint32_t acc = (t > 0 || ks > 0 || part > 0) ? 1u : 0u;
-            const uint64_t bdesc = desc_mn_sw128(st + (2 + part) * C::kTileBytes + koff, kHalfBytes);
+            const uint64_t bdesc = desc_mn_sw128(kw + part * C::kTileBytes + koff, kHalfBytes);
             if (D == 128) {
               mma_ss(tmem, desc_mn_sw128(k_addr + koff, kHalfBytes), bdesc, idesc, acc);
               mma_ss(tmem + 128, desc_mn_sw128(v_addr + koff, kHalfBytes), bdesc, idesc, acc);
@@ -185,6 +197,7 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
           }
         }
         tc_commit(&bars->empty[s]);
+        tc_commit(&bars->kw_empty[j]);
       }
       tc_commit(&bars->done);
       if (!ok) gwait(&bars->done, 0, abort, false);
@@ -207,13 +220,20 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     bool ok = true;
     for (int t = 0; t < n_tiles && ok; ++t) {
       const int s = t % C::kStages, use = t / C::kStages;
+      const int j = t % C::kKwSlots, juse = t / C::kKwSlots;
       const float bu = bnext;
       if (t + 1 < n_tiles) bnext = beta_of(t + 1);
       if (!__all_sync(0xffffffffu, gwait(&bars->full[s], use & 1, abort))) {
         ok = false;
         break;
       }
+      // the Kw slot is free once the MMAs of tile t - kKwSlots have completed
+      if (juse > 0 && !__all_sync(0xffffffffu, gwait(&bars->kw_empty[j], (juse - 1) & 1, abort))) {
+        ok = false;
+        break;
+      }
       uint8_t* st = smem + s * C::kStageBytes;
+      uint8_t* kwp = sKw + j * C::kKwBytes;
 #pragma unroll
       for (int cc = 0; cc < kCpt; ++cc) {
         const int chunk = part * kCpt + cc;       // 0 .. D/8 - 1 within the row
@@ -232,11 +252,11 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
           hi4[e] = pack_bf16(h0, h1);
           lo4[e] = pack_bf16(p0 - h0, p1 - h1);
         }
-        *reinterpret_cast<uint4*>(st + 2 * C::kTileBytes + off) = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
-        *reinterpret_cast<uint4*>(st + 3 * C::kTileBytes + off) = make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
+        *reinterpret_cast<uint4*>(kwp + off) = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
+        *reinterpret_cast<uint4*>(kwp + C::kTileBytes + off) = make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive(&bars->scaled[s]);
+      mbar_arrive(&bars->kw_full[j]);
     }
     if (ok) ok = __all_sync(0xffffffffu, gwait(&bars->done, 0, abort));
     if (ok) {
