@@ -279,3 +279,18 @@ def test_host_pipeline_chunks_match_device_path(head_chunk):
     out_d = vdn.hybrid_attn_fwd(layout, d["q"], d["k"], d["v"], d["k_text"], d["v_text"], d["beta"],
                                 d["beta_text"], d["g_s"], d["g_l"], rms_weight=w.cuda(), rms_eps=1e-5)
     assert torch.equal(out_h, out_d.cpu())
+
+
+def test_host_pipeline_batch_and_ragged_text():
+    """Host-buffer entry with B = 2, ragged N and T and a ragged last head chunk
+    (3 heads in chunks of 2) equals the device entry bit for bit."""
+    layout = Layout(B=2, F=7, N=200, T=130, c=1, H=3, d=128)
+    inp = make_inputs(layout, "bf16", 77)
+    host = {k: v.pin_memory() for k, v in inp.items()}
+    out_h = vdn.hybrid_attn_fwd_host(layout, host["q"], host["k"], host["v"], host["k_text"],
+                                     host["v_text"], host["beta"], host["beta_text"], host["g_s"],
+                                     host["g_l"], head_chunk=2)
+    d = _dev(inp)
+    out_d = vdn.hybrid_attn_fwd(layout, d["q"], d["k"], d["v"], d["k_text"], d["v_text"], d["beta"],
+                                d["beta_text"], d["g_s"], d["g_l"])
+    assert torch.equal(out_h, out_d.cpu())
