@@ -41,3 +41,43 @@ def bf16_storage_ratio(got, ref, allowance=4e-3, rms=None):
         rms = np.sqrt(np.mean(ref[m] ** 2))
     bound = 2.0 ** -8 * np.abs(ref[m]) + allowance * max(rms, 1e-300)
     return float(np.max(np.abs(got[m] - ref[m]) / bound))
+
+
+# The stated tolerance on the output of the op for bf16 inputs with float32
+# accumulation: max |err| / RMS(out) <= 2e-2.
+OUT_TOL_BF16 = 2e-2
+
+
+def bf16_rounding_floor(ref):
+    """max|round_bf16(ref) - ref| / RMS(ref): the error that storing the exact
+    result in bf16 alone carries (no arithmetic error at all)."""
+    import numpy as np
+    import torch
+    ref = np.asarray(ref, dtype=np.float64)
+    r32 = torch.from_numpy(np.nan_to_num(ref).astype(np.float32))
+    rounded = r32.to(torch.bfloat16).to(torch.float64).numpy()
+    rounded[np.isnan(ref)] = np.nan
+    return rel_err(rounded, ref)
+
+
+def check_out_bf16(got, ref, res, key="out"):
+    """The bf16 criterion on the op's output. Asserts the raw max|err|/RMS <=
+    2e-2. Only where rounding the oracle's own output to bf16 already exceeds
+    2e-2 (a few small edge layouts whose outputs have a heavy tail) is the
+    raw figure out of reach for any bf16 result; there the same 2e-2 is
+    applied beyond that rounding, per element: |got - ref| <= 2^-8 |ref| +
+    2e-2 RMS(ref). Records the raw figure, the floor and which rule applied in
+    res."""
+    floor = bf16_rounding_floor(ref)
+    raw = rel_err(got, ref)
+    res[key] = raw
+    res[key + "_bf16_floor"] = floor
+    if floor <= OUT_TOL_BF16:
+        res[key + "_rule"] = "raw"
+        assert raw <= OUT_TOL_BF16, (key, raw, floor)
+    else:
+        res[key + "_rule"] = "beyond-rounding"
+        ratio = bf16_storage_ratio(got, ref, allowance=OUT_TOL_BF16)
+        print(f"{key}: bf16 rounding floor {floor:.4f} > {OUT_TOL_BF16}; raw {raw:.4f}; "
+              f"ratio to the bound beyond rounding {ratio:.3f}")
+        assert ratio <= 1.0, (key, raw, floor, ratio)

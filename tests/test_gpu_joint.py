@@ -4,8 +4,11 @@ vdn_joint_attn_fwd) against the float64 oracle on the same seeded inputs.
 Video rows: the softmax branch also sees every audio key; the linear branch is
 unchanged (audio is never written into the VDA states). Text and audio query
 rows: the dense softmax over every video, text and audio key. Bounds as in
-test_gpu_parity: fp32 max|err|/RMS <= 1e-4; bf16 results held to 2e-2 RMS
-beyond their own storage rounding; lse <= 1e-3 absolute (1e-4 for fp32).
+test_gpu_parity: fp32 max|err|/RMS <= 1e-4; the bf16 output `out` to a raw
+max|err|/RMS(out) <= 2e-2 wherever rounding the exact result to bf16 stays
+within 2e-2 (the 480p-like and 768p-like layers assert that this raw rule
+applied), the other bf16 results to 2e-2 RMS beyond their own storage
+rounding; lse <= 1e-3 absolute (1e-4 for fp32).
 """
 
 import numpy as np
@@ -17,7 +20,7 @@ from linear_attention_video_block_b200.synth import (Layout, WORKLOADS, audio_to
                                                      make_decay, make_inputs)
 from oracle import vdn_oracle as O
 
-from conftest import bf16_storage_ratio, rel_err
+from conftest import bf16_storage_ratio, check_out_bf16, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -87,19 +90,22 @@ def _check_joint(layout, dtype, inp, cx, heads=None, rows=None, alpha=None, text
         lses[name.replace("o_", "lse_")] = (lse, rl)
     rms_out = float(np.sqrt(np.nanmean(ref_out ** 2)))
     res = {}
+    if dtype == "bf16":
+        # the op's output: raw max|err|/RMS <= 2e-2 (see check_out_bf16)
+        check_out_bf16(_np(out, hsel), ref_out, res)
     for key, (g, r, scale_of) in comp.items():
         gv = _np(g, hsel)
         res[key] = rel_err(gv, r)
-        if dtype == "bf16":
+        if dtype == "bf16" and key != "out":
             res[key + "_storage_ratio"] = bf16_storage_ratio(
                 gv, r, allowance=2e-2, rms=rms_out if scale_of == "out" else None)
     for key, (g, r) in lses.items():
         res[key] = float(np.nanmax(np.abs(g.cpu().double().numpy()[:, :, hsel] - r)))
-    print(layout, dtype, {k: round(v, 6) for k, v in res.items()})
+    print(layout, dtype, {k: (round(v, 6) if isinstance(v, float) else v) for k, v in res.items()})
     for key in comp:
         if dtype == "f32":
             assert res[key] <= 1e-4, (key, res)
-        else:
+        elif key != "out":
             assert res[key + "_storage_ratio"] <= 1.0, (key, res)
     for key in lses:
         assert res[key] <= (1e-4 if dtype == "f32" else 1e-3), (key, res)
@@ -145,8 +151,10 @@ def test_joint_full_size_sampled(name):
     {0, H-1}."""
     layout, dtype, seed = WORKLOADS[name]
     A = audio_tokens(layout.F)
-    _check_joint(layout, dtype, make_inputs(layout, dtype, seed), make_context(layout, A, dtype, seed + 7),
-                 heads=[0, layout.H - 1], rows=_sample_rows(layout, 12))
+    res = _check_joint(layout, dtype, make_inputs(layout, dtype, seed),
+                       make_context(layout, A, dtype, seed + 7), heads=[0, layout.H - 1],
+                       rows=_sample_rows(layout, 12))
+    assert res["out_rule"] == "raw"
 
 
 def test_joint_without_context_is_the_plain_hybrid():

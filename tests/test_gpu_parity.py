@@ -2,18 +2,19 @@
 the same seeded inputs.
 
 Bounds. Float32 workloads: max |gpu - oracle| / RMS(oracle) <= 1e-4 for the
-hybrid output and every intermediate. Bf16 workloads store their results in
-bf16, whose rounding alone (half an ulp, up to 2^-8 |x|) puts max|err|/RMS at
-1.4e-2 .. 2.4e-2 on these distributions (measured by rounding the oracle's own
-output), above the 2e-2 target on some layouts. So every bf16 result (out,
-o_soft, o_lin, the gated branches) is held to the 2e-2 target on the error
-beyond its own storage rounding: per element |gpu - oracle| <= 2^-8 |oracle|
-+ 2e-2 RMS (RMS of `out` for its two gated summands, of the result itself
-otherwise): the 2e-2 target applied to what remains after the half-ulp
-rounding that every bf16 output carries. The raw max|err|/RMS is printed
-beside it. The observed excess is 0.2e-2 .. 1.1e-2 RMS, largest where the
-softmax weights P, which enter the tensor cores in bf16, round alike
-(repeated keys). The fp32 chunk states meet 1e-3 relative (1e-4 for f32).
+hybrid output and every intermediate. Bf16 workloads: the hybrid output `out`
+is held to the stated max|err|/RMS(out) <= 2e-2 as a raw figure on every
+layout where that is reachable at all, i.e. where rounding the oracle's own
+output to bf16 stays within 2e-2 (all five named workloads, the decayed and
+joint layers among them; observed 0.0146 .. 0.0152). Where that rounding alone
+exceeds 2e-2 (a few small edge layouts, e.g. F = 3), the same 2e-2 applies to
+the error beyond the half-ulp rounding: per element |gpu - oracle| <=
+2^-8 |oracle| + 2e-2 RMS, and the test prints the floor. The intermediates
+(o_soft, o_lin and the two gated branches) are bf16 results too; their
+rounding floor reaches 2e-2 on the long workloads (o_lin), so they are held
+to the bound beyond rounding (RMS of `out` for the two gated summands of
+`out`), their raw figure printed beside it. The fp32 chunk states meet 1e-3
+relative (1e-4 for f32).
 
 Small workloads are checked element by element in full. At the full workload
 sizes the softmax branch is checked on sampled query rows of sampled heads
@@ -29,7 +30,7 @@ from linear_attention_video_block_b200 import vdn
 from linear_attention_video_block_b200.synth import Layout, WORKLOADS, make_decay, make_inputs
 from oracle import vdn_oracle as O
 
-from conftest import bf16_storage_ratio, rel_err
+from conftest import bf16_storage_ratio, check_out_bf16, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -102,9 +103,12 @@ def _check_all(layout, dtype, inp, heads=None, rows=None, alpha=None):
     comp = {"out": (out, ref_out), "o_soft": (o_soft, ref_soft), "o_lin": (o_lin, ref_lin),
             "out_soft": (out_soft, ref_gs), "out_lin": (out_lin, ref_gl)}
     rms_out = float(np.sqrt(np.nanmean(ref_out ** 2)))
+    if dtype == "bf16":
+        # the op's output: raw max|err|/RMS <= 2e-2 (see check_out_bf16)
+        check_out_bf16(_np(out, hsel), ref_out, res)
     for key, (g, r) in comp.items():
         res[key] = rel_err(_np(g, hsel), r)
-        if dtype == "bf16":
+        if dtype == "bf16" and key != "out":
             scale = rms_out if key in ("out_soft", "out_lin") else None
             res[key + "_storage_ratio"] = bf16_storage_ratio(_np(g, hsel), r, allowance=2e-2, rms=scale)
     res["lse"] = float(np.nanmax(np.abs(lse.cpu().double().numpy()[:, :, hsel] - ref_lse)))
@@ -130,11 +134,11 @@ def _check_all(layout, dtype, inp, heads=None, rows=None, alpha=None):
     for key in comp:
         if dtype == "f32":
             assert res[key] <= tol, (key, res)
-        else:
+        elif key != "out":
             assert res[key + "_storage_ratio"] <= 1.0, (key, res)
     assert res["lse"] <= (1e-4 if dtype == "f32" else 1e-3), res
     print(name_of(layout), dtype, "decay" if alpha is not None else "",
-          {k: round(v, 6) for k, v in res.items()})
+          {k: (round(v, 6) if isinstance(v, float) else v) for k, v in res.items()})
     return res
 
 
@@ -142,21 +146,25 @@ def _check_all(layout, dtype, inp, heads=None, rows=None, alpha=None):
 def test_small_workloads_full(name):
     layout, dtype, seed = WORKLOADS[name]
     inp = make_inputs(layout, dtype, seed)
-    _check_all(layout, dtype, inp)
+    res = _check_all(layout, dtype, inp)
+    if dtype == "bf16":
+        assert res["out_rule"] == "raw"
 
 
 @pytest.mark.parametrize("repeated", [False, True])
 def test_480p_like(repeated):
     layout, dtype, seed = WORKLOADS["480p-bf16"]
     inp = make_inputs(layout, dtype, seed, repeated_keys=repeated)
-    _check_all(layout, dtype, inp, heads=[0, layout.H - 1], rows=_sample_rows(layout, 32))
+    res = _check_all(layout, dtype, inp, heads=[0, layout.H - 1], rows=_sample_rows(layout, 32))
+    assert res["out_rule"] == "raw"
 
 
 @pytest.mark.parametrize("name", ["768p-bf16", "long-bf16"])
 def test_full_size_sampled(name):
     layout, dtype, seed = WORKLOADS[name]
     inp = make_inputs(layout, dtype, seed)
-    _check_all(layout, dtype, inp, heads=[0, layout.H - 1], rows=_sample_rows(layout, 24))
+    res = _check_all(layout, dtype, inp, heads=[0, layout.H - 1], rows=_sample_rows(layout, 24))
+    assert res["out_rule"] == "raw"
 
 
 EDGE = [
@@ -192,7 +200,7 @@ def test_rms_weight_and_eps():
     ref = O.hybrid(a["q"], a["k"], a["v"], a["k_text"], a["v_text"], a["beta"], a["beta_text"],
                    a["g_s"], a["g_l"], layout.F, layout.N, layout.c, eps=1e-3,
                    weight=w.cpu().double().numpy())["out"]
-    assert rel_err(_np(out), ref) <= TOL["bf16"]
+    check_out_bf16(_np(out), ref, {})
 
 
 def test_host_buffers_public_api():
@@ -244,8 +252,9 @@ def test_decay_small_full(name, layout):
 def test_decay_full_size_sampled(name):
     layout, dtype, seed = WORKLOADS[name]
     inp = make_inputs(layout, dtype, seed)
-    _check_all(layout, dtype, inp, heads=[0, layout.H - 1], rows=_sample_rows(layout, 16),
-               alpha=make_decay(layout, seed + 1))
+    res = _check_all(layout, dtype, inp, heads=[0, layout.H - 1], rows=_sample_rows(layout, 16),
+                     alpha=make_decay(layout, seed + 1))
+    assert res["out_rule"] == "raw"
 
 
 def test_unit_decay_is_bit_identical_to_no_decay():
