@@ -116,6 +116,76 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
+def _expect(name, t, shape, dtype=None, required=True):
+    """Checks one tensor argument against the layout before anything reaches
+    the library: the kernels build their TMA tensor maps and index arithmetic
+    from the layout alone, so a tensor of another shape would be read or
+    written out of bounds on the device."""
+    if t is None:
+        if required:
+            raise ValueError(f"{name} is required")
+        return
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}; the layout needs {tuple(shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}; expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _same_device(*ts):
+    devs = {t.device for t in ts if t is not None}
+    if len(devs) > 1:
+        raise ValueError(f"tensors on several devices: {sorted(str(d) for d in devs)}")
+
+
+def _io_dtype(q):
+    if q is None:
+        raise ValueError("q is required")
+    if q.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError(f"unsupported dtype {q.dtype}; float32 or bfloat16")
+    return q.dtype
+
+
+def _validate(layout: Layout, q=None, io=(), text=(), beta=None, beta_text=None, alpha=None,
+              rms_weight=None, lse=None, chunk_states=None, io_dtype=None, optional_io=(),
+              text_dtype=None):
+    """Shape, dtype and device checks of the common arguments. io / optional_io:
+    (name, tensor) pairs of [B, L, H, d] tensors in the io dtype (required /
+    nullable); text: (name, tensor) pairs of [B, T, H, d] tensors (required
+    when T > 0)."""
+    B, F, N, T, c, H, d = layout.B, layout.F, layout.N, layout.T, layout.c, layout.H, layout.d
+    L = F * N
+    dt = io_dtype if io_dtype is not None else _io_dtype(q)
+    video = (B, L, H, d)
+    _expect("q", q, video, dt)
+    for name, t in io:
+        _expect(name, t, video, dt)
+    for name, t in optional_io:
+        _expect(name, t, video, dt, required=False)
+    for name, t in text:
+        _expect(name, t, (B, T, H, d), text_dtype or dt, required=T > 0)
+    _expect("beta", beta, (B, L, H), torch.float32, required=False)
+    _expect("beta_text", beta_text, (B, T, H), torch.float32, required=False)
+    _expect("alpha", alpha, (B, F, H, d), torch.float32, required=False)
+    _expect("rms_weight", rms_weight, (d,), torch.float32, required=False)
+    _expect("lse", lse, (B, L, H), torch.float32, required=False)
+    J = -(-F // c) if c > 0 else 0
+    _expect("chunk_states", chunk_states, (B, H, 2, J, d, d), torch.float32, required=False)
+    _same_device(q, *(t for _, t in io), *(t for _, t in optional_io), *(t for _, t in text), beta,
+                 beta_text, alpha, rms_weight, lse, chunk_states)
+
+
+def _validate_workspace(workspace, q):
+    if workspace is None:
+        return
+    if workspace.dtype != torch.uint8 or workspace.dim() != 1 or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous 1-D torch.uint8 tensor")
+    _same_device(q, workspace)
+
+
 def _ptr(t):
     if t is None:
         return None
@@ -148,6 +218,8 @@ def workspace_bytes(layout: Layout, dtype: torch.dtype) -> int:
 def window_softmax_fwd(layout: Layout, q, k, v, k_text, v_text, o_soft=None, lse=None,
                        want_lse=False):
     """Softmax branch: returns o_soft (and lse [B, L, H] if want_lse)."""
+    _validate(layout, q, io=[("k", k), ("v", v)], optional_io=[("o_soft", o_soft)],
+              text=[("k_text", k_text), ("v_text", v_text)], lse=lse)
     _require_cuda()
     if o_soft is None:
         o_soft = torch.empty_like(q)
@@ -165,6 +237,13 @@ def vda_scan_fwd(layout: Layout, q, k, v, k_text, v_text, beta, beta_text, o_lin
     """Linear branch: returns o_lin (ungated, pre-norm) and, if want_states, the
     chunk table [B, H, 2, J, d, d] float32. alpha (optional, [B, F, H, d]
     float32) decays the state per key channel before each frame's write."""
+    _validate(layout, q, io=[("k", k), ("v", v)], optional_io=[("o_lin", o_lin)],
+              text=[("k_text", k_text), ("v_text", v_text)], beta=beta, beta_text=beta_text,
+              alpha=alpha, chunk_states=chunk_states)
+    _expect("beta", beta, (layout.B, layout.F * layout.N, layout.H), torch.float32)
+    _expect("beta_text", beta_text, (layout.B, layout.T, layout.H), torch.float32,
+            required=layout.T > 0)
+    _validate_workspace(workspace, q)
     _require_cuda()
     if o_lin is None:
         o_lin = torch.empty_like(q)
@@ -197,6 +276,14 @@ def hybrid_attn_fwd(layout: Layout, q, k, v, k_text, v_text, beta, beta_text, g_
     copies in, computes and copies out in pipelined head chunks; returns the
     host output (pinned inputs let the copies overlap the kernels).
     """
+    _validate(layout, q, io=[("k", k), ("v", v), ("g_soft", g_soft), ("g_lin", g_lin)],
+              optional_io=[("out", out), ("out_soft", out_soft), ("out_lin", out_lin)],
+              text=[("k_text", k_text), ("v_text", v_text)], beta=beta, beta_text=beta_text,
+              alpha=alpha, rms_weight=rms_weight)
+    _expect("beta", beta, (layout.B, layout.F * layout.N, layout.H), torch.float32)
+    _expect("beta_text", beta_text, (layout.B, layout.T, layout.H), torch.float32,
+            required=layout.T > 0)
+    _validate_workspace(workspace, q)
     _require_cuda()
     if not q.is_cuda:
         if out_soft is not None or out_lin is not None or alpha is not None:
@@ -243,6 +330,12 @@ def hybrid_attn_fwd_host(layout: Layout, q, k, v, k_text, v_text, beta, beta_tex
     computes and copies out in pipelined chunks of head_chunk heads (0: about
     ten chunks). workspace: device uint8 tensor of host_workspace_bytes (made
     here if None). Returns out, a host tensor (pinned when made here)."""
+    _validate(layout, q, io=[("k", k), ("v", v), ("g_soft", g_soft), ("g_lin", g_lin)],
+              optional_io=[("out", out)], text=[("k_text", k_text), ("v_text", v_text)],
+              beta=beta, beta_text=beta_text, rms_weight=rms_weight)
+    _expect("beta", beta, (layout.B, layout.F * layout.N, layout.H), torch.float32)
+    _expect("beta_text", beta_text, (layout.B, layout.T, layout.H), torch.float32,
+            required=layout.T > 0)
     _require_cuda()
     dev = torch.device(device or "cuda:0")
     if out is None:
@@ -270,6 +363,12 @@ def vda_scan_fwd_noalloc(layout: Layout, q, k, v, k_text, v_text, beta, beta_tex
     from a static 64 MiB device array inside the library (shared by all calls;
     overlapping calls race). o_lin (and chunk_states, if wanted) are
     caller-provided device tensors."""
+    _validate(layout, q, io=[("k", k), ("v", v), ("o_lin", o_lin)],
+              text=[("k_text", k_text), ("v_text", v_text)], beta=beta, beta_text=beta_text,
+              chunk_states=chunk_states)
+    _expect("beta", beta, (layout.B, layout.F * layout.N, layout.H), torch.float32)
+    _expect("beta_text", beta_text, (layout.B, layout.T, layout.H), torch.float32,
+            required=layout.T > 0)
     _require_cuda()
     code = lib().vdn_vda_scan_fwd_noalloc(ctypes.byref(_clayout(layout)), _dtype_code(q), _ptr(q), _ptr(k), _ptr(v),
              _ptr(k_text), _ptr(v_text), _ptr(beta), _ptr(beta_text), _ptr(o_lin),
@@ -281,6 +380,28 @@ def vda_scan_fwd_noalloc(layout: Layout, q, k, v, k_text, v_text, beta, beta_tex
 def device_status() -> int:
     """Reads and clears libvdn's device status word (synchronises the device)."""
     return int(lib().vdn_device_status())
+
+
+def _validate_context(layout, q, k_audio, v_audio, q_text, q_audio, o_text, o_audio):
+    """Joint-layer tensors: audio keys/values [B, A, H, d] (both or neither),
+    text query rows and their output [B, T, H, d], audio query rows and their
+    output [B, A, H, d], all in the io dtype on q's device."""
+    B, T, H, d = layout.B, layout.T, layout.H, layout.d
+    dt = _io_dtype(q)
+    if (k_audio is None) != (v_audio is None):
+        raise ValueError("k_audio and v_audio go together")
+    A = 0 if k_audio is None else int(k_audio.shape[1]) if k_audio.dim() == 4 else -1
+    if A < 0:
+        raise ValueError(f"k_audio has shape {tuple(k_audio.shape)}; expected [B, A, H, d]")
+    _expect("k_audio", k_audio, (B, A, H, d), dt, required=False)
+    _expect("v_audio", v_audio, (B, A, H, d), dt, required=False)
+    _expect("q_text", q_text, (B, T, H, d), dt, required=False)
+    _expect("o_text", o_text, (B, T, H, d), dt, required=False)
+    _expect("q_audio", q_audio, (B, A, H, d), dt, required=False)
+    _expect("o_audio", o_audio, (B, A, H, d), dt, required=False)
+    if q_audio is not None and A == 0:
+        raise ValueError("q_audio needs k_audio and v_audio")
+    _same_device(q, k_audio, v_audio, q_text, o_text, q_audio, o_audio)
 
 
 def _context(k_audio, v_audio, q_text, q_audio, o_text, o_audio, lse_text=None, lse_audio=None):
@@ -310,6 +431,9 @@ def joint_softmax_fwd(layout: Layout, q, k, v, k_text, v_text, k_audio=None, v_a
     o_soft (video rows; their key sets include the audio keys), o_text and
     o_audio (dense context query rows, None when not asked for) and, with
     want_lse, lse / lse_text / lse_audio."""
+    _validate(layout, q, io=[("k", k), ("v", v)], optional_io=[("o_soft", o_soft)],
+              text=[("k_text", k_text), ("v_text", v_text)])
+    _validate_context(layout, q, k_audio, v_audio, q_text, q_audio, o_text, o_audio)
     _require_cuda()
     if o_soft is None:
         o_soft = torch.empty_like(q)
@@ -331,6 +455,15 @@ def joint_attn_fwd(layout: Layout, q, k, v, k_text, v_text, beta, beta_text, g_s
     """The attention of a joint text-video-audio layer: video rows get the
     hybrid (softmax branch with the audio keys; KDA decay when alpha is given),
     text/audio query rows the dense softmax. Returns (out, o_text, o_audio)."""
+    _validate(layout, q, io=[("k", k), ("v", v), ("g_soft", g_soft), ("g_lin", g_lin)],
+              optional_io=[("out", out), ("out_soft", out_soft), ("out_lin", out_lin)],
+              text=[("k_text", k_text), ("v_text", v_text)], beta=beta, beta_text=beta_text,
+              alpha=alpha, rms_weight=rms_weight)
+    _expect("beta", beta, (layout.B, layout.F * layout.N, layout.H), torch.float32)
+    _expect("beta_text", beta_text, (layout.B, layout.T, layout.H), torch.float32,
+            required=layout.T > 0)
+    _validate_context(layout, q, k_audio, v_audio, q_text, q_audio, o_text, o_audio)
+    _validate_workspace(workspace, q)
     _require_cuda()
     if out is None:
         out = torch.empty_like(q)
@@ -352,10 +485,13 @@ def window_softmax_fwd_fp8(layout: Layout, q, k, v, k_text, v_text, q_scale, k_s
     """Softmax branch with float8 e4m3 operands (torch.float8_e4m3fn tensors,
     one scale per tensor; text shares k / v scales). Returns o_soft (bf16) and,
     with want_lse, the natural-log normaliser."""
+    e4 = torch.float8_e4m3fn
+    _validate(layout, q, io=[("k", k), ("v", v)], text=[("k_text", k_text), ("v_text", v_text)],
+              io_dtype=e4)
+    _expect("o_soft", o_soft, (layout.B, layout.F * layout.N, layout.H, layout.d), torch.bfloat16,
+            required=False)
+    _same_device(q, o_soft)
     _require_cuda()
-    for t in (q, k, v):
-        if t.dtype != torch.float8_e4m3fn:
-            raise TypeError("q, k, v must be torch.float8_e4m3fn")
     if o_soft is None:
         o_soft = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if want_lse else None

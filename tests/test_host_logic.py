@@ -314,3 +314,151 @@ def test_host_pipeline_entry_validates(lib):
     assert f(ctypes.byref(ok), 0, 0, *args, need - 1) == 3
     assert f(ctypes.byref(ok), 0, 0, None, *args[1:], need) == 1
     assert f(ctypes.byref(ok), 0, 0, *args[:10], ctypes.c_float(-1.0), FAKE, FAKE, need) == 1
+
+
+# ------------------------------------------------------ binding validation
+# The kernels derive every address from the layout (TMA tensor maps, token
+# offsets), so the Python binding checks each tensor's shape, dtype and device
+# against the layout before the library is touched. These run on the CPU: a
+# well-formed call gets as far as the "needs a CUDA device" check, and a
+# mis-sized argument is refused before that.
+
+def _binding_inputs(layout, dtype):
+    import torch
+    from linear_attention_video_block_b200.synth import make_inputs
+    inp = make_inputs(layout, dtype, 5)
+    J = -(-layout.F // layout.c)
+    extra = {
+        "alpha": torch.ones((layout.B, layout.F, layout.H, layout.d)),
+        "rms_weight": torch.ones(layout.d),
+        "chunk_states": torch.zeros((layout.B, layout.H, 2, J, layout.d, layout.d)),
+        "lse": torch.zeros((layout.B, layout.L, layout.H)),
+        "out": torch.empty_like(inp["q"]),
+    }
+    return inp, extra
+
+
+@pytest.fixture
+def no_library(monkeypatch):
+    from linear_attention_video_block_b200 import vdn
+
+    def refuse():
+        raise AssertionError("the library was reached")
+    monkeypatch.setattr(vdn, "lib", refuse)
+    return vdn
+
+
+def _calls(vdn, layout, inp, extra, bad):
+    """The public calls with argument `bad` = (name, tensor) substituted."""
+    a = dict(inp, **extra)
+    if bad is not None:
+        a[bad[0]] = bad[1]
+    L = layout
+    return {
+        "window_softmax_fwd": lambda: vdn.window_softmax_fwd(
+            L, a["q"], a["k"], a["v"], a["k_text"], a["v_text"], o_soft=a.get("o_soft"), lse=a["lse"]),
+        "vda_scan_fwd": lambda: vdn.vda_scan_fwd(
+            L, a["q"], a["k"], a["v"], a["k_text"], a["v_text"], a["beta"], a["beta_text"],
+            chunk_states=a["chunk_states"], alpha=a["alpha"]),
+        "hybrid_attn_fwd": lambda: vdn.hybrid_attn_fwd(
+            L, a["q"], a["k"], a["v"], a["k_text"], a["v_text"], a["beta"], a["beta_text"], a["g_s"],
+            a["g_l"], rms_weight=a["rms_weight"], out=a["out"]),
+        "vda_scan_fwd_noalloc": lambda: vdn.vda_scan_fwd_noalloc(
+            L, a["q"], a["k"], a["v"], a["k_text"], a["v_text"], a["beta"], a["beta_text"], a["out"],
+            chunk_states=a["chunk_states"]),
+    }
+
+
+BAD_ARGS = [
+    # (argument, how it is made wrong, calls that take it)
+    ("q", "short", ["window_softmax_fwd", "vda_scan_fwd", "hybrid_attn_fwd", "vda_scan_fwd_noalloc"]),
+    ("k", "short", ["window_softmax_fwd", "vda_scan_fwd", "hybrid_attn_fwd", "vda_scan_fwd_noalloc"]),
+    ("v", "heads", ["window_softmax_fwd", "vda_scan_fwd", "hybrid_attn_fwd", "vda_scan_fwd_noalloc"]),
+    ("k_text", "short", ["window_softmax_fwd", "vda_scan_fwd", "hybrid_attn_fwd", "vda_scan_fwd_noalloc"]),
+    ("v_text", "dtype", ["window_softmax_fwd", "vda_scan_fwd", "hybrid_attn_fwd", "vda_scan_fwd_noalloc"]),
+    ("beta", "dtype", ["vda_scan_fwd", "hybrid_attn_fwd", "vda_scan_fwd_noalloc"]),
+    ("beta", "short", ["vda_scan_fwd", "hybrid_attn_fwd", "vda_scan_fwd_noalloc"]),
+    ("beta_text", "short", ["vda_scan_fwd", "hybrid_attn_fwd", "vda_scan_fwd_noalloc"]),
+    ("beta_text", "none", ["vda_scan_fwd", "hybrid_attn_fwd", "vda_scan_fwd_noalloc"]),
+    ("g_s", "short", ["hybrid_attn_fwd"]),
+    ("g_l", "dtype", ["hybrid_attn_fwd"]),
+    ("alpha", "short", ["vda_scan_fwd"]),
+    ("rms_weight", "short", ["hybrid_attn_fwd"]),
+    ("chunk_states", "short", ["vda_scan_fwd", "vda_scan_fwd_noalloc"]),
+    ("lse", "short", ["window_softmax_fwd"]),
+    ("out", "short", ["hybrid_attn_fwd", "vda_scan_fwd_noalloc"]),
+    ("q", "noncontiguous", ["window_softmax_fwd", "hybrid_attn_fwd"]),
+]
+
+
+def _spoil(t, how):
+    import torch
+    if how == "none":
+        return None
+    if how == "short":
+        return t.reshape(-1)[: t.numel() - 1].clone() if t.dim() == 1 else t[..., :-1, :].clone() \
+            if t.dim() >= 2 and t.shape[-2] > 1 else t[..., :-1].clone()
+    if how == "heads":
+        return torch.cat([t, t[:, :, :1]], dim=2)
+    if how == "dtype":
+        return t.to(torch.float16)
+    if how == "noncontiguous":
+        return t.transpose(1, 2).contiguous().transpose(1, 2)
+    raise ValueError(how)
+
+
+@pytest.mark.parametrize("name,how,calls", BAD_ARGS, ids=[f"{a}-{b}" for a, b, _ in BAD_ARGS])
+def test_binding_refuses_mis_sized_arguments_before_the_library(no_library, name, how, calls):
+    from linear_attention_video_block_b200.synth import Layout
+    layout = Layout(B=1, F=7, N=24, T=5, c=2, H=3, d=64)
+    inp, extra = _binding_inputs(layout, "bf16")
+    base = dict(inp, **extra)
+    bad = _spoil(base[name], how)
+    for call in calls:
+        with pytest.raises((ValueError, TypeError)):
+            _calls(no_library, layout, inp, extra, (name, bad))[call]()
+
+
+def test_binding_well_formed_calls_reach_the_device_check(no_library):
+    """The same calls with every argument well-formed pass validation and stop
+    only at the missing CUDA device (this host has none)."""
+    import torch
+    from linear_attention_video_block_b200.synth import Layout
+    layout = Layout(B=1, F=7, N=24, T=5, c=2, H=3, d=64)
+    inp, extra = _binding_inputs(layout, "bf16")
+    for name, call in _calls(no_library, layout, inp, extra, None).items():
+        if torch.cuda.is_available():
+            pytest.skip("a CUDA device is present")
+        with pytest.raises(RuntimeError, match="CUDA device"):
+            call()
+
+
+def test_binding_checks_joint_and_fp8_tensors(no_library):
+    import torch
+    from linear_attention_video_block_b200.synth import Layout, make_context
+    vdn = no_library
+    layout = Layout(B=1, F=7, N=24, T=5, c=2, H=3, d=64)
+    inp, _ = _binding_inputs(layout, "bf16")
+    cx = make_context(layout, 9, "bf16", 3)
+    args = (layout, inp["q"], inp["k"], inp["v"], inp["k_text"], inp["v_text"])
+    with pytest.raises(ValueError):  # audio keys without values
+        vdn.joint_softmax_fwd(*args, k_audio=cx["k_audio"])
+    with pytest.raises(ValueError):  # audio values of another length
+        vdn.joint_softmax_fwd(*args, k_audio=cx["k_audio"], v_audio=cx["v_audio"][:, :-1].clone())
+    with pytest.raises(ValueError):  # text query rows of another length
+        vdn.joint_softmax_fwd(*args, q_text=cx["q_text"][:, :-1].clone())
+    with pytest.raises(ValueError):  # audio query rows without audio keys
+        vdn.joint_softmax_fwd(*args, q_audio=cx["q_audio"])
+    with pytest.raises(TypeError):  # fp8 entry given bf16 operands
+        vdn.window_softmax_fwd_fp8(*args, 1.0, 1.0, 1.0)
+    e4 = {k: inp[k].to(torch.float8_e4m3fn) for k in ("q", "k", "v", "k_text", "v_text")}
+    with pytest.raises(ValueError):  # fp8 output of another shape
+        vdn.window_softmax_fwd_fp8(layout, e4["q"], e4["k"], e4["v"], e4["k_text"], e4["v_text"],
+                                   1.0, 1.0, 1.0, o_soft=torch.empty(3, dtype=torch.bfloat16))
+    if not torch.cuda.is_available():
+        with pytest.raises(RuntimeError, match="CUDA device"):
+            vdn.joint_softmax_fwd(*args, k_audio=cx["k_audio"], v_audio=cx["v_audio"],
+                                  q_text=cx["q_text"], q_audio=cx["q_audio"])
+        with pytest.raises(RuntimeError, match="CUDA device"):
+            vdn.window_softmax_fwd_fp8(layout, e4["q"], e4["k"], e4["v"], e4["k_text"], e4["v_text"],
+                                       1.0, 1.0, 1.0)
