@@ -49,7 +49,8 @@
  * the layout struct which is read on the host during the call. The library
  * allocates no memory and keeps no state between calls besides a device-side
  * status word (vdn_device_status) and the static scratch array used by
- * vdn_vda_scan_fwd_noalloc. Calls are asynchronous on `stream`;
+ * vdn_vda_scan_fwd_noalloc (and the host-buffer entry's streams, below).
+ * Calls are asynchronous on `stream`;
  * the return code reports host-detectable errors (VDN_ERR_INVALID for a bad
  * layout or a NULL required pointer, VDN_ERR_UNSUPPORTED for a dtype/d
  * combination not built or a pointer not 16-byte aligned, VDN_ERR_WORKSPACE
@@ -137,7 +138,9 @@ int vdn_hybrid_attn_fwd(const vdn_layout_t* layout, int dtype,
  * vdn_hybrid_attn_fwd's bit for bit. Host memory should be pinned
  * (cudaHostAlloc / cudaHostRegister) for the copies to overlap. workspace:
  * device memory of vdn_hybrid_host_workspace_bytes bytes (two chunk buffers).
- * Synchronous: returns when out holds the result. Errors as
+ * Synchronous: returns when out holds the result. The three streams and their
+ * events are created by the first call on a device and kept until the process
+ * exits; calls on one device from several host threads take turns. Errors as
  * vdn_hybrid_attn_fwd (validation before any copy). */
 size_t vdn_hybrid_host_workspace_bytes(const vdn_layout_t* layout, int dtype, int head_chunk);
 int vdn_hybrid_attn_fwd_host(const vdn_layout_t* layout, int dtype, int head_chunk,
@@ -282,8 +285,8 @@ int vdn_device_status(void);
 const char* vdn_status_string(int status);
 
 /* The CUDA runtime's description of the error behind the last VDN_ERR_CUDA
- * returned on the calling host thread (by any entry point except
- * vdn_vda_scan_fwd_noalloc), or "no CUDA error". Static string. */
+ * returned on the calling host thread (by any entry point), or "no CUDA
+ * error". Static string. */
 const char* vdn_last_cuda_error(void);
 
 #ifdef __cplusplus

@@ -10,10 +10,43 @@
 // chunk i - 1 copied out while chunk i computes. PCIe carries both directions
 // at once; with pinned host memory the copies then hide under the kernels.
 #include <cstdint>
+#include <mutex>
 
 #include "vdn_internal.cuh"
 
 namespace {
+
+// The pipeline's three streams and six events, created on the first call on a
+// device and kept for the life of the process (creating and destroying them on
+// every call costs driver round trips per call). The call is synchronous, so
+// one call at a time uses them: concurrent calls on one device take turns.
+struct Pipeline {
+  std::mutex mu;
+  bool ready = false;
+  cudaStream_t s_in = nullptr, s_comp = nullptr, s_out = nullptr;
+  cudaEvent_t ev_in[2] = {nullptr, nullptr}, ev_comp[2] = {nullptr, nullptr},
+              ev_out[2] = {nullptr, nullptr};
+};
+constexpr int kMaxDevicesH = 64;
+Pipeline g_pipe[kMaxDevicesH];
+
+// Creates the streams and events of the current device's pipeline (caller
+// holds its mutex).
+cudaError_t pipeline_init(Pipeline& p) {
+  if (p.ready) return cudaSuccess;
+  cudaError_t e = cudaSuccess;
+  auto ok = [&](cudaError_t r) { if (e == cudaSuccess) e = r; };
+  ok(cudaStreamCreateWithFlags(&p.s_in, cudaStreamNonBlocking));
+  ok(cudaStreamCreateWithFlags(&p.s_comp, cudaStreamNonBlocking));
+  ok(cudaStreamCreateWithFlags(&p.s_out, cudaStreamNonBlocking));
+  for (int i = 0; i < 2; ++i) {
+    ok(cudaEventCreateWithFlags(&p.ev_in[i], cudaEventDisableTiming));
+    ok(cudaEventCreateWithFlags(&p.ev_comp[i], cudaEventDisableTiming));
+    ok(cudaEventCreateWithFlags(&p.ev_out[i], cudaEventDisableTiming));
+  }
+  p.ready = e == cudaSuccess;
+  return e;
+}
 
 constexpr size_t kAlignH = 256;
 size_t align_h(size_t x) { return (x + kAlignH - 1) / kAlignH * kAlignH; }
@@ -128,9 +161,7 @@ int vdn_hybrid_attn_fwd_host(const vdn_layout_t* layout, int dtype, int head_chu
                              const void* v_text, const float* beta, const float* beta_text,
                              const void* g_soft, const void* g_lin, const float* rms_weight,
                              float rms_eps, void* out, void* workspace, size_t workspace_bytes) {
-  if (!layout || layout->B < 1 || layout->F < 1 || layout->N < 1 || layout->T < 0 || layout->c < 1 ||
-      layout->H < 1 || layout->d < 1)
-    return VDN_ERR_INVALID;
+  if (!vdn::layout_ok(layout)) return VDN_ERR_INVALID;
   const size_t need = vdn_hybrid_host_workspace_bytes(layout, dtype, head_chunk);
   if (need == 0) return VDN_ERR_UNSUPPORTED;
   if (!q || !k || !v || !beta || !g_soft || !g_lin || !out) return VDN_ERR_INVALID;
@@ -153,18 +184,21 @@ int vdn_hybrid_attn_fwd_host(const vdn_layout_t* layout, int dtype, int head_chu
   base += align_h((size_t)d * 4);
   const size_t buf_bytes = carve_chunk(lmax, dtype, nullptr).bytes;
 
-  cudaStream_t s_in = nullptr, s_comp = nullptr, s_out = nullptr;
-  cudaEvent_t ev_in[2] = {nullptr, nullptr}, ev_comp[2] = {nullptr, nullptr}, ev_out[2] = {nullptr, nullptr};
-  int status = VDN_OK;
-  auto fail = [&](cudaError_t e) { if (e != cudaSuccess && status == VDN_OK) status = VDN_ERR_CUDA; };
-  fail(cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking));
-  fail(cudaStreamCreateWithFlags(&s_comp, cudaStreamNonBlocking));
-  fail(cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking));
-  for (int i = 0; i < 2; ++i) {
-    fail(cudaEventCreateWithFlags(&ev_in[i], cudaEventDisableTiming));
-    fail(cudaEventCreateWithFlags(&ev_comp[i], cudaEventDisableTiming));
-    fail(cudaEventCreateWithFlags(&ev_out[i], cudaEventDisableTiming));
-  }
+  int dev = 0;
+  int status = vdn::cuda_status(cudaGetDevice(&dev));
+  if (status != VDN_OK) return status;
+  if (dev < 0 || dev >= kMaxDevicesH) return VDN_ERR_UNSUPPORTED;
+  Pipeline& pipe = g_pipe[dev];
+  std::lock_guard<std::mutex> lock(pipe.mu);
+  status = vdn::cuda_status(pipeline_init(pipe));
+  if (status != VDN_OK) return status;
+  cudaStream_t s_in = pipe.s_in, s_comp = pipe.s_comp, s_out = pipe.s_out;
+  cudaEvent_t* ev_in = pipe.ev_in;
+  cudaEvent_t* ev_comp = pipe.ev_comp;
+  cudaEvent_t* ev_out = pipe.ev_out;
+  auto fail = [&](cudaError_t e) {
+    if (e != cudaSuccess && status == VDN_OK) status = vdn::cuda_status(e);
+  };
 
   if (rms_weight)
     fail(cudaMemcpyAsync(rms_w_dev, rms_weight, (size_t)d * 4, cudaMemcpyHostToDevice, s_in));
@@ -208,15 +242,7 @@ int vdn_hybrid_attn_fwd_host(const vdn_layout_t* layout, int dtype, int head_chu
     fail(cudaEventRecord(ev_out[slot], s_out));
   }
   // the call returns with the output in host memory (and nothing in flight)
-  for (cudaStream_t st : {s_in, s_comp, s_out})
-    if (st) fail(cudaStreamSynchronize(st));
-  for (int i = 0; i < 2; ++i) {
-    if (ev_in[i]) cudaEventDestroy(ev_in[i]);
-    if (ev_comp[i]) cudaEventDestroy(ev_comp[i]);
-    if (ev_out[i]) cudaEventDestroy(ev_out[i]);
-  }
-  for (cudaStream_t st : {s_in, s_comp, s_out})
-    if (st) cudaStreamDestroy(st);
+  for (cudaStream_t st : {s_in, s_comp, s_out}) fail(cudaStreamSynchronize(st));
   return status;
 }
 

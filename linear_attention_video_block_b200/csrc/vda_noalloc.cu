@@ -63,8 +63,6 @@ size_t scratch_bytes(const vdn::Layout& l, bool own_states) {
   return n;
 }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 }  // namespace
 
 extern "C" int vdn_vda_scan_fwd_noalloc(const vdn_layout_t* layout, int dtype, const void* q,
@@ -72,31 +70,25 @@ extern "C" int vdn_vda_scan_fwd_noalloc(const vdn_layout_t* layout, int dtype, c
                                         const void* v_text, const float* beta,
                                         const float* beta_text, void* o_lin, float* chunk_states,
                                         cudaStream_t stream) {
-  if (!layout || layout->B < 1 || layout->F < 1 || layout->N < 1 || layout->T < 0 || layout->c < 1 ||
-      layout->H < 1 || layout->d < 1)
-    return VDN_ERR_INVALID;
-  const long long L = (long long)layout->F * layout->N;
-  if (L > (1LL << 30) || layout->T > (1 << 30)) return VDN_ERR_INVALID;
-  const int d = layout->d;
-  const bool d_ok = (dtype == VDN_F32 && (d == 16 || d == 32 || d == 64 || d == 128)) ||
-                    (dtype == VDN_BF16 && (d == 64 || d == 128));
-  if (!d_ok) return VDN_ERR_UNSUPPORTED;
+  // the same checks as vdn_vda_scan_fwd (vdn_internal.cuh)
+  if (!vdn::layout_ok(layout)) return VDN_ERR_INVALID;
+  if (!vdn::dtype_d_ok(dtype, layout->d)) return VDN_ERR_UNSUPPORTED;
   if (!q || !k || !v || !beta || !o_lin) return VDN_ERR_INVALID;
   if (layout->T > 0 && (!k_text || !v_text || !beta_text)) return VDN_ERR_INVALID;
   const void* ptrs[] = {q, k, v, beta, o_lin, chunk_states};
   for (const void* p : ptrs)
-    if (p && !aligned16(p)) return VDN_ERR_UNSUPPORTED;
-  if (layout->T > 0 && (!aligned16(k_text) || !aligned16(v_text) || !aligned16(beta_text)))
+    if (p && !vdn::aligned16(p)) return VDN_ERR_UNSUPPORTED;
+  if (layout->T > 0 &&
+      (!vdn::aligned16(k_text) || !vdn::aligned16(v_text) || !vdn::aligned16(beta_text)))
     return VDN_ERR_UNSUPPORTED;
 
-  vdn::Layout l;
-  l.B = layout->B; l.F = layout->F; l.N = layout->N; l.T = layout->T; l.c = layout->c;
-  l.H = layout->H; l.d = layout->d;
+  const vdn::Layout l = vdn::to_layout(layout);
   const bool own_states = chunk_states == nullptr;
   if (scratch_bytes(l, own_states) > kStaticScratchBytes) return VDN_ERR_WORKSPACE;
 
   void* base = nullptr;
-  if (scratch_address(&base) != cudaSuccess) return VDN_ERR_CUDA;
+  int s = vdn::cuda_status(scratch_address(&base));
+  if (s != VDN_OK) return s;
   const size_t dd = (size_t)l.d * l.d, bh = (size_t)l.B * l.H;
   char* p = static_cast<char*>(base);
   float* am = reinterpret_cast<float*>(p);
@@ -108,13 +100,11 @@ extern "C" int vdn_vda_scan_fwd_noalloc(const vdn_layout_t* layout, int dtype, c
   const void* kt = layout->T ? k_text : nullptr;
   const void* vt = layout->T ? v_text : nullptr;
   const float* bt = layout->T ? beta_text : nullptr;
-  if (vdn::launch_vda_states(l, dtype, k, v, kt, vt, beta, bt, nullptr, am, bw, states, stream) != cudaSuccess)
-    return VDN_ERR_CUDA;
-  cudaError_t e;
+  s = vdn::cuda_status(
+      vdn::launch_vda_states(l, dtype, k, v, kt, vt, beta, bt, nullptr, am, bw, states, stream));
+  if (s != VDN_OK) return s;
   if (vdn::readout_tc_supported(l, dtype))
-    e = vdn::launch_readout_tc(l, q, states, o_lin, stream);
-  else
-    e = vdn::launch_readout(l, dtype, 0, q, states, nullptr, nullptr, nullptr, nullptr, 0.f, o_lin,
-                            nullptr, nullptr, stream);
-  return e == cudaSuccess ? VDN_OK : VDN_ERR_CUDA;
+    return vdn::cuda_status(vdn::launch_readout_tc(l, q, states, o_lin, stream));
+  return vdn::cuda_status(vdn::launch_readout(l, dtype, 0, q, states, nullptr, nullptr, nullptr,
+                                              nullptr, 0.f, o_lin, nullptr, nullptr, stream));
 }

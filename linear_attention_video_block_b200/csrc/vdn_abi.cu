@@ -5,37 +5,31 @@
 
 #include "vdn_internal.cuh"
 
+namespace vdn {
+
+// The CUDA error behind the last VDN_ERR_CUDA returned on this host thread.
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return VDN_OK;
+  t_last_cuda_error = e;
+  return VDN_ERR_CUDA;
+}
+
+}  // namespace vdn
+
 namespace {
 
 using vdn::Layout;
+using vdn::aligned16;
+using vdn::cuda_status;
+using vdn::dtype_d_ok;
+using vdn::layout_ok;
+using vdn::to_layout;
 
 constexpr size_t kAlign = 256;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
-
-bool layout_ok(const vdn_layout_t* l) {
-  if (!l) return false;
-  if (l->B < 1 || l->F < 1 || l->N < 1 || l->T < 0 || l->c < 1 || l->H < 1 || l->d < 1) return false;
-  // token offsets and TMA coordinates are 32-bit signed per dimension
-  long long L = (long long)l->F * l->N;
-  if (L > (1LL << 30) || l->T > (1 << 30)) return false;
-  if ((long long)l->B * L * l->H * l->d > (1LL << 46)) return false;
-  return true;
-}
-
-bool dtype_d_ok(int dtype, int d) {
-  if (dtype == VDN_F32) return d == 16 || d == 32 || d == 64 || d == 128;
-  if (dtype == VDN_BF16) return d == 64 || d == 128;
-  return false;
-}
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-Layout to_layout(const vdn_layout_t* l) {
-  Layout x;
-  x.B = l->B; x.F = l->F; x.N = l->N; x.T = l->T; x.c = l->c; x.H = l->H; x.d = l->d;
-  return x;
-}
 
 struct Workspace {
   float* am = nullptr;
@@ -63,15 +57,6 @@ Workspace carve(const Layout& l, int dtype, void* base, bool need_states, bool n
   if (need_osoft) w.o_soft = static_cast<float*>(take((size_t)l.B * l.L() * l.H * l.d * sizeof(float)));
   w.bytes = off;
   return w;
-}
-
-// The CUDA error behind the last VDN_ERR_CUDA returned on this host thread.
-thread_local cudaError_t t_last_cuda_error = cudaSuccess;
-
-int cuda_status(cudaError_t e) {
-  if (e == cudaSuccess) return VDN_OK;
-  t_last_cuda_error = e;
-  return VDN_ERR_CUDA;
 }
 
 int run_window(const Layout& l, int dtype, const void* q, const void* k, const void* v,
@@ -320,7 +305,8 @@ int vdn_device_status(void) {
 }
 
 const char* vdn_last_cuda_error(void) {
-  return t_last_cuda_error == cudaSuccess ? "no CUDA error" : cudaGetErrorString(t_last_cuda_error);
+  return vdn::t_last_cuda_error == cudaSuccess ? "no CUDA error"
+                                                : cudaGetErrorString(vdn::t_last_cuda_error);
 }
 
 const char* vdn_status_string(int status) {

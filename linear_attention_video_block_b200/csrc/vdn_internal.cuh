@@ -36,6 +36,38 @@ struct Layout {
   __host__ __device__ int groups() const { return J() + 4; }
 };
 
+// ------------------------------------------------- argument validation
+// Shared by every entry point of the C ABI (vdn_abi.cu, vda_noalloc.cu,
+// host_pipeline.cu), so that their checks cannot drift apart.
+
+inline bool layout_ok(const vdn_layout_t* l) {
+  if (!l) return false;
+  if (l->B < 1 || l->F < 1 || l->N < 1 || l->T < 0 || l->c < 1 || l->H < 1 || l->d < 1) return false;
+  // token offsets and TMA coordinates are 32-bit signed per dimension
+  const long long L = (long long)l->F * l->N;
+  if (L > (1LL << 30) || l->T > (1 << 30)) return false;
+  if ((long long)l->B * L * l->H * l->d > (1LL << 46)) return false;
+  return true;
+}
+
+inline bool dtype_d_ok(int dtype, int d) {
+  if (dtype == VDN_F32) return d == 16 || d == 32 || d == 64 || d == 128;
+  if (dtype == VDN_BF16) return d == 64 || d == 128;
+  return false;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline Layout to_layout(const vdn_layout_t* l) {
+  Layout x;
+  x.B = l->B; x.F = l->F; x.N = l->N; x.T = l->T; x.c = l->c; x.H = l->H; x.d = l->d;
+  return x;
+}
+
+// VDN_OK for cudaSuccess; otherwise records e as the calling host thread's
+// last CUDA error (vdn_last_cuda_error) and returns VDN_ERR_CUDA.
+int cuda_status(cudaError_t e);
+
 constexpr int kCtxText = 1;
 constexpr int kCtxAudio = 2;
 
