@@ -26,6 +26,7 @@ float8 e4m3 operands (vdn_window_softmax_fwd_fp8).
 
 Printed on rank 0: one JSON line with the throughput (video tokens/s over all
 ranks), the roofline of the dominant kernel (window softmax, tensor-core bound),
+the roofline of the linear branch (vdn_vda_scan_fwd, HBM-bound),
 the end-to-end figure through the public call with host buffers, the CPU
 oracle baseline on a bounded sample, and the SM clocks seen during timing.
 """
@@ -349,6 +350,24 @@ def run_ours(args, rank, world, local_rank):
     w1.record(stream)
     torch.cuda.synchronize(dev)
     win_ms = w0.elapsed_time(w1) / args.steps
+
+    # The linear branch alone (vdn_vda_scan_fwd: Gram, inverse, scans, zero
+    # fill, readout), HBM-bound, timed over the same number of launches.
+    o_lin = torch.empty_like(inp["q"])
+    for _ in range(2):
+        vdn.vda_scan_fwd(lay, inp["q"], inp["k"], inp["v"], inp["k_text"], inp["v_text"], inp["beta"],
+                         inp["beta_text"], o_lin=o_lin, workspace=ws)
+    torch.cuda.synchronize(dev)
+    v0 = torch.cuda.Event(enable_timing=True)
+    v1 = torch.cuda.Event(enable_timing=True)
+    v0.record(stream)
+    for _ in range(args.steps):
+        vdn.vda_scan_fwd(lay, inp["q"], inp["k"], inp["v"], inp["k_text"], inp["v_text"], inp["beta"],
+                         inp["beta_text"], o_lin=o_lin, workspace=ws)
+    v1.record(stream)
+    torch.cuda.synchronize(dev)
+    vda_ms = v0.elapsed_time(v1) / args.steps
+    del o_lin
     clk = clocks.stop(None) if rank == 0 else None
 
     # End to end through the public call with pinned host buffers: every step
@@ -384,7 +403,7 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = x0.elapsed_time(x1) / e2e_steps
     assert vdn.device_status() == 0, "device status set during timing"
 
-    ms, win_ms, e2e_ms = max_over_ranks([ms, win_ms, e2e_ms], world, device=dev)
+    ms, win_ms, vda_ms, e2e_ms = max_over_ranks([ms, win_ms, vda_ms, e2e_ms], world, device=dev)
     if rank != 0:
         return
     tokens = lay.L * lay.B * world
@@ -407,6 +426,7 @@ def run_ours(args, rank, world, local_rank):
                      "peak_source": f"{peak_kind} bf16 dense (burst)",
                      "flops_per_launch": flops, "launch_ms": win_ms,
                      "share_of_step": win_ms / ms},
+        "roofline_vda": vda_roofline(lay, vda_ms, peaks, peak_kind),
         "cpu_baseline": {"value": cpu_val, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                          "sample": cpu_desc, "seconds": cpu_s},
         "e2e": {"value": job_throughput(lay.L * lay.B, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
@@ -436,6 +456,20 @@ def vda_bytes(lay) -> float:
     tok = len(frames) * N + T
     per_bh = tok * (2 * d * 2 + 4) + 2 * F * N * d * 2 + 2 * J * d * d * 4
     return float(per_bh * H * B)
+
+
+def vda_roofline(lay, ms, peaks, peak_kind):
+    """Roofline object of the linear-branch entry (HBM-bound): its algorithmic
+    bytes per launch (vda_bytes) over the measured launch time, against the
+    measured HBM copy bandwidth."""
+    peak = float(peaks["hbm_gbs"])
+    nbytes = vda_bytes(lay)
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "kernel": "linear branch (vdn_vda_scan_fwd: gram, inverse, scans, "
+                                      "readout)",
+            "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "traffic": None, "peak_source": f"{peak_kind} HBM copy bandwidth",
+            "bytes_per_launch": nbytes, "launch_ms": ms}
 
 
 def decay_bytes(lay) -> float:
