@@ -250,6 +250,43 @@ int vdn_joint_attn_fwd(const vdn_layout_t* layout, int dtype, const vdn_context_
                        void* out, void* out_soft, void* out_lin,
                        void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* The two branches with a float32 output whatever the input dtype: the same
+ * computations as vdn_window_softmax_fwd and vdn_vda_scan_fwd, o_soft / o_lin
+ * written as float32 [B, L, H, d] (the form the hybrid entry combines
+ * internally). They serve callers that run the branches apart and combine
+ * later with vdn_gated_combine_fwd, e.g. the branch-specialised sequence-
+ * parallel split (project page, "Parallelization & Few-Step Generation"):
+ * rounding each branch to bf16 before the combine would add two roundings of
+ * its own to the output, beyond the op's tolerance. Arguments, workspace and
+ * errors as the plain entries. */
+int vdn_window_softmax_fwd_f32out(const vdn_layout_t* layout, int dtype,
+                                  const void* q, const void* k, const void* v,
+                                  const void* k_text, const void* v_text,
+                                  float* o_soft, float* lse, cudaStream_t stream);
+int vdn_vda_scan_fwd_f32out(const vdn_layout_t* layout, int dtype,
+                            const void* q, const void* k, const void* v,
+                            const void* k_text, const void* v_text,
+                            const float* beta, const float* beta_text,
+                            float* o_lin, float* chunk_states,
+                            void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* The gated combine alone (project page, "Gating the Softmax and Linear Branch
+ * Outputs"): out = sigmoid(g_soft) * o_soft + sigmoid(g_lin) * RMSNorm(o_lin),
+ * RMSNorm over the head dim with rms_eps and rms_weight (nullable, [d] float32,
+ * defaults to ones). o_soft and o_lin are float32 [tokens, H, d] (the _f32out
+ * branch outputs of the same tokens; o_lin zero on boundary frames); g_soft,
+ * g_lin and out are [tokens, H, d] in dtype. tokens is any number of (batch,
+ * token) rows, e.g. B times the length of a token shard. It finishes the
+ * hybrid forward when the two branches were computed apart, for instance on
+ * different GPUs of a branch-specialised split, and returned to the token
+ * shard that holds the gates. tokens == 0 is a no-op. Errors as
+ * vdn_hybrid_attn_fwd. */
+int vdn_gated_combine_fwd(long long tokens, int H, int d, int dtype,
+                          const float* o_soft, const float* o_lin,
+                          const void* g_soft, const void* g_lin,
+                          const float* rms_weight, float rms_eps, void* out,
+                          cudaStream_t stream);
+
 /* Size of the device scratch array behind vdn_vda_scan_fwd_noalloc: 64 MiB. */
 #define VDN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 

@@ -16,7 +16,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libvdn.so")
 SOURCES = ["vdn_abi.cu", "window_simt.cu", "window_tc.cu", "window_fp8.cu", "gram_tc.cu", "vda.cu",
-           "readout.cu", "readout_tc.cu", "vda_noalloc.cu", "host_pipeline.cu"]
+           "readout.cu", "readout_tc.cu", "combine.cu", "vda_noalloc.cu", "host_pipeline.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-Xcompiler", "-Wall", "-diag-suppress", "177"]

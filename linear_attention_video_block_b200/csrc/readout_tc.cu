@@ -13,7 +13,8 @@
 //              2-5 drains the accumulator of the even tiles and warpgroup 6-9
 //              that of the odd tiles to global memory (one row per thread), so
 //              that two tiles' worth of loads and stores are in flight
-// Boundary-frame groups write zeros. HBM-bound: q is read once, o_lin written once.
+// Boundary-frame groups write zeros. HBM-bound: q is read once, o_lin written once
+// (bf16, or float32 for the branch-specialised split's exchange).
 //
 // Combine variant (project page, "Gating the Softmax and Linear Branch
 // Outputs"): instead of o_lin, each drain thread finishes its row of the hybrid
@@ -111,11 +112,16 @@ __device__ __forceinline__ bool rwait(unsigned long long* bar, uint32_t parity, 
   return mbar_wait_impl(bar, parity, abort, &g_readout_status, watch_abort);
 }
 
-template <int D, bool kCombine>
+// kMode: 0 writes o_lin in bf16, 1 the combined output (CombineArgs), 2 o_lin
+// in float32 (the branch output a branch-specialised split sends on).
+template <int D, int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
 readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Layout l,
-                  const float* __restrict__ states, __nv_bfloat16* __restrict__ o_lin,
+                  const float* __restrict__ states, void* __restrict__ o_lin_out,
                   const CombineArgs cx) {
+  constexpr bool kCombine = kMode == 1;
+  __nv_bfloat16* o_lin = static_cast<__nv_bfloat16*>(o_lin_out);
+  float* o_lin32 = static_cast<float*>(o_lin_out);
   using C = RCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -145,6 +151,9 @@ readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Layout l,
         const float lin[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         combine8(cx, off, o, lin, *reinterpret_cast<const uint4*>(cx.g_soft + off),
                  make_uint4(0u, 0u, 0u, 0u), false);
+      } else if constexpr (kMode == 2) {
+        *reinterpret_cast<float4*>(o_lin32 + off) = make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4*>(o_lin32 + off + 4) = make_float4(0.f, 0.f, 0.f, 0.f);
       } else {
         *reinterpret_cast<uint4*>(o_lin + off) = make_uint4(0u, 0u, 0u, 0u);
       }
@@ -273,7 +282,6 @@ readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Layout l,
       const int grow = r0 + t * kRows + m;
       const bool store = grow < G.q0 + G.nq;
       const long long rbase = ((long long)b * l.L() + grow) * HD + (long long)h * D;
-      __nv_bfloat16* dst = o_lin + rbase;
       if constexpr (kCombine) {
         // RMSNorm statistic of the row, then the gated sum in 32-column pieces
         const uint32_t tacc = tmem + lane_base + s * D;
@@ -314,8 +322,14 @@ readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Layout l,
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t r[32];
         tmem_ld_x32(tmem + lane_base + s * D + c0, r);
-        if (store) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+        if (kMode == 2 && store) {
+          float4* d4 = reinterpret_cast<float4*>(o_lin32 + rbase + c0);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            d4[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+        } else if (store) {
+          uint4* d4 = reinterpret_cast<uint4*>(o_lin + rbase + c0);
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             d4[i] = make_uint4(pack_bf16(__uint_as_float(r[8 * i]), __uint_as_float(r[8 * i + 1])),
@@ -338,18 +352,18 @@ readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Layout l,
   }
 }
 
-template <int D, bool kCombine>
+template <int D, int kMode>
 cudaError_t launch_readout_t(const Layout& l, const void* q, const float* states, void* o_lin,
                              const CombineArgs& cx, cudaStream_t st) {
   CUtensorMap mq;
   if (!make_map(&mq, q, D, l.H, l.L(), l.B)) return cudaErrorInvalidValue;
-  auto kern = readout_tc_kernel<D, kCombine>;
+  auto kern = readout_tc_kernel<D, kMode>;
   const int smem = RCfg<D>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(tiles_per_head(l, kRows * kTilesPerCta), l.H, l.B);
   if (grid.x == 0) return cudaSuccess;
-  kern<<<grid, kThreads, smem, st>>>(mq, l, states, static_cast<__nv_bfloat16*>(o_lin), cx);
+  kern<<<grid, kThreads, smem, st>>>(mq, l, states, o_lin, cx);
   return cudaGetLastError();
 }
 
@@ -360,10 +374,14 @@ bool readout_tc_supported(const Layout& l, int dtype) {
 }
 
 cudaError_t launch_readout_tc(const Layout& l, const void* q, const float* states, void* o_lin,
-                              cudaStream_t st) {
+                              bool out_f32, cudaStream_t st) {
   const CombineArgs cx{};
-  if (l.d == 128) return launch_readout_t<128, false>(l, q, states, o_lin, cx, st);
-  if (l.d == 64) return launch_readout_t<64, false>(l, q, states, o_lin, cx, st);
+  if (l.d == 128)
+    return out_f32 ? launch_readout_t<128, 2>(l, q, states, o_lin, cx, st)
+                   : launch_readout_t<128, 0>(l, q, states, o_lin, cx, st);
+  if (l.d == 64)
+    return out_f32 ? launch_readout_t<64, 2>(l, q, states, o_lin, cx, st)
+                   : launch_readout_t<64, 0>(l, q, states, o_lin, cx, st);
   return cudaErrorInvalidValue;
 }
 
@@ -375,8 +393,8 @@ cudaError_t launch_combine_tc(const Layout& l, const void* q, const float* state
                        static_cast<const __nv_bfloat16*>(gl), rms_w, eps,
                        static_cast<__nv_bfloat16*>(out), static_cast<__nv_bfloat16*>(out_soft),
                        static_cast<__nv_bfloat16*>(out_lin)};
-  if (l.d == 128) return launch_readout_t<128, true>(l, q, states, nullptr, cx, st);
-  if (l.d == 64) return launch_readout_t<64, true>(l, q, states, nullptr, cx, st);
+  if (l.d == 128) return launch_readout_t<128, 1>(l, q, states, nullptr, cx, st);
+  if (l.d == 64) return launch_readout_t<64, 1>(l, q, states, nullptr, cx, st);
   return cudaErrorInvalidValue;
 }
 

@@ -104,7 +104,7 @@ extern "C" int vdn_vda_scan_fwd_noalloc(const vdn_layout_t* layout, int dtype, c
       vdn::launch_vda_states(l, dtype, k, v, kt, vt, beta, bt, nullptr, am, bw, states, stream));
   if (s != VDN_OK) return s;
   if (vdn::readout_tc_supported(l, dtype))
-    return vdn::cuda_status(vdn::launch_readout_tc(l, q, states, o_lin, stream));
+    return vdn::cuda_status(vdn::launch_readout_tc(l, q, states, o_lin, false, stream));
   return vdn::cuda_status(vdn::launch_readout(l, dtype, 0, q, states, nullptr, nullptr, nullptr,
                                               nullptr, 0.f, o_lin, nullptr, nullptr, stream));
 }

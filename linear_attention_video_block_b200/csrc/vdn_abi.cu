@@ -100,7 +100,7 @@ int joint_setup(const vdn_layout_t* layout, const vdn_context_t* ctx, Layout& ls
 
 int window_impl(const vdn_layout_t* layout, int dtype, const vdn_context_t* ctx, const void* q,
                 const void* k, const void* v, const void* k_text, const void* v_text,
-                void* o_soft, float* lse, cudaStream_t stream) {
+                void* o_soft, float* lse, cudaStream_t stream, bool out_f32 = false) {
   if (!layout_ok(layout)) return VDN_ERR_INVALID;
   if (!dtype_d_ok(dtype, layout->d)) return VDN_ERR_UNSUPPORTED;
   if (!q || !k || !v || !o_soft) return VDN_ERR_INVALID;
@@ -113,7 +113,7 @@ int window_impl(const vdn_layout_t* layout, int dtype, const vdn_context_t* ctx,
   const int s = joint_setup(layout, ctx, ls, ja);
   if (s != VDN_OK) return s;
   return run_window(ls, dtype, q, k, v, layout->T ? k_text : nullptr,
-                    layout->T ? v_text : nullptr, o_soft, false, lse, ja, stream);
+                    layout->T ? v_text : nullptr, o_soft, out_f32, lse, ja, stream);
 }
 
 }  // namespace
@@ -130,6 +130,13 @@ int vdn_window_softmax_fwd(const vdn_layout_t* layout, int dtype, const void* q,
                            const void* v, const void* k_text, const void* v_text, void* o_soft,
                            float* lse, cudaStream_t stream) {
   return window_impl(layout, dtype, nullptr, q, k, v, k_text, v_text, o_soft, lse, stream);
+}
+
+int vdn_window_softmax_fwd_f32out(const vdn_layout_t* layout, int dtype, const void* q,
+                                  const void* k, const void* v, const void* k_text,
+                                  const void* v_text, float* o_soft, float* lse,
+                                  cudaStream_t stream) {
+  return window_impl(layout, dtype, nullptr, q, k, v, k_text, v_text, o_soft, lse, stream, true);
 }
 
 int vdn_window_softmax_fwd_fp8(const vdn_layout_t* layout, const void* q, const void* k,
@@ -166,7 +173,8 @@ namespace {
 int vda_scan_impl(const vdn_layout_t* layout, int dtype, const void* q, const void* k,
                   const void* v, const void* k_text, const void* v_text, const float* beta,
                   const float* beta_text, const float* alpha, void* o_lin, float* chunk_states,
-                  void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+                  void* workspace, size_t workspace_bytes, cudaStream_t stream,
+                  bool out_f32 = false) {
   if (!layout_ok(layout)) return VDN_ERR_INVALID;
   if (!dtype_d_ok(dtype, layout->d)) return VDN_ERR_UNSUPPORTED;
   if (!q || !k || !v || !beta || !o_lin) return VDN_ERR_INVALID;
@@ -188,7 +196,8 @@ int vda_scan_impl(const vdn_layout_t* layout, int dtype, const void* q, const vo
                                              states, stream));
   if (s != VDN_OK) return s;
   if (vdn::readout_tc_supported(l, dtype))
-    return cuda_status(vdn::launch_readout_tc(l, q, states, o_lin, stream));
+    return cuda_status(vdn::launch_readout_tc(l, q, states, o_lin, out_f32, stream));
+  // the CUDA-core readout serves fp32 tensors, whose o_lin is float32 anyway
   return cuda_status(vdn::launch_readout(l, dtype, 0, q, states, nullptr, nullptr, nullptr, nullptr,
                                          0.f, o_lin, nullptr, nullptr, stream));
 }
@@ -246,6 +255,15 @@ int vdn_vda_scan_fwd(const vdn_layout_t* layout, int dtype, const void* q, const
                        chunk_states, workspace, workspace_bytes, stream);
 }
 
+int vdn_vda_scan_fwd_f32out(const vdn_layout_t* layout, int dtype, const void* q, const void* k,
+                            const void* v, const void* k_text, const void* v_text,
+                            const float* beta, const float* beta_text, float* o_lin,
+                            float* chunk_states, void* workspace, size_t workspace_bytes,
+                            cudaStream_t stream) {
+  return vda_scan_impl(layout, dtype, q, k, v, k_text, v_text, beta, beta_text, nullptr, o_lin,
+                       chunk_states, workspace, workspace_bytes, stream, true);
+}
+
 int vdn_vda_scan_fwd_decay(const vdn_layout_t* layout, int dtype, const void* q, const void* k,
                            const void* v, const void* k_text, const void* v_text, const float* beta,
                            const float* beta_text, const float* alpha, void* o_lin,
@@ -290,6 +308,21 @@ int vdn_joint_attn_fwd(const vdn_layout_t* layout, int dtype, const vdn_context_
   return hybrid_impl(layout, dtype, ctx, q, k, v, k_text, v_text, beta, beta_text, alpha, g_soft,
                      g_lin, rms_weight, rms_eps, out, out_soft, out_lin, workspace, workspace_bytes,
                      stream);
+}
+
+int vdn_gated_combine_fwd(long long tokens, int H, int d, int dtype, const float* o_soft,
+                          const float* o_lin, const void* g_soft, const void* g_lin,
+                          const float* rms_weight, float rms_eps, void* out, cudaStream_t stream) {
+  if (tokens < 0 || H < 1 || d < 1) return VDN_ERR_INVALID;
+  if (tokens > (1LL << 36) || tokens * H * d > (1LL << 46)) return VDN_ERR_INVALID;
+  if (!dtype_d_ok(dtype, d)) return VDN_ERR_UNSUPPORTED;
+  if (!(rms_eps >= 0.f)) return VDN_ERR_INVALID;
+  if (tokens == 0) return VDN_OK;
+  if (!o_soft || !o_lin || !g_soft || !g_lin || !out) return VDN_ERR_INVALID;
+  const void* ptrs[] = {o_soft, o_lin, g_soft, g_lin, rms_weight, out};
+  for (const void* p : ptrs) if (p && !aligned16(p)) return VDN_ERR_UNSUPPORTED;
+  return cuda_status(vdn::launch_gated_combine(tokens * H, d, dtype, o_soft, o_lin, g_soft, g_lin,
+                                               rms_weight, rms_eps, out, stream));
 }
 
 int vdn_device_status(void) {

@@ -289,10 +289,11 @@ cudaError_t launch_gram_tc(const Layout& l, int has_text, int fwd_max, int rev_l
                            cudaStream_t st);
 cudaError_t read_and_clear_gram_status(int* status);
 
-// tcgen05 linear readout o_lin = S_sum q (bf16, d in {64, 128}).
+// tcgen05 linear readout o_lin = S_sum q (bf16 q, d in {64, 128}); o_lin in
+// bf16, or in float32 when out_f32.
 bool readout_tc_supported(const Layout& l, int dtype);
 cudaError_t launch_readout_tc(const Layout& l, const void* q, const float* states, void* o_lin,
-                              cudaStream_t st);
+                              bool out_f32, cudaStream_t st);
 cudaError_t read_and_clear_readout_status(int* status);
 
 // The same readout finishing the hybrid output instead of writing o_lin:
@@ -303,6 +304,13 @@ cudaError_t launch_combine_tc(const Layout& l, const void* q, const float* state
                               const float* o_soft, const void* gs, const void* gl,
                               const float* rms_w, float eps, void* out, void* out_soft,
                               void* out_lin, cudaStream_t st);
+
+// out = sig(gs) o_soft + sig(gl) RMSNorm_d(o_lin) over rows x d elements: o_soft
+// and o_lin float32 [rows, d], the gates and out in the io dtype (a
+// token-sharded combine of the two branches computed elsewhere).
+cudaError_t launch_gated_combine(long long rows, int d, int dtype, const void* o_soft,
+                                 const void* o_lin, const void* gs, const void* gl,
+                                 const float* rms_w, float eps, void* out, cudaStream_t st);
 
 // VDA: Gram into (am, bw) slots [B, H, F, d, d] (slot 0 = text), inverse in place
 // of am, scans into states [B, H, 2, J, d, d]. alpha (nullable) [B, F, H, d]: KDA

@@ -34,8 +34,9 @@ EXPORTS = ("vdn_workspace_bytes", "vdn_window_softmax_fwd", "vdn_vda_scan_fwd",
            "vdn_vda_scan_fwd_decay", "vdn_hybrid_attn_fwd", "vdn_hybrid_attn_fwd_decay",
            "vdn_vda_scan_fwd_noalloc", "vdn_joint_softmax_fwd", "vdn_joint_attn_fwd",
            "vdn_window_softmax_fwd_fp8", "vdn_hybrid_attn_fwd_host",
-           "vdn_hybrid_host_workspace_bytes", "vdn_device_status", "vdn_status_string",
-           "vdn_last_cuda_error")
+           "vdn_hybrid_host_workspace_bytes", "vdn_gated_combine_fwd",
+           "vdn_window_softmax_fwd_f32out", "vdn_vda_scan_fwd_f32out", "vdn_device_status",
+           "vdn_status_string", "vdn_last_cuda_error")
 
 
 class VdnError(RuntimeError):
@@ -94,6 +95,12 @@ def lib():
         L.vdn_joint_attn_fwd.restype = I
         L.vdn_vda_scan_fwd_noalloc.argtypes = [LP, I] + [P] * 10
         L.vdn_vda_scan_fwd_noalloc.restype = I
+        L.vdn_window_softmax_fwd_f32out.argtypes = [LP, I] + [P] * 8
+        L.vdn_window_softmax_fwd_f32out.restype = I
+        L.vdn_vda_scan_fwd_f32out.argtypes = [LP, I] + [P] * 9 + [P, S, P]
+        L.vdn_vda_scan_fwd_f32out.restype = I
+        L.vdn_gated_combine_fwd.argtypes = [ctypes.c_longlong, I, I, I] + [P] * 5 + [F, P, P]
+        L.vdn_gated_combine_fwd.restype = I
         L.vdn_device_status.argtypes = []
         L.vdn_device_status.restype = I
         L.vdn_status_string.argtypes = [I]
@@ -216,37 +223,44 @@ def workspace_bytes(layout: Layout, dtype: torch.dtype) -> int:
 
 
 def window_softmax_fwd(layout: Layout, q, k, v, k_text, v_text, o_soft=None, lse=None,
-                       want_lse=False):
-    """Softmax branch: returns o_soft (and lse [B, L, H] if want_lse)."""
-    _validate(layout, q, io=[("k", k), ("v", v)], optional_io=[("o_soft", o_soft)],
-              text=[("k_text", k_text), ("v_text", v_text)], lse=lse)
+                       want_lse=False, out_f32=False):
+    """Softmax branch: returns o_soft (and lse [B, L, H] if want_lse); o_soft in
+    the io dtype, or float32 with out_f32 (vdn_window_softmax_fwd_f32out)."""
+    _validate(layout, q, io=[("k", k), ("v", v)], text=[("k_text", k_text), ("v_text", v_text)],
+              lse=lse)
+    _expect("o_soft", o_soft, tuple(q.shape), torch.float32 if out_f32 else q.dtype, required=False)
+    _same_device(q, o_soft)
     _require_cuda()
     if o_soft is None:
-        o_soft = torch.empty_like(q)
+        o_soft = torch.empty(q.shape, dtype=torch.float32 if out_f32 else q.dtype, device=q.device)
     if want_lse and lse is None:
         lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
-    code = lib().vdn_window_softmax_fwd(
-        ctypes.byref(_clayout(layout)), _dtype_code(q), _ptr(q), _ptr(k), _ptr(v),
-        _ptr(k_text), _ptr(v_text), _ptr(o_soft), _ptr(lse), _stream(q.device))
-    _check(code, "vdn_window_softmax_fwd")
+    fn = lib().vdn_window_softmax_fwd_f32out if out_f32 else lib().vdn_window_softmax_fwd
+    code = fn(ctypes.byref(_clayout(layout)), _dtype_code(q), _ptr(q), _ptr(k), _ptr(v),
+              _ptr(k_text), _ptr(v_text), _ptr(o_soft), _ptr(lse), _stream(q.device))
+    _check(code, "vdn_window_softmax_fwd" + ("_f32out" if out_f32 else ""))
     return (o_soft, lse) if want_lse else o_soft
 
 
 def vda_scan_fwd(layout: Layout, q, k, v, k_text, v_text, beta, beta_text, o_lin=None,
-                 chunk_states=None, want_states=False, workspace=None, alpha=None):
+                 chunk_states=None, want_states=False, workspace=None, alpha=None, out_f32=False):
     """Linear branch: returns o_lin (ungated, pre-norm) and, if want_states, the
     chunk table [B, H, 2, J, d, d] float32. alpha (optional, [B, F, H, d]
-    float32) decays the state per key channel before each frame's write."""
-    _validate(layout, q, io=[("k", k), ("v", v)], optional_io=[("o_lin", o_lin)],
-              text=[("k_text", k_text), ("v_text", v_text)], beta=beta, beta_text=beta_text,
-              alpha=alpha, chunk_states=chunk_states)
+    float32) decays the state per key channel before each frame's write.
+    out_f32: o_lin in float32 (vdn_vda_scan_fwd_f32out; not with alpha)."""
+    _validate(layout, q, io=[("k", k), ("v", v)], text=[("k_text", k_text), ("v_text", v_text)],
+              beta=beta, beta_text=beta_text, alpha=alpha, chunk_states=chunk_states)
+    _expect("o_lin", o_lin, tuple(q.shape), torch.float32 if out_f32 else q.dtype, required=False)
+    _same_device(q, o_lin)
+    if out_f32 and alpha is not None:
+        raise ValueError("out_f32 is not offered with alpha")
     _expect("beta", beta, (layout.B, layout.F * layout.N, layout.H), torch.float32)
     _expect("beta_text", beta_text, (layout.B, layout.T, layout.H), torch.float32,
             required=layout.T > 0)
     _validate_workspace(workspace, q)
     _require_cuda()
     if o_lin is None:
-        o_lin = torch.empty_like(q)
+        o_lin = torch.empty(q.shape, dtype=torch.float32 if out_f32 else q.dtype, device=q.device)
     if want_states and chunk_states is None:
         J = -(-layout.F // layout.c)
         chunk_states = torch.empty((layout.B, layout.H, 2, J, layout.d, layout.d),
@@ -256,7 +270,9 @@ def vda_scan_fwd(layout: Layout, q, k, v, k_text, v_text, beta, beta_text, o_lin
     head = [ctypes.byref(_clayout(layout)), _dtype_code(q), _ptr(q), _ptr(k), _ptr(v),
             _ptr(k_text), _ptr(v_text), _ptr(beta), _ptr(beta_text)]
     tail = [_ptr(o_lin), _ptr(chunk_states), _ptr(workspace), workspace.numel(), _stream(q.device)]
-    if alpha is None:
+    if out_f32:
+        code, name = lib().vdn_vda_scan_fwd_f32out(*head, *tail), "vdn_vda_scan_fwd_f32out"
+    elif alpha is None:
         code, name = lib().vdn_vda_scan_fwd(*head, *tail), "vdn_vda_scan_fwd"
     else:
         code = lib().vdn_vda_scan_fwd_decay(*head, _ptr(alpha), *tail)
@@ -375,6 +391,35 @@ def vda_scan_fwd_noalloc(layout: Layout, q, k, v, k_text, v_text, beta, beta_tex
              _ptr(chunk_states), _stream(q.device))
     _check(code, "vdn_vda_scan_fwd_noalloc")
     return o_lin
+
+
+def gated_combine_fwd(o_soft, o_lin, g_soft, g_lin, rms_weight=None, rms_eps=1e-6, out=None):
+    """out = sigmoid(g_soft) o_soft + sigmoid(g_lin) RMSNorm(o_lin) over the last
+    dimension (vdn_gated_combine_fwd). o_soft, o_lin: float32 [..., H, d] (the
+    _f32out branch outputs); g_soft, g_lin (and out) of the same shape in the io
+    dtype; rms_weight [d] float32; one device. Returns out."""
+    if g_soft is None:
+        raise ValueError("g_soft is required")
+    dt = _io_dtype(g_soft)
+    shape = tuple(g_soft.shape)
+    if len(shape) < 2:
+        raise ValueError("tensors must be [..., H, d]")
+    _expect("o_soft", o_soft, shape, torch.float32)
+    _expect("o_lin", o_lin, shape, torch.float32)
+    _expect("g_lin", g_lin, shape, dt)
+    _expect("out", out, shape, dt, required=False)
+    _expect("rms_weight", rms_weight, (shape[-1],), torch.float32, required=False)
+    _same_device(o_soft, o_lin, g_soft, g_lin, rms_weight, out)
+    _require_cuda()
+    if out is None:
+        out = torch.empty_like(g_soft)
+    H, d = shape[-2], shape[-1]
+    tokens = g_soft.numel() // (H * d) if H * d else 0
+    code = lib().vdn_gated_combine_fwd(tokens, H, d, _dtype_code(g_soft), _ptr(o_soft), _ptr(o_lin),
+                                       _ptr(g_soft), _ptr(g_lin), _ptr(rms_weight),
+                                       ctypes.c_float(rms_eps), _ptr(out), _stream(g_soft.device))
+    _check(code, "vdn_gated_combine_fwd")
+    return out
 
 
 def device_status() -> int:
