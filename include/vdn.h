@@ -86,7 +86,8 @@ typedef enum {
   VDN_ERR_UNSUPPORTED = 2,
   VDN_ERR_WORKSPACE = 3,
   VDN_ERR_CUDA = 4,
-  VDN_ERR_TIMEOUT = 5
+  VDN_ERR_TIMEOUT = 5,
+  VDN_ERR_BOUNDS = 6   /* only from a library built with bound checks (see below) */
 } vdn_status_t;
 
 /* Bytes of device workspace that vdn_vda_scan_fwd and vdn_hybrid_attn_fwd (and
@@ -320,6 +321,18 @@ int vdn_device_status(void);
 
 /* Static string for a status code. */
 const char* vdn_status_string(int status);
+
+/* Limit, in nanoseconds, of the bounded waits between the roles of the
+ * tensor-core kernels (producer, MMA issuer, softmax / scaler / drain warps):
+ * default 4 s; ns = 0 restores it. Process-wide for the current device; set it
+ * only while no call of this library is in flight. It exists to exercise the
+ * failure path without a fault: with a limit of a few nanoseconds a kernel
+ * gives up its waits, records VDN_ERR_TIMEOUT (vdn_device_status), leaves its
+ * tile unfinished and exits cleanly. The waits in which a kernel drains its own
+ * copies and MMAs before exit keep the 4 s limit, so no copy lands in shared
+ * memory of an exited block and no MMA writes freed TMEM. Returns VDN_OK or
+ * VDN_ERR_CUDA. */
+int vdn_set_wait_limit_ns(unsigned long long ns);
 
 /* The CUDA runtime's description of the error behind the last VDN_ERR_CUDA
  * returned on the calling host thread (by any entry point), or "no CUDA

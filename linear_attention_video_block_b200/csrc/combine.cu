@@ -19,6 +19,17 @@
 #include "vdn_internal.cuh"
 
 namespace vdn {
+
+// Device status word of this translation unit (bound checks of the checked build).
+__device__ int g_combine_status = 0;
+
+cudaError_t read_and_clear_combine_status(int* status) {
+  cudaError_t e = cudaMemcpyFromSymbol(status, g_combine_status, sizeof(int));
+  if (e != cudaSuccess) return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_combine_status, &zero, sizeof(int));
+}
+
 namespace {
 
 constexpr int kCombineThreads = 256;
@@ -79,7 +90,7 @@ combine_kernel(long long rows, const float* __restrict__ o_soft, const float* __
        r0 += (long long)gridDim.x * kRowsPerBlock) {
     const long long row = r0 + threadIdx.x / kLanes;
     // rows past the end still take part in the shuffles (with zeros)
-    const bool live = row < rows;
+    const bool live = row < rows && VDN_IN_BOUNDS(c0 + 8 <= D, &g_combine_status);
     const long long off = (live ? row : 0) * D + c0;
     float lin[8], ss = 0.f;
     if (live) Vec8<float>::load(o_lin + off, lin);

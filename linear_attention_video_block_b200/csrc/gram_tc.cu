@@ -28,6 +28,8 @@ namespace vdn {
 
 __device__ int g_gram_status = 0;
 
+cudaError_t set_role_wait_gram(unsigned long long ns) { return set_role_wait_ns(ns); }
+
 cudaError_t read_and_clear_gram_status(int* status) {
   cudaError_t e = cudaMemcpyFromSymbol(status, g_gram_status, sizeof(int));
   if (e != cudaSuccess) return e;
@@ -213,6 +215,7 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     auto beta_of = [&](int t) -> float {
       const int tok = t * kTok + r;
       if (tok >= U) return 0.f;
+      if (!VDN_IN_BOUNDS(text || row0 + tok < l.L(), &g_gram_status)) return 0.f;
       return text ? beta_t[((long long)b * l.T + tok) * l.H + h]
                   : beta[((long long)b * l.L() + row0 + tok) * l.H + h];
     };
@@ -264,6 +267,7 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       const int m = 32 * (warp & 3) + lane;  // TMEM lane = output row
       const uint32_t taddr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
       const long long slot = ((long long)b * l.H + h) * l.F + f;
+      const bool slot_ok = VDN_IN_BOUNDS(f >= 0 && f < l.F && h < l.H && b < l.B, &g_gram_status);
       float* arow;
       float* brow;
       if (D == 128) {
@@ -279,7 +283,7 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         tmem_ld_x32(taddr + c0, r);
         float4* dst = reinterpret_cast<float4*>(arow + c0);
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 8 && slot_ok; ++i)
           dst[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
                                __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
       }
@@ -290,7 +294,7 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
           tmem_ld_x32(taddr + 128 + c0, r);
           float4* dst = reinterpret_cast<float4*>(brow + c0);
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
+          for (int i = 0; i < 8 && slot_ok; ++i)
             dst[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
                                  __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
         }

@@ -11,6 +11,17 @@
 #include "vdn_internal.cuh"
 
 namespace vdn {
+
+// Device status word of this translation unit (bound checks of the checked build).
+__device__ int g_ro32_status = 0;
+
+cudaError_t read_and_clear_ro32_status(int* status) {
+  cudaError_t e = cudaMemcpyFromSymbol(status, g_ro32_status, sizeof(int));
+  if (e != cudaSuccess) return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_ro32_status, &zero, sizeof(int));
+}
+
 namespace {
 
 constexpr int BQ = 64;
@@ -34,7 +45,7 @@ readout_kernel(Layout l, int mode, const T* __restrict__ q, const float* __restr
   if (g < 0) return;
   const Group G = make_group(l, g);
   const int rows_valid = min(BQ, G.q0 + G.nq - r0);
-  const bool has_lin = G.chunk >= 0;
+  const bool has_lin = G.chunk >= 0 && VDN_IN_BOUNDS(G.chunk < l.J(), &g_ro32_status);
   const long long L = l.L();
   const long long HD = (long long)l.H * D;
   if (has_lin) {
@@ -47,7 +58,8 @@ readout_kernel(Layout l, int mode, const T* __restrict__ q, const float* __restr
     }
     for (int i = tid; i < BQ * D; i += NT) {
       int r = i / D, cidx = i % D;
-      qs[i] = (r < rows_valid) ? to_f32(q[((long long)b * L + r0 + r) * HD + (long long)h * D + cidx]) : 0.f;
+      const bool in = r < rows_valid && VDN_IN_BOUNDS(r0 + r < L, &g_ro32_status);
+      qs[i] = in ? to_f32(q[((long long)b * L + r0 + r) * HD + (long long)h * D + cidx]) : 0.f;
     }
   }
   __syncthreads();
@@ -70,7 +82,7 @@ readout_kernel(Layout l, int mode, const T* __restrict__ q, const float* __restr
   for (int i = 0; i < OC; ++i) ss = fmaf(acc[i], acc[i], ss);
   ss += __shfl_xor_sync(0xffffffffu, ss, 1);
   ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-  if (row >= rows_valid) return;
+  if (row >= rows_valid || !VDN_IN_BOUNDS(r0 + row < L, &g_ro32_status)) return;
   const long long base = ((long long)b * L + r0 + row) * HD + (long long)h * D + c0;
   if (mode == 0) {
 #pragma unroll

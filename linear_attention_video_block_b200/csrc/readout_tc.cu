@@ -28,6 +28,8 @@ namespace vdn {
 
 __device__ int g_readout_status = 0;
 
+cudaError_t set_role_wait_readout(unsigned long long ns) { return set_role_wait_ns(ns); }
+
 cudaError_t read_and_clear_readout_status(int* status) {
   cudaError_t e = cudaMemcpyFromSymbol(status, g_readout_status, sizeof(int));
   if (e != cudaSuccess) return e;
@@ -143,6 +145,7 @@ readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Layout l,
     // boundary frame: no linear readout
     for (int i = threadIdx.x; i < rows * (D / 8); i += kThreads) {
       const int r = i / (D / 8), c = i % (D / 8);
+      if (!VDN_IN_BOUNDS(r0 + r < l.L(), &g_readout_status)) continue;
       const long long off = ((long long)b * l.L() + r0 + r) * HD + (long long)h * D + c * 8;
       if constexpr (kCombine) {
         const float4 o0 = *reinterpret_cast<const float4*>(cx.o_soft + off);
@@ -244,6 +247,7 @@ readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Layout l,
     // stage S_sum (hi, lo) once
     {
       const int J = l.J();
+      VDN_IN_BOUNDS(G.chunk < J, &g_readout_status);
       const float* sf = states + ((((long long)b * l.H + h) * 2 + 0) * J + G.chunk) * D * D;
       const float* sr = states + ((((long long)b * l.H + h) * 2 + 1) * J + G.chunk) * D * D;
       constexpr int kChunks = D / 8;
@@ -280,7 +284,7 @@ readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Layout l,
       if (!__all_sync(0xffffffffu, rwait(&bars->d_full[s], use & 1, abort))) break;
       tc_fence_after();
       const int grow = r0 + t * kRows + m;
-      const bool store = grow < G.q0 + G.nq;
+      const bool store = grow < G.q0 + G.nq && VDN_IN_BOUNDS(grow >= 0 && grow < l.L(), &g_readout_status);
       const long long rbase = ((long long)b * l.L() + grow) * HD + (long long)h * D;
       if constexpr (kCombine) {
         // RMSNorm statistic of the row, then the gated sum in 32-column pieces

@@ -13,7 +13,19 @@
 namespace vdn {
 namespace {
 
+// Limit of the bounded waits. The waits between the roles of a kernel use
+// g_role_wait_ns (default kWaitLimitNs; set_role_wait_ns changes it, for tests
+// of the failure path); the waits that drain a kernel's own copies and MMAs
+// before it exits always use kWaitLimitNs, so that no copy can land in the
+// shared memory of a CTA that has left and no MMA can write freed TMEM.
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;
+__device__ unsigned long long g_role_wait_ns = kWaitLimitNs;
+
+// Sets this translation unit's role-wait limit (0: the default).
+cudaError_t set_role_wait_ns(unsigned long long ns) {
+  const unsigned long long v = ns ? ns : kWaitLimitNs;
+  return cudaMemcpyToSymbol(g_role_wait_ns, &v, sizeof(v));
+}
 
 // ------------------------------------------------------------- PTX wrappers
 
@@ -46,25 +58,44 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking probe of the phase (mbarrier.test_wait never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ unsigned long long global_ns() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
 
-// Waits for the phase of `bar` with the given parity to complete. Gives up when
-// another role has aborted (if watch_abort) or after kWaitLimitNs, in which case
+// Waits for the phase of `bar` with the given parity to complete. A role wait
+// (watch_abort) gives up when another role has aborted or after
+// g_role_wait_ns; a drain wait (!watch_abort) after kWaitLimitNs. On a timeout
 // it records VDN_ERR_TIMEOUT in *status and raises the CTA's abort flag.
+// With a shortened role limit (tests of this path) the loop polls without
+// suspending and checks the clock on every probe, so that a wait gives up as
+// soon as its limit has passed.
 __device__ __noinline__ bool mbar_wait_impl(unsigned long long* bar, uint32_t parity,
                                             volatile int* abort, int* status, bool watch_abort) {
   const uint32_t addr = smem_u32(bar);
-  if (mbar_try_wait(addr, parity)) return true;
+  const unsigned long long limit = watch_abort ? g_role_wait_ns : kWaitLimitNs;
+  const bool eager = limit < kWaitLimitNs;
+  if (!eager && mbar_try_wait(addr, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(addr, parity)) return true;
-    if ((i & 63u) == 0u) {
+    if (eager ? mbar_test_wait(addr, parity) : mbar_try_wait(addr, parity)) return true;
+    if (eager || (i & 63u) == 0u) {
       if (watch_abort && *abort) return false;
-      if (global_ns() - t0 > kWaitLimitNs) {
+      if (global_ns() - t0 > limit) {
         atomicCAS(status, 0, (int)VDN_ERR_TIMEOUT);
         *abort = 1;
         return false;

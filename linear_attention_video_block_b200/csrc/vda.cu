@@ -18,6 +18,17 @@
 #include "vdn_internal.cuh"
 
 namespace vdn {
+
+// Device status word of this translation unit (bound checks of the checked build).
+__device__ int g_vda_status = 0;
+
+cudaError_t read_and_clear_vda_status(int* status) {
+  cudaError_t e = cudaMemcpyFromSymbol(status, g_vda_status, sizeof(int));
+  if (e != cudaSuccess) return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_vda_status, &zero, sizeof(int));
+}
+
 namespace {
 
 constexpr int NT = 256;
@@ -74,7 +85,7 @@ gram_kernel(Layout l, SlotMap sm_map, const T* __restrict__ k, const T* __restri
     for (int i = tid; i < TU * D; i += NT) {
       int r = i / D, cidx = i % D;
       float kx = 0.f, vx = 0.f, bx = 0.f;
-      if (r < nu) {
+      if (r < nu && VDN_IN_BOUNDS(u0 + r < U && (text || f * l.N + u0 + r < l.L()), &g_vda_status)) {
         long long off = (long long)(u0 + r) * HD + cidx;
         kx = to_f32(kp[off]);
         vx = to_f32(vp[off]);
@@ -103,6 +114,7 @@ gram_kernel(Layout l, SlotMap sm_map, const T* __restrict__ k, const T* __restri
     }
   }
   const long long slot = ((long long)b * l.H + h) * l.F + f;
+  if (!VDN_IN_BOUNDS(f >= 0 && f < l.F && h < l.H && b < l.B, &g_vda_status)) return;
   float* ao = am + slot * D * D;
   float* bo = bw + slot * D * D;
 #pragma unroll
@@ -133,6 +145,7 @@ inverse_kernel(Layout l, SlotMap sm_map, float* __restrict__ am) {
   const int h = blockIdx.y, b = blockIdx.z;
   const int f = sm_map.frame(blockIdx.x);
   const long long slot = ((long long)b * l.H + h) * l.F + f;
+  if (!VDN_IN_BOUNDS(f >= 0 && f < l.F && h < l.H && b < l.B, &g_vda_status)) return;
   float* g = am + slot * D * D;
   float a[RA][RA];
 #pragma unroll
@@ -240,6 +253,7 @@ scan_kernel(Layout l, int fwd_max, int rev_min, int has_text, const float* __res
   // global chunk sequence q = t * NCH + c: rows 16c..16c+15 of M_{frame_of(t)}
   auto load_chunk = [&](int q) {
     const int t = q / NCH, c = q % NCH;
+    VDN_IN_BOUNDS(frame_of(t) >= 0 && frame_of(t) < l.F, &g_vda_status);
     const float* src = am_bh + (long long)frame_of(t) * D * D + (long long)c * CH * D;
     float* dst = ring[q % C::kRing];
     for (int i = tid * 4; i < CH * D; i += C::kThreads * 4) cp_async16(dst + i, src + i);
@@ -256,6 +270,7 @@ scan_kernel(Layout l, int fwd_max, int rev_min, int has_text, const float* __res
       if (G.nq == 0) continue;
       const int want = dir == 0 ? G.fwd_idx : G.rev_idx;
       if (want != idx) continue;
+      if (!VDN_IN_BOUNDS(j < J && row0 + R <= D, &g_vda_status)) continue;
       float* dst = st_bh + (long long)j * D * D;
 #pragma unroll
       for (int r = 0; r < RR; ++r)

@@ -327,13 +327,29 @@ int vdn_gated_combine_fwd(long long tokens, int H, int d, int dtype, const float
 
 int vdn_device_status(void) {
   if (cuda_status(cudaDeviceSynchronize()) != VDN_OK) return VDN_ERR_CUDA;
-  int s[4] = {0, 0, 0, 0};
-  if (cuda_status(vdn::read_and_clear_tc_status(&s[0])) != VDN_OK) return VDN_ERR_CUDA;
-  if (cuda_status(vdn::read_and_clear_gram_status(&s[1])) != VDN_OK) return VDN_ERR_CUDA;
-  if (cuda_status(vdn::read_and_clear_readout_status(&s[2])) != VDN_OK) return VDN_ERR_CUDA;
-  if (cuda_status(vdn::read_and_clear_fp8_status(&s[3])) != VDN_OK) return VDN_ERR_CUDA;
-  for (int i = 0; i < 4; ++i)
+  cudaError_t (*const readers[])(int*) = {
+      vdn::read_and_clear_tc_status,   vdn::read_and_clear_gram_status,
+      vdn::read_and_clear_readout_status, vdn::read_and_clear_fp8_status,
+      vdn::read_and_clear_simt_status, vdn::read_and_clear_vda_status,
+      vdn::read_and_clear_ro32_status, vdn::read_and_clear_combine_status};
+  constexpr int kReaders = sizeof(readers) / sizeof(readers[0]);
+  int s[kReaders] = {};
+  for (int i = 0; i < kReaders; ++i)
+    if (cuda_status(readers[i](&s[i])) != VDN_OK) return VDN_ERR_CUDA;
+  for (int i = 0; i < kReaders; ++i)
     if (s[i] != 0) return s[i];
+  return VDN_OK;
+}
+
+int vdn_set_wait_limit_ns(unsigned long long ns) {
+  cudaError_t (*const setters[])(unsigned long long) = {vdn::set_role_wait_tc,
+                                                        vdn::set_role_wait_gram,
+                                                        vdn::set_role_wait_readout,
+                                                        vdn::set_role_wait_fp8};
+  for (auto f : setters) {
+    const int s = cuda_status(f(ns));
+    if (s != VDN_OK) return s;
+  }
   return VDN_OK;
 }
 
@@ -350,6 +366,7 @@ const char* vdn_status_string(int status) {
     case VDN_ERR_WORKSPACE: return "workspace missing or too small";
     case VDN_ERR_CUDA: return "CUDA error";
     case VDN_ERR_TIMEOUT: return "a kernel gave up a bounded wait";
+    case VDN_ERR_BOUNDS: return "a bound check of the checked build failed";
   }
   return "unknown status";
 }

@@ -68,6 +68,18 @@ inline Layout to_layout(const vdn_layout_t* l) {
 // last CUDA error (vdn_last_cuda_error) and returns VDN_ERR_CUDA.
 int cuda_status(cudaError_t e);
 
+// Bound checks of the checked build (-DVDN_BOUND_CHECKS): VDN_IN_BOUNDS(cond,
+// status) is true when cond holds; otherwise it records VDN_ERR_BOUNDS in the
+// device status word *status and is false, and the caller skips the access
+// (no trap, so a failed check never takes the GPU context down). In the
+// regular build it is the constant true and costs nothing.
+#ifdef VDN_BOUND_CHECKS
+#define VDN_IN_BOUNDS(cond, status) \
+  ((cond) ? true : (atomicCAS((status), 0, (int)VDN_ERR_BOUNDS), false))
+#else
+#define VDN_IN_BOUNDS(cond, status) true
+#endif
+
 constexpr int kCtxText = 1;
 constexpr int kCtxAudio = 2;
 
@@ -280,6 +292,19 @@ cudaError_t read_and_clear_fp8_status(int* status);
 // Reads and clears the device status word of the tcgen05 kernels' translation
 // unit (bounded waits record VDN_ERR_TIMEOUT there).
 cudaError_t read_and_clear_tc_status(int* status);
+
+// Status words of the CUDA-core kernels' translation units (only the bound
+// checks of the checked build write them).
+cudaError_t read_and_clear_simt_status(int* status);
+cudaError_t read_and_clear_vda_status(int* status);
+cudaError_t read_and_clear_ro32_status(int* status);
+cudaError_t read_and_clear_combine_status(int* status);
+
+// Role-wait limit of each tcgen05 translation unit (0: the 4 s default).
+cudaError_t set_role_wait_tc(unsigned long long ns);
+cudaError_t set_role_wait_gram(unsigned long long ns);
+cudaError_t set_role_wait_readout(unsigned long long ns);
+cudaError_t set_role_wait_fp8(unsigned long long ns);
 
 // tcgen05 frame Gram (bf16, d in {64, 128}) into the (am, bw) slots.
 bool gram_tc_supported(const Layout& l, int dtype);

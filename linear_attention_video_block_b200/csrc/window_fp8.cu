@@ -31,6 +31,8 @@ namespace vdn {
 
 __device__ int g_fp8_status = 0;
 
+cudaError_t set_role_wait_fp8(unsigned long long ns) { return set_role_wait_ns(ns); }
+
 cudaError_t read_and_clear_fp8_status(int* status) {
   cudaError_t e = cudaMemcpyFromSymbol(status, g_fp8_status, sizeof(int));
   if (e != cudaSuccess) return e;
@@ -188,6 +190,7 @@ window_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       bool ok = true;
       for (int t = 0; t < n_tiles && ok; ++t) {
         const KeyTile kt = key_tile(G, l.T, 0, t, kRows);
+        VDN_IN_BOUNDS(kt.row >= 0 && kt.row < (kt.src == kKVideo ? l.L() : l.T), &g_fp8_status);
         for (int kv = 0; kv < 2; ++kv, ++fill) {
           const int slot = fill % kSlots;
           const int use = fill / kSlots;
@@ -390,7 +393,7 @@ window_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (ok) {
       tc_fence_after();
       const int grow = r0 + kRows * w + row;
-      const bool store = grow < q_end;
+      const bool store = grow < q_end && VDN_IN_BOUNDS(grow >= 0 && grow < l.L(), &g_fp8_status);
       const float inv = v_scale / lsum;
       const long long base = (((long long)b * l.L() + grow) * l.H + h) * kD;
 #pragma unroll 1

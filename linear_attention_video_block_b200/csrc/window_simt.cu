@@ -12,6 +12,17 @@
 #include "vdn_internal.cuh"
 
 namespace vdn {
+
+// Device status word of this translation unit (bound checks of the checked build).
+__device__ int g_simt_status = 0;
+
+cudaError_t read_and_clear_simt_status(int* status) {
+  cudaError_t e = cudaMemcpyFromSymbol(status, g_simt_status, sizeof(int));
+  if (e != cudaSuccess) return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_simt_status, &zero, sizeof(int));
+}
+
 namespace {
 
 constexpr int BQ = 64;
@@ -69,7 +80,8 @@ window_simt_kernel(Layout l, const T* __restrict__ q, const T* __restrict__ k,
 
   for (int i = tid; i < BQ * D; i += NT) {
     int r = i / D, cidx = i % D;
-    sm.q[r][cidx] = (r < rows_valid) ? to_f32(qb[(long long)(r0 + r) * HD + cidx]) : 0.f;
+    const bool in = r < rows_valid && VDN_IN_BOUNDS(r0 + r < qrows, &g_simt_status);
+    sm.q[r][cidx] = in ? to_f32(qb[(long long)(r0 + r) * HD + cidx]) : 0.f;
   }
   // Score mapping: thread (ty, tx) owns rows ty + 16m and keys tx + 16n.
   const int ty = tid / 16, tx = tid % 16;
@@ -96,7 +108,8 @@ window_simt_kernel(Layout l, const T* __restrict__ q, const T* __restrict__ k,
       for (int i = tid; i < BK * D; i += NT) {
         int r = i / D, cidx = i % D;
         float kx = 0.f, vx = 0.f;
-        if (r < kv) {
+        const long long src_rows = text ? l.T : (audio ? l.A : L);
+        if (r < kv && VDN_IN_BOUNDS(seg_start + k0 + r < src_rows, &g_simt_status)) {
           long long off = (long long)(seg_start + k0 + r) * HD + cidx;
           kx = to_f32(ks[off]);
           vx = to_f32(vs[off]);
@@ -162,7 +175,7 @@ window_simt_kernel(Layout l, const T* __restrict__ q, const T* __restrict__ k,
       }
     }
   }
-  if (orow < rows_valid) {
+  if (orow < rows_valid && VDN_IN_BOUNDS(r0 + orow < qrows, &g_simt_status)) {
     const float inv = 1.f / l_run;
     const long long rix = (long long)b * qrows + r0 + orow;
     if (G.qsrc == kQVideo) {

@@ -44,6 +44,8 @@ namespace vdn {
 // Device-side status word of this translation unit.
 __device__ int g_vdn_status = 0;
 
+cudaError_t set_role_wait_tc(unsigned long long ns) { return set_role_wait_ns(ns); }
+
 cudaError_t read_and_clear_tc_status(int* status) {
   cudaError_t e = cudaMemcpyFromSymbol(status, g_vdn_status, sizeof(int));
   if (e != cudaSuccess) return e;
@@ -188,6 +190,10 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       bool ok = true;
       for (int t = 0; t < n_tiles && ok; ++t) {
         const KeyTile kt = key_tile(G, l.T, l.A, t, kRows);
+        // checked build: the schedule's key rows lie inside their tensor (a copy
+        // past the end would read zeros, so this is a check of the schedule)
+        VDN_IN_BOUNDS(kt.row >= 0 && kt.row < (kt.src == kKVideo ? l.L() : kt.src == kKText ? l.T : l.A),
+                      &g_vdn_status);
         for (int kv = 0; kv < 2; ++kv, ++fill) {
           const int slot = fill % C::kSlots;
           const int use = fill / C::kSlots;
@@ -230,25 +236,30 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tc_fence_after();
         return r;
       };
+      // descriptors: the start address sits in the low 14 bits (address / 16),
+      // so an operand's k-step descriptors are its base descriptor plus offset / 16
+      const uint64_t qd0 = desc_k_sw128(q_addr), kvd0 = desc_k_sw128(kv_addr);
+      const uint64_t vd0 = desc_mn_sw128(kv_addr, C::kHalfBytes);
       auto issue_s = [&](int w, int slot) {
         const uint32_t d_tmem = tmem + 128 * w;
+        const uint64_t qd = qd0 + (uint64_t)((w * C::kTileBytes) >> 4);
+        const uint64_t kd = kvd0 + (uint64_t)((slot * C::kTileBytes) >> 4);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t off = (uint32_t)((ks / 4) * C::kHalfBytes + (ks % 4) * 32);
-          mma_ss(d_tmem, desc_k_sw128(q_addr + w * C::kTileBytes + off),
-                 desc_k_sw128(kv_addr + slot * C::kTileBytes + off), idesc_s, ks > 0 ? 1u : 0u);
+          const uint32_t off = (uint32_t)((ks / 4) * C::kHalfBytes + (ks % 4) * 32) >> 4;
+          mma_ss(d_tmem, qd + off, kd + off, idesc_s, ks > 0 ? 1u : 0u);
         }
       };
       // O_w += P_w V for one half of the key tile (keys 64 half .. 64 half + 63)
       auto issue_pv_half = [&](int w, int slot, bool acc, int half) {
         const uint32_t d_tmem = tmem + 256 + D * w;
         const uint32_t a_tmem = tmem + 128 * w;
+        const uint64_t vd = vd0 + (uint64_t)((slot * C::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kRows / 32; ++kk) {
           const int ks = 4 * half + kk;
-          mma_ts(d_tmem, a_tmem + ks * 8,
-                 desc_mn_sw128(kv_addr + slot * C::kTileBytes + ks * 16 * 128, C::kHalfBytes),
-                 idesc_o, (acc || ks > 0) ? 1u : 0u);
+          mma_ts(d_tmem, a_tmem + ks * 8, vd + (uint64_t)(ks * 16 * 128 / 16), idesc_o,
+                 (acc || ks > 0) ? 1u : 0u);
         }
       };
       // P_w(t) is published in two halves; the first half's P.V runs while the
@@ -409,6 +420,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       // audio [B, A, H, D]
       const long long qrows = G.qsrc == kQVideo ? l.L() : (G.qsrc == kQText ? l.T : l.A);
       const long long base = (((long long)b * qrows + grow) * l.H + h) * D;
+      const bool store_ok = !store || VDN_IN_BOUNDS(grow >= 0 && grow < qrows, &g_vdn_status);
       {
         void* dst_o = out;
         float* dst_lse = lse;
@@ -422,7 +434,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t o[32];
           tmem_ld_x32(tO + c0, o);
-          if (store) {
+          if (store && store_ok) {
             if (f32) {
               float4* dst = reinterpret_cast<float4*>(static_cast<float*>(dst_o) + base + c0);
 #pragma unroll
@@ -440,7 +452,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
           }
         }
-        if (store && dst_lse)
+        if (store && store_ok && dst_lse)
           dst_lse[((long long)b * qrows + grow) * l.H + h] = (m + log2f(lsum)) * 0.6931471805599453f;
       }
     }

@@ -65,6 +65,10 @@ WORKLOADS = {
     # profiling case: the 768p-like token grid with 4 heads (inputs 149 MB per
     # video tensor, above the 126 MB L2, a few GB on the device in total)
     "768p-h4-bf16": (Layout(B=1, F=36, N=4032, T=512, c=5, H=4, d=128), "bf16", 3),
+    # profiling case for the linear branch's kernels: 12 heads fill the GPU
+    # (420 Gram / inverse CTAs, 192 scan CTAs) with inputs of 446 MB per video
+    # tensor, a few GB on the device in total
+    "768p-h12-bf16": (Layout(B=1, F=36, N=4032, T=512, c=5, H=12, d=128), "bf16", 3),
 }
 
 TORCH_DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16}

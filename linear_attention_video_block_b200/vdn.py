@@ -29,13 +29,15 @@ _lib = None
 
 VDN_F32, VDN_BF16 = 0, 1
 STATUS = {0: "VDN_OK", 1: "VDN_ERR_INVALID", 2: "VDN_ERR_UNSUPPORTED",
-          3: "VDN_ERR_WORKSPACE", 4: "VDN_ERR_CUDA", 5: "VDN_ERR_TIMEOUT"}
+          3: "VDN_ERR_WORKSPACE", 4: "VDN_ERR_CUDA", 5: "VDN_ERR_TIMEOUT",
+          6: "VDN_ERR_BOUNDS"}
 EXPORTS = ("vdn_workspace_bytes", "vdn_window_softmax_fwd", "vdn_vda_scan_fwd",
            "vdn_vda_scan_fwd_decay", "vdn_hybrid_attn_fwd", "vdn_hybrid_attn_fwd_decay",
            "vdn_vda_scan_fwd_noalloc", "vdn_joint_softmax_fwd", "vdn_joint_attn_fwd",
            "vdn_window_softmax_fwd_fp8", "vdn_hybrid_attn_fwd_host",
            "vdn_hybrid_host_workspace_bytes", "vdn_gated_combine_fwd",
-           "vdn_window_softmax_fwd_f32out", "vdn_vda_scan_fwd_f32out", "vdn_device_status",
+           "vdn_window_softmax_fwd_f32out", "vdn_vda_scan_fwd_f32out", "vdn_set_wait_limit_ns",
+           "vdn_device_status",
            "vdn_status_string", "vdn_last_cuda_error")
 
 
@@ -101,6 +103,8 @@ def lib():
         L.vdn_vda_scan_fwd_f32out.restype = I
         L.vdn_gated_combine_fwd.argtypes = [ctypes.c_longlong, I, I, I] + [P] * 5 + [F, P, P]
         L.vdn_gated_combine_fwd.restype = I
+        L.vdn_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+        L.vdn_set_wait_limit_ns.restype = I
         L.vdn_device_status.argtypes = []
         L.vdn_device_status.restype = I
         L.vdn_status_string.argtypes = [I]
@@ -420,6 +424,13 @@ def gated_combine_fwd(o_soft, o_lin, g_soft, g_lin, rms_weight=None, rms_eps=1e-
                                        ctypes.c_float(rms_eps), _ptr(out), _stream(g_soft.device))
     _check(code, "vdn_gated_combine_fwd")
     return out
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    """Limit of the tensor-core kernels' role waits (vdn_set_wait_limit_ns; 0:
+    the 4 s default). For tests of the timeout path only."""
+    _require_cuda()
+    _check(lib().vdn_set_wait_limit_ns(int(ns)), "vdn_set_wait_limit_ns")
 
 
 def device_status() -> int:

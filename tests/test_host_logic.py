@@ -36,7 +36,7 @@ def test_library_exports_every_declared_function(lib):
 
 
 def test_status_strings(lib):
-    for code in range(6):
+    for code in range(7):
         assert lib.vdn_status_string(code)
     assert lib.vdn_status_string(99) == b"unknown status"
     assert lib.vdn_last_cuda_error() == b"no CUDA error"
