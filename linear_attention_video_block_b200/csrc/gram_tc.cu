@@ -22,6 +22,14 @@
 //   d = 64:  one M = 128 MMA with [K^T; V^T] stacked along M (the V tile sits
 //            one leading-byte-offset after the K tile): lanes 0-63 = A, 64-127 = B.
 // The work is HBM-bound: each token's k and v are read once.
+//
+// Epilogue: B_f goes to global memory; A_f is staged in the freed shared rings
+// and all 256 threads (warps 6-7 join here) invert I + A_f in place with the
+// register-blocked Gauss-Jordan of spd_inverse.cuh, writing M_f = (I + A_f)^-1
+// to the am slot. The inverse is a latency-bound chain of d dependent pivots;
+// done here, it overlaps the other CTA of the SM streaming its frame instead
+// of running as a separate launch after every Gram has finished.
+#include "spd_inverse.cuh"
 #include "tc_common.cuh"
 
 namespace vdn {
@@ -40,7 +48,7 @@ cudaError_t read_and_clear_gram_status(int* status) {
 namespace {
 
 constexpr int kTok = 32;        // tokens per tile (96 KB of stages: two CTAs per SM)
-constexpr int kThreads = 192;
+constexpr int kThreads = 256;  // warps 6-7 join only the in-place inverse
 constexpr int kHalfBytes = kTok * 128;  // kTok tokens x 64 bf16 (one swizzle atom column)
 
 template <int D>
@@ -53,6 +61,12 @@ struct GCfg {
   static constexpr int kKwSlots = 2;
   static constexpr int kTmemCols = (D == 128) ? 256 : 64;
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kKwSlots * kKwBytes + 256;
+  // after the last MMA the K/V ring and Kw slots are free: I + A is staged there
+  // (row stride kAStride floats, padded against bank conflicts) for the inverse,
+  // followed by the inverse's pivot row / column buffers
+  static constexpr int kAStride = D + 4;
+  static_assert(D * kAStride * 4 + 4 * D * 4 <= kStages * kStageBytes + kKwSlots * kKwBytes,
+                "the inverse's staging must fit in the freed rings");
 };
 
 struct GBars {
@@ -204,7 +218,7 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       tc_commit(&bars->done);
       if (!ok) gwait(&bars->done, 0, abort, false);
     }
-  } else {
+  } else if (warp < 6) {
     // ---------------------------------------------------- scalers / epilogue
     // 4 threads per token row, each scaling (D / 8) / 4 of the row's 16-byte chunks;
     // beta of the next tile is fetched one tile ahead (it is a strided 4-byte read)
@@ -268,13 +282,18 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       const uint32_t taddr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
       const long long slot = ((long long)b * l.H + h) * l.F + f;
       const bool slot_ok = VDN_IN_BOUNDS(f >= 0 && f < l.F && h < l.H && b < l.B, &g_gram_status);
+      // A_f (rows of TMEM columns 0..D-1 for d = 128, lanes 0..63 for d = 64) goes
+      // to the shared staging of the inverse, B_f to global memory; the staging
+      // reuses ring memory last touched by the copies and the tensor cores
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      float* as = reinterpret_cast<float*>(smem);
       float* arow;
       float* brow;
       if (D == 128) {
-        arow = am + slot * D * D + (long long)m * D;
+        arow = as + m * C::kAStride;
         brow = bw + slot * D * D + (long long)m * D;
       } else {
-        arow = (m < 64) ? am + slot * D * D + (long long)m * D : bw + slot * D * D + (long long)(m - 64) * D;
+        arow = (m < 64) ? as + m * C::kAStride : bw + slot * D * D + (long long)(m - 64) * D;
         brow = nullptr;
       }
 #pragma unroll 1
@@ -308,6 +327,33 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::kTmemCols)
                  : "memory");
+  }
+  // M_f = (I + A_f)^-1 in place of A_f, by all 256 threads (spd_inverse.cuh),
+  // while the other CTA on the SM streams its frame; skipped as a whole when a
+  // role gave up (the staging is then incomplete)
+  if (*abort) return;
+  {
+    constexpr int RA = D / 16;
+    const float* as = reinterpret_cast<const float*>(smem);
+    float (*rowk)[D] = reinterpret_cast<float (*)[D]>(smem + D * C::kAStride * 4);
+    float (*colk)[D] = rowk + 2;
+    const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
+    float a[RA][RA];
+#pragma unroll
+    for (int x = 0; x < RA; ++x)
+#pragma unroll
+      for (int y = 0; y < RA; ++y) {
+        const int i = tr + 16 * x, j = tc + 16 * y;
+        a[x][y] = as[i * C::kAStride + j] + (i == j ? 1.f : 0.f);
+      }
+    spd_inverse_blocks<D>(a, tr, tc, rowk, colk);
+    const long long slot = ((long long)b * l.H + h) * l.F + f;
+    if (!VDN_IN_BOUNDS(f >= 0 && f < l.F && h < l.H && b < l.B, &g_gram_status)) return;
+    float* g = am + slot * D * D;
+#pragma unroll
+    for (int x = 0; x < RA; ++x)
+#pragma unroll
+      for (int y = 0; y < RA; ++y) g[(tr + 16 * x) * D + tc + 16 * y] = a[x][y];
   }
 }
 

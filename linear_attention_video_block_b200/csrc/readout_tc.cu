@@ -50,7 +50,12 @@ struct RCfg {
   static constexpr int kHalfBytes = kRows * 128;
   static constexpr int kTileBytes = kRows * D * 2;
   static constexpr int kTmemCols = 2 * D;
-  static constexpr int kSmemBytes = 1024 + 4 * kTileBytes + 256;  // S_hi, S_lo, 2 Q stages
+  // row stride of the drain staging in floats: padded so that the rows written
+  // by 8 consecutive lanes fall on different banks
+  static constexpr int kStgStride = D + 4;
+  // S_hi, S_lo, 2 Q stages, barriers, then the drain warps' row staging
+  // (8 warps x 16 rows)
+  static constexpr int kSmemBytes = 1024 + 4 * kTileBytes + 256 + 8 * 16 * kStgStride * 4;
 };
 
 struct RBars {
@@ -247,7 +252,7 @@ readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Layout l,
     // stage S_sum (hi, lo) once
     {
       const int J = l.J();
-      VDN_IN_BOUNDS(G.chunk < J, &g_readout_status);
+      (void)VDN_IN_BOUNDS(G.chunk < J, &g_readout_status);
       const float* sf = states + ((((long long)b * l.H + h) * 2 + 0) * J + G.chunk) * D * D;
       const float* sr = states + ((((long long)b * l.H + h) * 2 + 1) * J + G.chunk) * D * D;
       constexpr int kChunks = D / 8;
@@ -276,19 +281,36 @@ readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Layout l,
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       mbar_arrive(&bars->ssum_ready);
     }
-    // drain accumulators
-    const int m = 32 * (warp & 3) + lane;
+    // drain accumulators. TMEM holds one row per thread; global memory wants
+    // each warp access on one row. So each warp copies its 32 rows out through
+    // a shared-memory staging of 16 rows (two passes): the lanes whose rows go
+    // in this pass write them, then the warp emits the staged rows one at a
+    // time with its lanes on consecutive columns, several rows per batch so
+    // that enough loads (the combine's o_soft and gates) are in flight. The
+    // combine reads the accumulator once for the row's RMS statistic and once
+    // per pass (TMEM reads are cheap; the registers are not), and stages
+    // acc * rstd so that every lane can finish any row.
+    const int m0 = 32 * (warp & 3);
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    static_assert(sizeof(RBars) <= 256, "barriers overlap the staging");
+    float* stg = reinterpret_cast<float*>(smem + 4 * C::kTileBytes + 256) + (warp - 2) * 16 * C::kStgStride;
+    float* my_stg = stg + (lane & 15) * C::kStgStride;  // this lane's staging row
+    const bool cols_lane = 4 * lane < D;                  // lanes cover 4 columns each
+    float w4[4] = {1.f, 1.f, 1.f, 1.f};                   // RMSNorm weight of those columns
+    if constexpr (kCombine) {
+      if (cx.rms_w != nullptr && cols_lane) {
+        const float4 wv = *reinterpret_cast<const float4*>(cx.rms_w + 4 * lane);
+        w4[0] = wv.x; w4[1] = wv.y; w4[2] = wv.z; w4[3] = wv.w;
+      }
+    }
+    constexpr int kBatch = 8;  // rows emitted per batch
     for (int t = dg; t < n_tiles; t += 2) {
       const int s = t & 1, use = t >> 1;
       if (!__all_sync(0xffffffffu, rwait(&bars->d_full[s], use & 1, abort))) break;
       tc_fence_after();
-      const int grow = r0 + t * kRows + m;
-      const bool store = grow < G.q0 + G.nq && VDN_IN_BOUNDS(grow >= 0 && grow < l.L(), &g_readout_status);
-      const long long rbase = ((long long)b * l.L() + grow) * HD + (long long)h * D;
+      const uint32_t tacc = tmem + lane_base + s * D;
+      const int tile_row0 = r0 + t * kRows + m0;  // global row of lane 0's row
       if constexpr (kCombine) {
-        // RMSNorm statistic of the row, then the gated sum in 32-column pieces
-        const uint32_t tacc = tmem + lane_base + s * D;
         float ss4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
@@ -299,51 +321,101 @@ readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Layout l,
         }
         const float rstd = rsqrtf(((ss4[0] + ss4[1]) + (ss4[2] + ss4[3])) / (float)D + cx.eps);
 #pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t r[32];
-          tmem_ld_x32(tacc + c0, r);
-          if (store) {
+        for (int pass = 0; pass < 2; ++pass) {
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t r[32];
+            tmem_ld_x32(tacc + c0, r);
+            if ((lane >> 4) == pass) {
 #pragma unroll
-            for (int g8 = 0; g8 < 4; ++g8) {
-              const long long off = rbase + c0 + 8 * g8;
-              const float4 o0 = *reinterpret_cast<const float4*>(cx.o_soft + off);
-              const float4 o1 = *reinterpret_cast<const float4*>(cx.o_soft + off + 4);
-              const float o[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
-              float lin[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e)
-                lin[e] = __uint_as_float(r[8 * g8 + e]) * rstd * (cx.rms_w ? cx.rms_w[c0 + 8 * g8 + e] : 1.f);
-              combine8(cx, off, o, lin, *reinterpret_cast<const uint4*>(cx.g_soft + off),
-                       *reinterpret_cast<const uint4*>(cx.g_lin + off), true);
+              for (int c = 0; c < 32; c += 4)
+                *reinterpret_cast<float4*>(my_stg + c0 + c) =
+                    make_float4(__uint_as_float(r[c]) * rstd, __uint_as_float(r[c + 1]) * rstd,
+                                __uint_as_float(r[c + 2]) * rstd, __uint_as_float(r[c + 3]) * rstd);
             }
           }
-        }
-        tc_fence_before();
-        mbar_arrive(&bars->d_empty[s]);
-        continue;
-      }
+          if (pass == 1) {
+            tc_fence_before();
+            mbar_arrive(&bars->d_empty[s]);  // the accumulator is free for tile t + 2
+          }
+          __syncwarp();
+          const int lim = min(16, G.q0 + G.nq - (tile_row0 + 16 * pass));  // rows of the group
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld_x32(tmem + lane_base + s * D + c0, r);
-        if (kMode == 2 && store) {
-          float4* d4 = reinterpret_cast<float4*>(o_lin32 + rbase + c0);
+          for (int rb = 0; rb < lim; rb += kBatch) {
+            float4 o4[kBatch];
+            uint2 gs2[kBatch], gl2[kBatch];
+            long long off[kBatch];
+            bool ok[kBatch];
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            d4[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
-        } else if (store) {
-          uint4* d4 = reinterpret_cast<uint4*>(o_lin + rbase + c0);
+            for (int u = 0; u < kBatch; ++u) {
+              const int grow = tile_row0 + 16 * pass + rb + u;
+              ok[u] = cols_lane && rb + u < lim && VDN_IN_BOUNDS(grow >= 0 && grow < l.L(), &g_readout_status);
+              off[u] = ((long long)b * l.L() + grow) * HD + (long long)h * D + 4 * lane;
+              if (ok[u]) {
+                o4[u] = *reinterpret_cast<const float4*>(cx.o_soft + off[u]);
+                gs2[u] = *reinterpret_cast<const uint2*>(cx.g_soft + off[u]);
+                gl2[u] = *reinterpret_cast<const uint2*>(cx.g_lin + off[u]);
+              }
+            }
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            d4[i] = make_uint4(pack_bf16(__uint_as_float(r[8 * i]), __uint_as_float(r[8 * i + 1])),
-                               pack_bf16(__uint_as_float(r[8 * i + 2]), __uint_as_float(r[8 * i + 3])),
-                               pack_bf16(__uint_as_float(r[8 * i + 4]), __uint_as_float(r[8 * i + 5])),
-                               pack_bf16(__uint_as_float(r[8 * i + 6]), __uint_as_float(r[8 * i + 7])));
+            for (int u = 0; u < kBatch; ++u) {
+              if (!ok[u]) continue;
+              const float4 a4 = *reinterpret_cast<const float4*>(stg + (rb + u) * C::kStgStride + 4 * lane);
+              const float o[4] = {o4[u].x, o4[u].y, o4[u].z, o4[u].w};
+              const float lin[4] = {a4.x * w4[0], a4.y * w4[1], a4.z * w4[2], a4.w * w4[3]};
+              const float gs[4] = {bf16_lo(gs2[u].x), bf16_hi(gs2[u].x), bf16_lo(gs2[u].y), bf16_hi(gs2[u].y)};
+              const float gl[4] = {bf16_lo(gl2[u].x), bf16_hi(gl2[u].x), bf16_lo(gl2[u].y), bf16_hi(gl2[u].y)};
+              float so[4], sl[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                so[e] = sigmoid_approx(gs[e]) * o[e];
+                sl[e] = sigmoid_approx(gl[e]) * lin[e];
+              }
+              *reinterpret_cast<uint2*>(cx.out + off[u]) =
+                  make_uint2(pack_bf16(so[0] + sl[0], so[1] + sl[1]), pack_bf16(so[2] + sl[2], so[3] + sl[3]));
+              if (cx.out_soft)
+                *reinterpret_cast<uint2*>(cx.out_soft + off[u]) =
+                    make_uint2(pack_bf16(so[0], so[1]), pack_bf16(so[2], so[3]));
+              if (cx.out_lin)
+                *reinterpret_cast<uint2*>(cx.out_lin + off[u]) =
+                    make_uint2(pack_bf16(sl[0], sl[1]), pack_bf16(sl[2], sl[3]));
+            }
+          }
+          __syncwarp();  // the staging is rewritten by the next pass
+        }
+      } else {
+        // o_lin only: the whole row is taken out of TMEM at once (no loads to
+        // hold registers for), and the accumulator freed before the stores
+        uint32_t r[D];
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) tmem_ld_x32(tacc + c0, r + c0);
+        tc_fence_before();
+        mbar_arrive(&bars->d_empty[s]);  // the accumulator is free for tile t + 2
+#pragma unroll 1
+        for (int pass = 0; pass < 2; ++pass) {
+          if ((lane >> 4) == pass) {
+#pragma unroll
+            for (int c = 0; c < D; c += 4)
+              *reinterpret_cast<float4*>(my_stg + c) =
+                  make_float4(__uint_as_float(r[c]), __uint_as_float(r[c + 1]), __uint_as_float(r[c + 2]),
+                              __uint_as_float(r[c + 3]));
+          }
+          __syncwarp();
+          const int lim = min(16, G.q0 + G.nq - (tile_row0 + 16 * pass));  // rows of the group
+#pragma unroll 1
+          for (int rr = 0; rr < lim; ++rr) {
+            const int grow = tile_row0 + 16 * pass + rr;
+            if (!cols_lane || !VDN_IN_BOUNDS(grow >= 0 && grow < l.L(), &g_readout_status)) continue;
+            const long long off = ((long long)b * l.L() + grow) * HD + (long long)h * D + 4 * lane;
+            const float4 a4 = *reinterpret_cast<const float4*>(stg + rr * C::kStgStride + 4 * lane);
+            if constexpr (kMode == 2)
+              *reinterpret_cast<float4*>(o_lin32 + off) = a4;
+            else
+              *reinterpret_cast<uint2*>(o_lin + off) = make_uint2(pack_bf16(a4.x, a4.y), pack_bf16(a4.z, a4.w));
+          }
+          __syncwarp();  // the staging is rewritten by the next pass
         }
       }
-      tc_fence_before();
-      mbar_arrive(&bars->d_empty[s]);
     }
   }
   __syncwarp();

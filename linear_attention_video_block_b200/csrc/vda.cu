@@ -6,8 +6,10 @@
 //   gram     A_f = K_f^T Diag(beta_f) K_f and B_f = V_f^T Diag(beta_f) K_f for
 //            every scanned frame and for the text (slot 0), fp32 (bf16 inputs:
 //            tensor-core kernel in gram_tc.cu; fp32 inputs: CUDA-core kernel here).
-//   inverse  M_f = (I + A_f)^-1 in place of A_f (register-blocked Gauss-Jordan;
-//            I + A_f is SPD with every pivot >= 1, so no pivoting is needed).
+//   inverse  M_f = (I + A_f)^-1 in place of A_f (register-blocked Gauss-Jordan,
+//            spd_inverse.cuh; I + A_f is SPD with every pivot >= 1, so no
+//            pivoting is needed). The bf16 tensor-core Gram kernel does it in
+//            its own epilogue; the fp32 path launches inverse_kernel.
 //   scan     S <- (S Diag(alpha_f) + B_f) M_f (alpha: optional KDA decay), forward over 1..fwd_max and reverse over
 //            F-2..rev_min, from S0 = 1/2 B_T M_T. Rows of S evolve independently
 //            (the update multiplies on the right), so each CTA owns 16 rows of
@@ -15,6 +17,7 @@
 //            all CTAs are resident at once and M_f streams through a small
 //            cp.async ring.
 //            States read by each chunk are stored into [B, H, 2, J, d, d].
+#include "spd_inverse.cuh"
 #include "vdn_internal.cuh"
 
 namespace vdn {
@@ -126,14 +129,8 @@ gram_kernel(Layout l, SlotMap sm_map, const T* __restrict__ k, const T* __restri
     }
 }
 
-// In-place inverse of (I + A) for one slot: Gauss-Jordan elimination without
-// pivoting (every pivot of an SPD matrix with eigenvalues >= 1 is >= 1).
-// Step k written as a rank-1 update: with row k and column k zeroed,
-//   a <- a - c r^T,  c = column k (c_k = -1),  r = row k / p (r_k = 1/p),
-// which yields the Gauss-Jordan result in every entry. Thread (tr, tc) of a
-// 16 x 16 grid keeps the interleaved block of rows tr + 16x and columns
-// tc + 16y in registers; the pivot row and column go through double-buffered
-// shared memory, one barrier per step.
+// In-place inverse of (I + A) for one slot (spd_inverse.cuh); the bf16 path
+// does the same inside the tensor-core Gram kernel.
 template <int D>
 __global__ void __launch_bounds__(NT, 2)
 inverse_kernel(Layout l, SlotMap sm_map, float* __restrict__ am) {
@@ -155,44 +152,7 @@ inverse_kernel(Layout l, SlotMap sm_map, float* __restrict__ am) {
       const int i = tr + 16 * x, j = tc + 16 * y;
       a[x][y] = g[i * D + j] + (i == j ? 1.f : 0.f);
     }
-  // pivot k = 16 kb + kr; kb is a compile-time index into the register block
-#pragma unroll
-  for (int kb = 0; kb < RA; ++kb) {
-#pragma unroll 1
-    for (int kr = 0; kr < 16; ++kr) {
-      const int k = 16 * kb + kr;
-      const int buf = k & 1;
-      // owners publish row k and column k, then zero them in their registers
-      if (tr == kr) {
-#pragma unroll
-        for (int y = 0; y < RA; ++y) {
-          rowk[buf][tc + 16 * y] = a[kb][y];
-          a[kb][y] = 0.f;
-        }
-      }
-      if (tc == kr) {
-#pragma unroll
-        for (int x = 0; x < RA; ++x) {
-          colk[buf][tr + 16 * x] = (x == kb && tr == kr) ? -1.f : a[x][kb];
-          a[x][kb] = 0.f;
-        }
-      }
-      __syncthreads();
-      const float rp = 1.f / rowk[buf][k];
-      float r[RA], c[RA];
-#pragma unroll
-      for (int y = 0; y < RA; ++y) {
-        const int j = tc + 16 * y;
-        r[y] = (j == k) ? rp : rowk[buf][j] * rp;
-      }
-#pragma unroll
-      for (int x = 0; x < RA; ++x) c[x] = colk[buf][tr + 16 * x];
-#pragma unroll
-      for (int x = 0; x < RA; ++x)
-#pragma unroll
-        for (int y = 0; y < RA; ++y) a[x][y] = fmaf(-c[x], r[y], a[x][y]);
-    }
-  }
+  spd_inverse_blocks<D>(a, tr, tc, rowk, colk);
 #pragma unroll
   for (int x = 0; x < RA; ++x)
 #pragma unroll
@@ -253,7 +213,7 @@ scan_kernel(Layout l, int fwd_max, int rev_min, int has_text, const float* __res
   // global chunk sequence q = t * NCH + c: rows 16c..16c+15 of M_{frame_of(t)}
   auto load_chunk = [&](int q) {
     const int t = q / NCH, c = q % NCH;
-    VDN_IN_BOUNDS(frame_of(t) >= 0 && frame_of(t) < l.F, &g_vda_status);
+    (void)VDN_IN_BOUNDS(frame_of(t) >= 0 && frame_of(t) < l.F, &g_vda_status);
     const float* src = am_bh + (long long)frame_of(t) * D * D + (long long)c * CH * D;
     float* dst = ring[q % C::kRing];
     for (int i = tid * 4; i < CH * D; i += C::kThreads * 4) cp_async16(dst + i, src + i);
@@ -380,17 +340,19 @@ cudaError_t launch_states_t(const Layout& l, int dtype, const void* k, const voi
     dim3 grid(nslots, l.H, l.B);
     cudaError_t e;
     if (gram_tc_supported(l, dtype)) {
+      // the tensor-core Gram kernel also inverts I + A_f in place (am = M_f)
       e = launch_gram_tc(l, map.has_text, map.fwd_max, map.rev_lo, nslots, k, v, kt, vt, beta,
                          beta_t, am, bw, st);
+      if (e != cudaSuccess) return e;
     } else {
       gram_kernel<T, D><<<grid, NT, 0, st>>>(l, map, (const T*)k, (const T*)v, (const T*)kt,
                                              (const T*)vt, beta, beta_t, am, bw);
       e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+      inverse_kernel<D><<<grid, NT, 0, st>>>(l, map, am);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
     }
-    if (e != cudaSuccess) return e;
-    inverse_kernel<D><<<grid, NT, 0, st>>>(l, map, am);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
   }
   {
     dim3 grid(D / 16, 2, l.B * l.H);

@@ -190,7 +190,7 @@ window_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       bool ok = true;
       for (int t = 0; t < n_tiles && ok; ++t) {
         const KeyTile kt = key_tile(G, l.T, 0, t, kRows);
-        VDN_IN_BOUNDS(kt.row >= 0 && kt.row < (kt.src == kKVideo ? l.L() : l.T), &g_fp8_status);
+        (void)VDN_IN_BOUNDS(kt.row >= 0 && kt.row < (kt.src == kKVideo ? l.L() : l.T), &g_fp8_status);
         for (int kv = 0; kv < 2; ++kv, ++fill) {
           const int slot = fill % kSlots;
           const int use = fill / kSlots;

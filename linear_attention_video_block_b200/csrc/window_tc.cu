@@ -192,7 +192,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const KeyTile kt = key_tile(G, l.T, l.A, t, kRows);
         // checked build: the schedule's key rows lie inside their tensor (a copy
         // past the end would read zeros, so this is a check of the schedule)
-        VDN_IN_BOUNDS(kt.row >= 0 && kt.row < (kt.src == kKVideo ? l.L() : kt.src == kKText ? l.T : l.A),
+        (void)VDN_IN_BOUNDS(kt.row >= 0 && kt.row < (kt.src == kKVideo ? l.L() : kt.src == kKText ? l.T : l.A),
                       &g_vdn_status);
         for (int kv = 0; kv < 2; ++kv, ++fill) {
           const int slot = fill % C::kSlots;
