@@ -16,9 +16,10 @@
 //              past the frame (which also masks the ragged last tile); then the
 //              epilogue reads A and B out of TMEM.
 // Both MMA operands are MN-major (token = K dimension, contiguous along d):
-//   d = 128: D_A[i][j] += sum_u K[u][i] Kw[u][j] (TMEM columns 0..127) and
-//            D_B[i][j] += sum_u V[u][i] Kw[u][j] (columns 128..255), each as the
-//            two MMAs with Kw_hi and Kw_lo;
+//   d = 128: one M = 128, N = 256 MMA per Kw part (hi, lo) and 16 tokens,
+//            D[j][n] += sum_u Kw[u][j] [K | V][u][n]: columns 0..127 hold
+//            A_f[j][n] (A_f is symmetric), columns 128..255 hold B_f[n][j],
+//            i.e. TMEM lane j holds row j of A_f and column j of B_f;
 //   d = 64:  one M = 128 MMA with [K^T; V^T] stacked along M (the V tile sits
 //            one leading-byte-offset after the K tile): lanes 0-63 = A, 64-127 = B.
 // The work is HBM-bound: each token's k and v are read once.
@@ -182,7 +183,8 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------------------------------------------------- MMA issuer
-      constexpr uint32_t idesc = idesc_mn_mn(D);
+      constexpr uint32_t idesc = idesc_mn_mn(D);      // d = 64: M = 128 ([K^T; V^T]), N = 64
+      constexpr uint32_t idesc256 = idesc_mn_mn(256);  // d = 128: M = 128 (Kw^T), N = 256
       bool ok = true;
       for (int t = 0; t < n_tiles && ok; ++t) {
         const int s = t % C::kStages;
@@ -195,20 +197,22 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         tc_fence_after();
         const uint32_t st = smem_u32(smem + s * C::kStageBytes);
         const uint32_t kw = smem_u32(sKw + j * C::kKwBytes);
-        const uint32_t k_addr = st, v_addr = st + C::kTileBytes;
+        const uint32_t k_addr = st;
 #pragma unroll
         for (int ks = 0; ks < kTok / 16; ++ks) {
           const uint32_t koff = ks * 16 * 128;
 #pragma unroll
           for (int part = 0; part < 2; ++part) {
             const uint32_t acc = (t > 0 || ks > 0 || part > 0) ? 1u : 0u;
-            const uint64_t bdesc = desc_mn_sw128(kw + part * C::kTileBytes + koff, kHalfBytes);
+            const uint64_t kwdesc = desc_mn_sw128(kw + part * C::kTileBytes + koff, kHalfBytes);
             if (D == 128) {
-              mma_ss(tmem, desc_mn_sw128(k_addr + koff, kHalfBytes), bdesc, idesc, acc);
-              mma_ss(tmem + 128, desc_mn_sw128(v_addr + koff, kHalfBytes), bdesc, idesc, acc);
+              // one N = 256 MMA: D[j][n] = sum_u Kw[u][j] [K | V][u][n] (the K and
+              // V tiles of a stage are adjacent, so their four 64-column atoms
+              // are one operand with a uniform atom stride)
+              mma_ss(tmem, kwdesc, desc_mn_sw128(k_addr + koff, kHalfBytes), idesc256, acc);
             } else {
               // [K^T; V^T]: the two 64-wide M blocks are the K and V tiles
-              mma_ss(tmem, desc_mn_sw128(k_addr + koff, C::kTileBytes), bdesc, idesc, acc);
+              mma_ss(tmem, desc_mn_sw128(k_addr + koff, C::kTileBytes), kwdesc, idesc, acc);
             }
           }
         }
@@ -233,47 +237,59 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       return text ? beta_t[((long long)b * l.T + tok) * l.H + h]
                   : beta[((long long)b * l.L() + row0 + tok) * l.H + h];
     };
-    float bnext = n_tiles > 0 ? beta_of(0) : 0.f;
+    // beta is a strided 4-byte read per token, a DRAM round trip per tile: the
+    // betas of the next kAhead tiles stay in flight in a register ring, so that
+    // no tile waits for its own (fetching one tile ahead left every tile a
+    // round trip long)
+    constexpr int kAhead = 8;
+    float bq[kAhead];
+#pragma unroll
+    for (int i = 0; i < kAhead; ++i) bq[i] = i < n_tiles ? beta_of(i) : 0.f;
     bool ok = true;
-    for (int t = 0; t < n_tiles && ok; ++t) {
-      const int s = t % C::kStages, use = t / C::kStages;
-      const int j = t % C::kKwSlots, juse = t / C::kKwSlots;
-      const float bu = bnext;
-      if (t + 1 < n_tiles) bnext = beta_of(t + 1);
-      if (!__all_sync(0xffffffffu, gwait(&bars->full[s], use & 1, abort))) {
-        ok = false;
-        break;
-      }
-      // the Kw slot is free once the MMAs of tile t - kKwSlots have completed
-      if (juse > 0 && !__all_sync(0xffffffffu, gwait(&bars->kw_empty[j], (juse - 1) & 1, abort))) {
-        ok = false;
-        break;
-      }
-      uint8_t* st = smem + s * C::kStageBytes;
-      uint8_t* kwp = sKw + j * C::kKwBytes;
+    for (int t0 = 0; t0 < n_tiles && ok; t0 += kAhead) {
 #pragma unroll
-      for (int cc = 0; cc < kCpt; ++cc) {
-        const int chunk = part * kCpt + cc;       // 0 .. D/8 - 1 within the row
-        const int hf = chunk / 8, c = chunk % 8;  // (swizzle permutes chunks within a row;
-                                                  //  the scaling does not care which)
-        const int off = hf * kHalfBytes + r * 128 + c * 16;
-        const uint4 x = *reinterpret_cast<const uint4*>(st + off);
-        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-        uint32_t hi4[4], lo4[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p0 = __uint_as_float(w[e] << 16) * bu;          // even element
-          const float p1 = __uint_as_float(w[e] & 0xFFFF0000u) * bu;  // odd element
-          const float h0 = __bfloat162float(__float2bfloat16_rn(p0));
-          const float h1 = __bfloat162float(__float2bfloat16_rn(p1));
-          hi4[e] = pack_bf16(h0, h1);
-          lo4[e] = pack_bf16(p0 - h0, p1 - h1);
+      for (int i = 0; i < kAhead; ++i) {
+        const int t = t0 + i;
+        if (t >= n_tiles || !ok) break;
+        const int s = t % C::kStages, use = t / C::kStages;
+        const int j = t % C::kKwSlots, juse = t / C::kKwSlots;
+        const float bu = bq[i];
+        bq[i] = t + kAhead < n_tiles ? beta_of(t + kAhead) : 0.f;
+        if (!__all_sync(0xffffffffu, gwait(&bars->full[s], use & 1, abort))) {
+          ok = false;
+          break;
         }
-        *reinterpret_cast<uint4*>(kwp + off) = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
-        *reinterpret_cast<uint4*>(kwp + C::kTileBytes + off) = make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
+        // the Kw slot is free once the MMAs of tile t - kKwSlots have completed
+        if (juse > 0 && !__all_sync(0xffffffffu, gwait(&bars->kw_empty[j], (juse - 1) & 1, abort))) {
+          ok = false;
+          break;
+        }
+        uint8_t* st = smem + s * C::kStageBytes;
+        uint8_t* kwp = sKw + j * C::kKwBytes;
+#pragma unroll
+        for (int cc = 0; cc < kCpt; ++cc) {
+          const int chunk = part * kCpt + cc;       // 0 .. D/8 - 1 within the row
+          const int hf = chunk / 8, c = chunk % 8;  // (swizzle permutes chunks within a row;
+                                                    //  the scaling does not care which)
+          const int off = hf * kHalfBytes + r * 128 + c * 16;
+          const uint4 x = *reinterpret_cast<const uint4*>(st + off);
+          const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+          uint32_t hi4[4], lo4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float p0 = __uint_as_float(w[e] << 16) * bu;          // even element
+            const float p1 = __uint_as_float(w[e] & 0xFFFF0000u) * bu;  // odd element
+            const float h0 = __bfloat162float(__float2bfloat16_rn(p0));
+            const float h1 = __bfloat162float(__float2bfloat16_rn(p1));
+            hi4[e] = pack_bf16(h0, h1);
+            lo4[e] = pack_bf16(p0 - h0, p1 - h1);
+          }
+          *reinterpret_cast<uint4*>(kwp + off) = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
+          *reinterpret_cast<uint4*>(kwp + C::kTileBytes + off) = make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive(&bars->kw_full[j]);
       }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive(&bars->kw_full[j]);
     }
     if (ok) ok = __all_sync(0xffffffffu, gwait(&bars->done, 0, abort));
     if (ok) {
@@ -288,13 +304,11 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       float* as = reinterpret_cast<float*>(smem);
       float* arow;
-      float* brow;
+      float* bcol = bw + slot * D * D + m;  // d = 128: column m of B_f
       if (D == 128) {
         arow = as + m * C::kAStride;
-        brow = bw + slot * D * D + (long long)m * D;
       } else {
         arow = (m < 64) ? as + m * C::kAStride : bw + slot * D * D + (long long)(m - 64) * D;
-        brow = nullptr;
       }
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
@@ -311,11 +325,10 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t r[32];
           tmem_ld_x32(taddr + 128 + c0, r);
-          float4* dst = reinterpret_cast<float4*>(brow + c0);
+          // lane m holds column m of B_f (rows c0 .. c0 + 31): each store of the
+          // warp is one 128-byte row segment
 #pragma unroll
-          for (int i = 0; i < 8 && slot_ok; ++i)
-            dst[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                 __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+          for (int i = 0; i < 32 && slot_ok; ++i) bcol[(long long)(c0 + i) * D] = __uint_as_float(r[i]);
         }
       }
     }
