@@ -135,7 +135,9 @@ int vdn_hybrid_attn_fwd(const vdn_layout_t* layout, int dtype,
  * given, a host array of d floats). The call copies in, computes and copies
  * the output back, in chunks of head_chunk heads (<= 0: about ten chunks)
  * pipelined on three internal streams so that the copies of one chunk overlap
- * the kernels of the next; the heads are independent, so the result equals
+ * the kernels of the next (a chunk's k, v and beta are copied first, then q,
+ * then the gates, and its kernels start as their own inputs arrive); the heads
+ * are independent, so the result equals
  * vdn_hybrid_attn_fwd's bit for bit. Host memory should be pinned
  * (cudaHostAlloc / cudaHostRegister) for the copies to overlap. workspace:
  * device memory of vdn_hybrid_host_workspace_bytes bytes (two chunk buffers).

@@ -9,6 +9,10 @@
 // compute, out) with two device buffers, so that chunk i + 1 is copied in and
 // chunk i - 1 copied out while chunk i computes. PCIe carries both directions
 // at once; with pinned host memory the copies then hide under the kernels.
+// A chunk's inputs arrive in the order its kernels need them: k, v and beta
+// (the linear branch starts), then q (the window softmax), then the gates (the
+// combine), each group with its own event, so that a chunk's kernels start
+// before its last bytes have crossed PCIe.
 #include <cstdint>
 #include <mutex>
 
@@ -16,7 +20,7 @@
 
 namespace {
 
-// The pipeline's three streams and six events, created on the first call on a
+// The pipeline's three streams and ten events, created on the first call on a
 // device and kept for the life of the process (creating and destroying them on
 // every call costs driver round trips per call). The call is synchronous, so
 // one call at a time uses them: concurrent calls on one device take turns.
@@ -24,8 +28,8 @@ struct Pipeline {
   std::mutex mu;
   bool ready = false;
   cudaStream_t s_in = nullptr, s_comp = nullptr, s_out = nullptr;
-  cudaEvent_t ev_in[2] = {nullptr, nullptr}, ev_comp[2] = {nullptr, nullptr},
-              ev_out[2] = {nullptr, nullptr};
+  cudaEvent_t ev_in[2] = {nullptr, nullptr}, ev_q[2] = {nullptr, nullptr}, ev_g[2] = {nullptr, nullptr},
+              ev_comp[2] = {nullptr, nullptr}, ev_out[2] = {nullptr, nullptr};
 };
 constexpr int kMaxDevicesH = 64;
 Pipeline g_pipe[kMaxDevicesH];
@@ -41,6 +45,8 @@ cudaError_t pipeline_init(Pipeline& p) {
   ok(cudaStreamCreateWithFlags(&p.s_out, cudaStreamNonBlocking));
   for (int i = 0; i < 2; ++i) {
     ok(cudaEventCreateWithFlags(&p.ev_in[i], cudaEventDisableTiming));
+    ok(cudaEventCreateWithFlags(&p.ev_q[i], cudaEventDisableTiming));
+    ok(cudaEventCreateWithFlags(&p.ev_g[i], cudaEventDisableTiming));
     ok(cudaEventCreateWithFlags(&p.ev_comp[i], cudaEventDisableTiming));
     ok(cudaEventCreateWithFlags(&p.ev_out[i], cudaEventDisableTiming));
   }
@@ -194,6 +200,8 @@ int vdn_hybrid_attn_fwd_host(const vdn_layout_t* layout, int dtype, int head_chu
   if (status != VDN_OK) return status;
   cudaStream_t s_in = pipe.s_in, s_comp = pipe.s_comp, s_out = pipe.s_out;
   cudaEvent_t* ev_in = pipe.ev_in;
+  cudaEvent_t* ev_q = pipe.ev_q;
+  cudaEvent_t* ev_g = pipe.ev_g;
   cudaEvent_t* ev_comp = pipe.ev_comp;
   cudaEvent_t* ev_out = pipe.ev_out;
   auto fail = [&](cudaError_t e) {
@@ -213,11 +221,10 @@ int vdn_hybrid_attn_fwd_host(const vdn_layout_t* layout, int dtype, int head_chu
     if (c >= 2) fail(cudaStreamWaitEvent(s_in, ev_out[slot], 0));
     const size_t w_vid = (size_t)hc * d * es, p_vid = (size_t)H * d * es, o_vid = (size_t)h0 * d * es;
     const size_t rows_v = (size_t)B * L, rows_t = (size_t)B * T;
-    const char* src[5] = {static_cast<const char*>(q), static_cast<const char*>(k),
-                          static_cast<const char*>(v), static_cast<const char*>(g_soft),
-                          static_cast<const char*>(g_lin)};
-    char* dst[5] = {buf.q, buf.k, buf.v, buf.gs, buf.gl};
-    for (int t = 0; t < 5; ++t) fail(copy_in(dst[t], src[t] + o_vid, w_vid, p_vid, rows_v, s_in));
+    const char* vsrc = static_cast<const char*>(v);
+    // the linear branch's inputs: k, v, the text, beta
+    fail(copy_in(buf.k, static_cast<const char*>(k) + o_vid, w_vid, p_vid, rows_v, s_in));
+    fail(copy_in(buf.v, vsrc + o_vid, w_vid, p_vid, rows_v, s_in));
     if (T > 0) {
       fail(copy_in(buf.kt, static_cast<const char*>(k_text) + o_vid, w_vid, p_vid, rows_t, s_in));
       fail(copy_in(buf.vt, static_cast<const char*>(v_text) + o_vid, w_vid, p_vid, rows_t, s_in));
@@ -225,14 +232,20 @@ int vdn_hybrid_attn_fwd_host(const vdn_layout_t* layout, int dtype, int head_chu
     }
     fail(copy_in(buf.beta, beta + h0, (size_t)hc * 4, (size_t)H * 4, rows_v, s_in));
     fail(cudaEventRecord(ev_in[slot], s_in));
+    // then q (the window softmax), then the gates (the combine)
+    fail(copy_in(buf.q, static_cast<const char*>(q) + o_vid, w_vid, p_vid, rows_v, s_in));
+    fail(cudaEventRecord(ev_q[slot], s_in));
+    fail(copy_in(buf.gs, static_cast<const char*>(g_soft) + o_vid, w_vid, p_vid, rows_v, s_in));
+    fail(copy_in(buf.gl, static_cast<const char*>(g_lin) + o_vid, w_vid, p_vid, rows_v, s_in));
+    fail(cudaEventRecord(ev_g[slot], s_in));
     if (status != VDN_OK) break;
-    // compute
+    // compute: the linear branch once k, v and beta are in, the window once q is
     fail(cudaStreamWaitEvent(s_comp, ev_in[slot], 0));
     const vdn_layout_t* lcp = &lc;
-    const int s = vdn_hybrid_attn_fwd(lcp, dtype, buf.q, buf.k, buf.v, T ? buf.kt : nullptr,
-                                      T ? buf.vt : nullptr, buf.beta, T ? buf.beta_t : nullptr, buf.gs,
-                                      buf.gl, rms_w_dev, rms_eps, buf.out, nullptr, nullptr, buf.ws,
-                                      vdn_workspace_bytes(lcp, dtype), s_comp);
+    const int s = vdn::hybrid_staged(lcp, dtype, buf.q, buf.k, buf.v, T ? buf.kt : nullptr,
+                                     T ? buf.vt : nullptr, buf.beta, T ? buf.beta_t : nullptr, buf.gs,
+                                     buf.gl, rms_w_dev, rms_eps, buf.out, buf.ws,
+                                     vdn_workspace_bytes(lcp, dtype), s_comp, ev_q[slot], ev_g[slot]);
     if (s != VDN_OK) { status = s; break; }
     fail(cudaEventRecord(ev_comp[slot], s_comp));
     // copy out into the strided host tensor

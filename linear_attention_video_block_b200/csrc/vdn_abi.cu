@@ -207,7 +207,8 @@ int hybrid_impl(const vdn_layout_t* layout, int dtype, const vdn_context_t* ctx,
                 const float* beta, const float* beta_text, const float* alpha, const void* g_soft,
                 const void* g_lin, const float* rms_weight, float rms_eps, void* out,
                 void* out_soft, void* out_lin, void* workspace, size_t workspace_bytes,
-                cudaStream_t stream) {
+                cudaStream_t stream, cudaEvent_t before_window = nullptr,
+                cudaEvent_t before_combine = nullptr) {
   if (!layout_ok(layout)) return VDN_ERR_INVALID;
   if (!dtype_d_ok(dtype, layout->d)) return VDN_ERR_UNSUPPORTED;
   if (!q || !k || !v || !beta || !g_soft || !g_lin || !out) return VDN_ERR_INVALID;
@@ -234,8 +235,16 @@ int hybrid_impl(const vdn_layout_t* layout, int dtype, const vdn_context_t* ctx,
   int s = cuda_status(vdn::launch_vda_states(l, dtype, k, v, kt, vt, beta, bt, alpha, w.am, w.bw,
                                              w.states, stream));
   if (s != VDN_OK) return s;
+  if (before_window) {
+    s = cuda_status(cudaStreamWaitEvent(stream, before_window, 0));
+    if (s != VDN_OK) return s;
+  }
   s = run_window(ls, dtype, q, k, v, kt, vt, w.o_soft, true, nullptr, ja, stream);
   if (s != VDN_OK) return s;
+  if (before_combine) {
+    s = cuda_status(cudaStreamWaitEvent(stream, before_combine, 0));
+    if (s != VDN_OK) return s;
+  }
   if (tc)
     return cuda_status(vdn::launch_combine_tc(l, q, w.states, w.o_soft, g_soft, g_lin, rms_weight,
                                               rms_eps, out, out_soft, out_lin, stream));
@@ -244,6 +253,20 @@ int hybrid_impl(const vdn_layout_t* layout, int dtype, const vdn_context_t* ctx,
 }
 
 }  // namespace
+
+namespace vdn {
+
+int hybrid_staged(const vdn_layout_t* layout, int dtype, const void* q, const void* k, const void* v,
+                  const void* k_text, const void* v_text, const float* beta, const float* beta_text,
+                  const void* g_soft, const void* g_lin, const float* rms_weight, float rms_eps, void* out,
+                  void* workspace, size_t workspace_bytes, cudaStream_t stream, cudaEvent_t before_window,
+                  cudaEvent_t before_combine) {
+  return hybrid_impl(layout, dtype, nullptr, q, k, v, k_text, v_text, beta, beta_text, nullptr, g_soft,
+                     g_lin, rms_weight, rms_eps, out, nullptr, nullptr, workspace, workspace_bytes, stream,
+                     before_window, before_combine);
+}
+
+}  // namespace vdn
 
 extern "C" {
 

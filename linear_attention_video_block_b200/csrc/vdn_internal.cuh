@@ -68,6 +68,16 @@ inline Layout to_layout(const vdn_layout_t* l) {
 // last CUDA error (vdn_last_cuda_error) and returns VDN_ERR_CUDA.
 int cuda_status(cudaError_t e);
 
+// vdn_hybrid_attn_fwd with two waits on the stream: before_window (the
+// softmax branch's inputs q, k, v) and before_combine (the gates), so that a
+// caller streaming its inputs in can start the linear branch once k, v and
+// beta have arrived. Either event may be null.
+int hybrid_staged(const vdn_layout_t* layout, int dtype, const void* q, const void* k, const void* v,
+                  const void* k_text, const void* v_text, const float* beta, const float* beta_text,
+                  const void* g_soft, const void* g_lin, const float* rms_weight, float rms_eps, void* out,
+                  void* workspace, size_t workspace_bytes, cudaStream_t stream, cudaEvent_t before_window,
+                  cudaEvent_t before_combine);
+
 // Bound checks of the checked build (-DVDN_BOUND_CHECKS): VDN_IN_BOUNDS(cond,
 // status) is true when cond holds; otherwise it records VDN_ERR_BOUNDS in the
 // device status word *status and is false, and the caller skips the access
