@@ -26,7 +26,8 @@
 //
 // Epilogue: B_f goes to global memory; A_f is staged in the freed shared rings
 // and all 256 threads (warps 6-7 join here) invert I + A_f in place with the
-// register-blocked Gauss-Jordan of spd_inverse.cuh, writing M_f = (I + A_f)^-1
+// register-blocked Gauss-Jordan of spd_inverse.cuh (two pivots per barrier,
+// packed f32x2 updates), writing M_f = (I + A_f)^-1
 // to the am slot. The inverse is a latency-bound chain of d dependent pivots;
 // done here, it overlaps the other CTA of the SM streaming its frame instead
 // of running as a separate launch after every Gram has finished.
@@ -66,7 +67,7 @@ struct GCfg {
   // (row stride kAStride floats, padded against bank conflicts) for the inverse,
   // followed by the inverse's pivot row / column buffers
   static constexpr int kAStride = D + 4;
-  static_assert(D * kAStride * 4 + 4 * D * 4 <= kStages * kStageBytes + kKwSlots * kKwBytes,
+  static_assert(D * kAStride * 4 + 8 * D * 4 <= kStages * kStageBytes + kKwSlots * kKwBytes,
                 "the inverse's staging must fit in the freed rings");
 };
 
@@ -348,8 +349,8 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
   {
     constexpr int RA = D / 16;
     const float* as = reinterpret_cast<const float*>(smem);
-    float (*rowk)[D] = reinterpret_cast<float (*)[D]>(smem + D * C::kAStride * 4);
-    float (*colk)[D] = rowk + 2;
+    float (*rowk)[2][D] = reinterpret_cast<float (*)[2][D]>(smem + D * C::kAStride * 4);
+    float (*colk)[2][D] = rowk + 2;
     const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
     float a[RA][RA];
 #pragma unroll
@@ -359,7 +360,7 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         const int i = tr + 16 * x, j = tc + 16 * y;
         a[x][y] = as[i * C::kAStride + j] + (i == j ? 1.f : 0.f);
       }
-    spd_inverse_blocks<D>(a, tr, tc, rowk, colk);
+    spd_inverse_blocks2x<D>(a, tr, tc, rowk, colk);
     const long long slot = ((long long)b * l.H + h) * l.F + f;
     if (!VDN_IN_BOUNDS(f >= 0 && f < l.F && h < l.H && b < l.B, &g_gram_status)) return;
     float* g = am + slot * D * D;
