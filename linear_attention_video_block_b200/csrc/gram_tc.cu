@@ -3,18 +3,18 @@
 //   A_f = K_f^T Diag(beta_f) K_f,   B_f = V_f^T Diag(beta_f) K_f
 // over the U tokens of one frame (or of the text, slot 0), fp32 results.
 //
-// CTA = one (b, h, slot); 192 threads:
+// CTA = one (b, h, slot); 256 threads:
 //   warp 0     TMA producer: 32-token K and V tiles into a ring of stages
 //   warp 1     MMA issuer (one lane) and TMEM owner
-//   warps 2-5  scalers: write Kw = beta (.) K into a ring of two Kw slots
+//   warps 2-7  scalers: write Kw = beta (.) K into a ring of two Kw slots
 //              (separate from the K/V ring, so that more K/V tiles are in
 //              flight in the same shared memory) as two bf16 parts,
 //              Kw_hi = bf16(beta k) and Kw_lo = bf16(beta k - Kw_hi), so that the
 //              products keep ~16 significant bits of beta k (a single bf16 copy
-//              put the chunk states 1e-2 off); four threads per token row, beta
-//              fetched one tile ahead, beta = 0
-//              past the frame (which also masks the ragged last tile); then the
-//              epilogue reads A and B out of TMEM.
+//              put the chunk states 1e-2 off); six threads per token row, the
+//              betas of the next tiles in flight in a register ring, beta = 0
+//              past the frame (which also masks the ragged last tile); then
+//              warps 2-5 read A and B out of TMEM.
 // Both MMA operands are MN-major (token = K dimension, contiguous along d):
 //   d = 128: one M = 128, N = 256 MMA per Kw part (hi, lo) and 16 tokens,
 //            D[j][n] += sum_u Kw[u][j] [K | V][u][n]: columns 0..127 hold
@@ -25,7 +25,7 @@
 // The work is HBM-bound: each token's k and v are read once.
 //
 // Epilogue: B_f goes to global memory; A_f is staged in the freed shared rings
-// and all 256 threads (warps 6-7 join here) invert I + A_f in place with the
+// and all 256 threads invert I + A_f in place with the
 // register-blocked Gauss-Jordan of spd_inverse.cuh (two pivots per barrier,
 // packed f32x2 updates), writing M_f = (I + A_f)^-1
 // to the am slot. The inverse is a latency-bound chain of d dependent pivots;
@@ -50,7 +50,8 @@ cudaError_t read_and_clear_gram_status(int* status) {
 namespace {
 
 constexpr int kTok = 32;        // tokens per tile (96 KB of stages: two CTAs per SM)
-constexpr int kThreads = 256;  // warps 6-7 join only the in-place inverse
+constexpr int kThreads = 256;
+constexpr int kScalers = 192;  // warps 2-7 scale beta k; warps 2-5 also drain TMEM
 constexpr int kHalfBytes = kTok * 128;  // kTok tokens x 64 bf16 (one swizzle atom column)
 
 template <int D>
@@ -142,7 +143,7 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       mbar_init(&bars->empty[s], 1);
     }
     for (int j = 0; j < C::kKwSlots; ++j) {
-      mbar_init(&bars->kw_full[j], 128);
+      mbar_init(&bars->kw_full[j], kScalers);
       mbar_init(&bars->kw_empty[j], 1);
     }
     mbar_init(&bars->done, 1);
@@ -233,14 +234,17 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
       tc_commit(&bars->done);
       if (!ok) gwait(&bars->done, 0, abort, false);
     }
-  } else if (warp < 6) {
+  } else {
     // ---------------------------------------------------- scalers / epilogue
-    // 4 threads per token row, each scaling (D / 8) / 4 of the row's 16-byte chunks;
-    // beta of the next tile is fetched one tile ahead (it is a strided 4-byte read)
+    // 6 threads per token row, each scaling chunks [c_lo, c_hi) of the row's
+    // D / 8 16-byte chunks (at most 3)
     const int u = threadIdx.x - 64;
-    constexpr int kTpr = 128 / kTok;              // threads per token row
-    constexpr int kCpt = (D / 8) / kTpr;          // 16-byte chunks per thread
+    constexpr int kTpr = kScalers / kTok;         // threads per token row
+    constexpr int kChunks = D / 8;                // 16-byte chunks per row
+    constexpr int kCpt = (kChunks + kTpr - 1) / kTpr;
+    static_assert(kTpr * kTok == kScalers, "scaler threads cover the tile's rows");
     const int r = u / kTpr, part = u % kTpr;
+    const int c_lo = part * kChunks / kTpr, c_hi = (part + 1) * kChunks / kTpr;
     auto beta_of = [&](int t) -> float {
       const int tok = t * kTok + r;
       if (tok >= U) return 0.f;
@@ -280,7 +284,8 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         uint8_t* kwp = sKw + j * C::kKwBytes;
 #pragma unroll
         for (int cc = 0; cc < kCpt; ++cc) {
-          const int chunk = part * kCpt + cc;       // 0 .. D/8 - 1 within the row
+          const int chunk = c_lo + cc;              // 0 .. D/8 - 1 within the row
+          if (chunk >= c_hi) break;
           const int hf = chunk / 8, c = chunk % 8;  // (swizzle permutes chunks within a row;
                                                     //  the scaling does not care which)
           const int off = hf * kHalfBytes + r * 128 + c * 16;
@@ -310,8 +315,9 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         mbar_arrive(&bars->kw_full[j]);
       }
     }
-    if (ok) ok = __all_sync(0xffffffffu, gwait(&bars->done, 0, abort));
-    if (ok) {
+    // warps 2-5 drain TMEM (warp w reaches lanes 32 (w mod 4) .. + 31)
+    if (warp < 6 && ok) ok = __all_sync(0xffffffffu, gwait(&bars->done, 0, abort));
+    if (warp < 6 && ok) {
       tc_fence_after();
       const int m = 32 * (warp & 3) + lane;  // TMEM lane = output row
       const uint32_t taddr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
