@@ -107,9 +107,8 @@ struct GramSlots {
   }
 };
 
-// Packed fp32 pairs (sm_100 f32x2 arithmetic) for the beta k split.
-__device__ __forceinline__ unsigned long long sp_pack(float lo, float hi) { return spd_pack(lo, hi); }
-__device__ __forceinline__ void sp_unpack(unsigned long long p, float& lo, float& hi) { spd_unpack(p, lo, hi); }
+// Packed fp32 multiply (sm_100 f32x2 arithmetic) for the beta k split; the
+// pack, unpack and fma helpers come from spd_inverse.cuh.
 __device__ __forceinline__ unsigned long long sp_mul2(unsigned long long a, unsigned long long b) {
   unsigned long long r;
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
@@ -269,7 +268,7 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         const int s = t % C::kStages, use = t / C::kStages;
         const int j = t % C::kKwSlots, juse = t / C::kKwSlots;
         const float bu = bq[i];
-        const unsigned long long bu2 = sp_pack(bu, bu);
+        const unsigned long long bu2 = spd_pack(bu, bu);
         bq[i] = t + kAhead < n_tiles ? beta_of(t + kAhead) : 0.f;
         if (!__all_sync(0xffffffffu, gwait(&bars->full[s], use & 1, abort))) {
           ok = false;
@@ -298,14 +297,14 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
             // beta in one packed multiply; hi = bf16(beta k); lo = bf16(beta k - hi)
             // with the exact difference from one packed fma with -1
             const unsigned long long p2 =
-                sp_mul2(sp_pack(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u)), bu2);
+                sp_mul2(spd_pack(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u)), bu2);
             float p0, p1;
-            sp_unpack(p2, p0, p1);
+            spd_unpack(p2, p0, p1);
             hi4[e] = pack_bf16(p0, p1);
             const unsigned long long h2 =
-                sp_pack(__uint_as_float(hi4[e] << 16), __uint_as_float(hi4[e] & 0xFFFF0000u));
+                spd_pack(__uint_as_float(hi4[e] << 16), __uint_as_float(hi4[e] & 0xFFFF0000u));
             float l0, l1;
-            sp_unpack(spd_fma2(h2, kMinusOne2, p2), l0, l1);
+            spd_unpack(spd_fma2(h2, kMinusOne2, p2), l0, l1);
             lo4[e] = pack_bf16(l0, l1);
           }
           *reinterpret_cast<uint4*>(kwp + off) = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);

@@ -221,10 +221,9 @@ int vdn_hybrid_attn_fwd_host(const vdn_layout_t* layout, int dtype, int head_chu
     if (c >= 2) fail(cudaStreamWaitEvent(s_in, ev_out[slot], 0));
     const size_t w_vid = (size_t)hc * d * es, p_vid = (size_t)H * d * es, o_vid = (size_t)h0 * d * es;
     const size_t rows_v = (size_t)B * L, rows_t = (size_t)B * T;
-    const char* vsrc = static_cast<const char*>(v);
     // the linear branch's inputs: k, v, the text, beta
     fail(copy_in(buf.k, static_cast<const char*>(k) + o_vid, w_vid, p_vid, rows_v, s_in));
-    fail(copy_in(buf.v, vsrc + o_vid, w_vid, p_vid, rows_v, s_in));
+    fail(copy_in(buf.v, static_cast<const char*>(v) + o_vid, w_vid, p_vid, rows_v, s_in));
     if (T > 0) {
       fail(copy_in(buf.kt, static_cast<const char*>(k_text) + o_vid, w_vid, p_vid, rows_t, s_in));
       fail(copy_in(buf.vt, static_cast<const char*>(v_text) + o_vid, w_vid, p_vid, rows_t, s_in));
