@@ -11,13 +11,15 @@
 //   warps 2-9  stage S_sum = S_fwd + S_rev once as two bf16 K-major operands
 //              (S_hi = bf16(S_sum), S_lo = bf16(S_sum - S_hi)); then warpgroup
 //              2-5 drains the accumulator of the even tiles and warpgroup 6-9
-//              that of the odd tiles to global memory (one row per thread), so
-//              that two tiles' worth of loads and stores are in flight
+//              that of the odd tiles, so that two tiles' worth of loads and
+//              stores are in flight; each warp passes its 32 TMEM rows through
+//              a 16-row shared-memory staging and writes one contiguous row per
+//              warp access
 // Boundary-frame groups write zeros. HBM-bound: q is read once, o_lin written once
 // (bf16, or float32 for the branch-specialised split's exchange).
 //
 // Combine variant (project page, "Gating the Softmax and Linear Branch
-// Outputs"): instead of o_lin, each drain thread finishes its row of the hybrid
+// Outputs"): instead of o_lin, the drain warps finish the rows of the hybrid
 // output, out = sigmoid(g_s) o_soft + sigmoid(g_l) RMSNorm(o_lin), from the
 // float32 softmax-branch output of the window kernel and the two gates
 // (boundary frames: out = sigmoid(g_s) o_soft); optionally the two gated
