@@ -194,7 +194,6 @@ scan_kernel(Layout l, int fwd_max, int rev_min, int has_text, const float* __res
   using C = ScanCfg<D>;
   constexpr int R = C::kR, RR = C::kRR, CH = C::kChunk, NCH = D / CH;
   __shared__ __align__(16) float ring[C::kRing][CH * D];
-  __shared__ __align__(16) float brows[R * D];
   __shared__ __align__(16) float x[R * D];
   const int tid = threadIdx.x;
   const int cg = tid % C::kCG, rg = tid / C::kCG;
@@ -355,7 +354,7 @@ cudaError_t launch_states_t(const Layout& l, int dtype, const void* k, const voi
     }
   }
   {
-    dim3 grid(D / 16, 2, l.B * l.H);
+    dim3 grid(D / ScanCfg<D>::kR, 2, l.B * l.H);
     scan_kernel<D><<<grid, ScanCfg<D>::kThreads, 0, st>>>(l, fwd_max, rev_min, map.has_text, am, bw, alpha, states);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
